@@ -1,0 +1,277 @@
+"""Plain, slow CPU oracle of the ISPA warmup path, in float64 NumPy. TEST INFRASTRUCTURE.
+
+Only the tests, the smoke check and the benchmark's CPU-baseline leg use this module; the
+product path never imports it, and it imports nothing from the product package.
+
+Source: "Towards Memory-Efficient Autoregressive Video Generation via Instance-Specific
+Parametric Absorption" (ISPA), paper text (paperpeel.com/paper/2607.00712), cited below as
+[ISPA §x]; and the reading notes at paper.gecl.asia (arxiv-cs-cv-2607-00712, section
+"Method"), cited as [notes: Method]. The paper's equations were lost from every page;
+where a step is open, the plainest reading is taken and named "Reading" below.
+
+What is computed (per layer, per warmup chunk, then once at the transition):
+
+1. Attention over the layer's KV cache, split into two partitions [ISPA §3.1 step 1]:
+   the local partition = sink frame rows + current-chunk rows, and the history partition =
+   every other cached row. A_full attends to all rows, A_loc to the local rows, A_hist to
+   the history rows, each a plain softmax over its own mask (scale 1/sqrt(head_dim)), with
+   its log-sum-exp. No causal mask inside the chunk (Reading: the chunk is denoised
+   jointly), no positional rotation (Q/K are taken as already positioned).
+2. Statistics for the closed-form absorption [ISPA §3.2; notes: Method, "ridge
+   regression" on the attention output projection]: R = A_full - A_loc and, summed over the
+   warmup chunks, G = A_loc^T A_loc, C = A_loc^T R, H = R^T R (row count kept too).
+   Reading (bf16 workloads): A_loc and R are rounded to bf16 before the products, because
+   the GPU feeds them to the tensor cores in bf16; the sums stay in float64 here.
+3. Absorption [ISPA §3.1 step 2, §3.2, §4.1 "Eq. 5", lambda]: the update of the output
+   projection minimises sum_t ||A_loc,t (W + dW) - A_full,t W||^2 + lambda ||dW||^2, so
+   (G + lambda I) dW = C W. Solved here with a dense LU solve (numpy.linalg.solve), not
+   with a Cholesky factorisation, so that it shares no algorithm with the GPU.
+4. Reconstruction error [ISPA §3.3]. Reading: eps = E^2 / T^2, the relative squared error
+   of the reconstructed projected output over the warmup, from traces:
+   E^2 = tr(dW^T G dW) - 2 tr(dW^T C W) + tr(W^T H W)  (= ||A_loc (W+dW) - A_full W||^2)
+   T^2 = tr(W^T (G + C + C^T + H) W)                   (= ||A_full W||^2)
+   eps = 0 when T^2 = 0.
+5. Selection [ISPA §3.3]: rank layers by eps ascending (ties by the lower layer index,
+   NaN ranks last); the first K become L-layers with W_new = W + dW [ISPA §3.1 step 3].
+6. After the switch an L-layer attends to the sink + chunk rows only and projects with
+   W_new [ISPA §3.1 step 3, §3.3].
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+NEG_INF = -np.inf
+
+
+# --------------------------------------------------------------------------------------
+# bf16 rounding (round to nearest, ties to even) of float64 values, directly from the
+# definition: a bf16 number carries 8 significant bits.
+# --------------------------------------------------------------------------------------
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bf16 value (ties to even), returned as float64.
+    Values are assumed to lie in bf16's normal range (true for every tensor here)."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                # x = m * 2**e, 0.5 <= |m| < 1
+    m = np.rint(m * 256.0) / 256.0    # 8 significant bits; rint rounds half to even
+    return np.ldexp(m, e)
+
+
+# --------------------------------------------------------------------------------------
+# Step 1: attention over explicit masks [ISPA §3.1 step 1, §3.4].
+# --------------------------------------------------------------------------------------
+def partition_masks(n_kv: int, sink: Tuple[int, int], chunk: Tuple[int, int]):
+    """Boolean masks over the KV rows: full, local (sink + chunk) and history (the rest)."""
+    full = np.ones(n_kv, dtype=bool)
+    local = np.zeros(n_kv, dtype=bool)
+    local[sink[0]:sink[1]] = True
+    local[chunk[0]:chunk[1]] = True
+    hist = ~local
+    return full, local, hist
+
+
+def masked_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask: np.ndarray, scale: float):
+    """Softmax attention restricted to the KV rows where `mask` is True.
+
+    q [n_q, h, d], k/v [n_kv, h, d] -> A [n_q, h, d] (float64), lse [h, n_q] (natural log of
+    the sum of exp(scale * q.k) over the masked rows). An empty mask gives A = 0, lse = -inf.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    n_q, h, d = q.shape
+    A = np.zeros((n_q, h, d), dtype=np.float64)
+    lse = np.full((h, n_q), NEG_INF, dtype=np.float64)
+    if not mask.any():
+        return A, lse
+    km = k[mask]
+    vm = v[mask]
+    for head in range(h):
+        S = scale * (q[:, head, :] @ km[:, head, :].T)          # [n_q, n_mask]
+        m = S.max(axis=1, keepdims=True)
+        P = np.exp(S - m)
+        l = P.sum(axis=1, keepdims=True)
+        A[:, head, :] = (P @ vm[:, head, :]) / l
+        lse[head] = (m + np.log(l))[:, 0]
+    return A, lse
+
+
+def split_attention(q, k, v, sink: Tuple[int, int], chunk: Tuple[int, int], scale: float) -> Dict[str, np.ndarray]:
+    """A_full, A_loc and A_hist (with their log-sum-exps), each from its own mask."""
+    full, local, hist = partition_masks(k.shape[0], sink, chunk)
+    A_full, lse_full = masked_attention(q, k, v, full, scale)
+    A_loc, lse_loc = masked_attention(q, k, v, local, scale)
+    A_hist, lse_hist = masked_attention(q, k, v, hist, scale)
+    return dict(A_full=A_full, lse_full=lse_full, A_loc=A_loc, lse_loc=lse_loc,
+                A_hist=A_hist, lse_hist=lse_hist)
+
+
+def lse_merge(A1, lse1, A2, lse2):
+    """Decomposable attention [ISPA §3.4, "Online Softmax"]: combine the outputs of two
+    disjoint key partitions into the output over their union.
+    A, lse in the layouts of masked_attention. lse = log(e^lse1 + e^lse2); each partition
+    is weighted by e^(lse_i - lse)."""
+    lse = np.logaddexp(lse1, lse2)                               # [h, n_q]
+    with np.errstate(invalid="ignore"):
+        w1 = np.where(np.isneginf(lse1), 0.0, np.exp(lse1 - lse))
+        w2 = np.where(np.isneginf(lse2), 0.0, np.exp(lse2 - lse))
+    w1 = w1.T[:, :, None]                                        # [n_q, h, 1]
+    w2 = w2.T[:, :, None]
+    return w1 * A1 + w2 * A2, lse
+
+
+def local_attention(q, k_loc, v_loc, scale: float):
+    """L-layer attention after the switch: all given rows are local (sink + chunk)."""
+    return masked_attention(q, k_loc, v_loc, np.ones(k_loc.shape[0], dtype=bool), scale)
+
+
+# --------------------------------------------------------------------------------------
+# Step 2: statistics [ISPA §3.2; notes: Method].
+# --------------------------------------------------------------------------------------
+def stats_init(D: int) -> Dict[str, np.ndarray]:
+    return dict(G=np.zeros((D, D)), C=np.zeros((D, D)), H=np.zeros((D, D)), rows=0)
+
+
+def stats_operands(A_loc: np.ndarray, A_full: np.ndarray, dtype: str):
+    """Rows of A_loc and R = A_full - A_loc as [n, D] matrices (column h*d + j), rounded
+    to bf16 in bf16 mode."""
+    n = A_loc.shape[0]
+    a = np.asarray(A_loc, dtype=np.float64).reshape(n, -1)
+    r = np.asarray(A_full, dtype=np.float64).reshape(n, -1) - a
+    if dtype == "bf16":
+        a = bf16_round(a)
+        r = bf16_round(r)
+    return a, r
+
+
+def stats_update(stats: Dict[str, np.ndarray], A_loc: np.ndarray, A_full: np.ndarray, dtype: str) -> None:
+    """G += A_loc^T A_loc, C += A_loc^T R, H += R^T R, rows += n."""
+    a, r = stats_operands(A_loc, A_full, dtype)
+    stats["G"] += a.T @ a
+    stats["C"] += a.T @ r
+    stats["H"] += r.T @ r
+    stats["rows"] += a.shape[0]
+
+
+# --------------------------------------------------------------------------------------
+# Steps 3-5: absorption, error, selection [ISPA §3.1-§3.3, §4.1].
+# --------------------------------------------------------------------------------------
+def absorb_solve(G: np.ndarray, C: np.ndarray, W: np.ndarray, lam: float) -> np.ndarray:
+    """dW solving (G + lambda I) dW = C W (ridge normal equations), dense LU solve."""
+    D = G.shape[0]
+    M = np.asarray(G, dtype=np.float64) + lam * np.eye(D)
+    return np.linalg.solve(M, np.asarray(C, dtype=np.float64) @ np.asarray(W, dtype=np.float64))
+
+
+def reconstruction_error(G, C, H, W, dW) -> Dict[str, float]:
+    """eps = E^2 / T^2 from the traces listed in the module docstring."""
+    G = np.asarray(G, np.float64); C = np.asarray(C, np.float64); H = np.asarray(H, np.float64)
+    W = np.asarray(W, np.float64); dW = np.asarray(dW, np.float64)
+    CW = C @ W
+    t_dgd = float(np.sum(dW * (G @ dW)))        # tr(dW^T G dW)
+    t_dcw = float(np.sum(dW * CW))              # tr(dW^T C W)
+    t_whw = float(np.sum(W * (H @ W)))          # tr(W^T H W)
+    t_wgw = float(np.sum(W * (G @ W)))          # tr(W^T G W)
+    t_wcw = float(np.sum(W * CW))               # tr(W^T C W) = tr(W^T C^T W)
+    E2 = t_dgd - 2.0 * t_dcw + t_whw
+    T2 = t_wgw + 2.0 * t_wcw + t_whw
+    eps = 0.0 if T2 == 0.0 else E2 / T2
+    return dict(eps=eps, E2=E2, T2=T2)
+
+
+def select_layers(eps: Sequence[float], K: int) -> Tuple[List[int], List[int]]:
+    """The K layers with the lowest eps (ties: lower layer index first; NaN last).
+    Returns (idx in rank order, is_local flags)."""
+    L = len(eps)
+    key = [(math.inf if (e != e) else float(e), l) for l, e in enumerate(eps)]
+    order = [l for _, l in sorted(key)]
+    idx = order[:max(0, min(K, L))]
+    is_local = [0] * L
+    for l in idx:
+        is_local[l] = 1
+    return idx, is_local
+
+
+def project(A: np.ndarray, W: np.ndarray) -> np.ndarray:
+    """y = A W with A as [n, D] (column h*d + j) and W stored [D_in, D_out]."""
+    n = A.shape[0]
+    return np.asarray(A, np.float64).reshape(n, -1) @ np.asarray(W, np.float64)
+
+
+# --------------------------------------------------------------------------------------
+# A whole streaming run, chunk by chunk [ISPA §3.1, §3.3 re-triggered warmup].
+# --------------------------------------------------------------------------------------
+def run_episode(cfg, n_chunks: Optional[int] = None, K: Optional[int] = None,
+                keep_outputs: bool = False) -> Dict[str, object]:
+    """Warmup -> transition -> L/F inference (-> re-warmup at a scene cut) for a workload
+    from `synth`. Reading of the schedule: the warmup covers cfg.warmup_chunks chunks; at
+    a scene cut every layer restores its original W, its statistics restart from zero and
+    it becomes an F-layer again; a former L-layer's history restarts at the cut. The new
+    dW replaces the old one.
+
+    Returns per-transition eps/dW/selection and, if asked, per-chunk outputs y = O W_cur.
+    """
+    import synth  # seeded inputs only
+
+    L = cfg.layers
+    K = cfg.K if K is None else K
+    n_chunks = cfg.n_chunks if n_chunks is None else n_chunks
+    W0 = [synth.w_out(cfg, l).astype(np.float64) for l in range(L)]
+    W_cur = [w.copy() for w in W0]
+    is_local = [0] * L
+    hist_from: List[Optional[int]] = [None] * L
+    stats = [stats_init(cfg.D) for _ in range(L)]
+    warm_start = 0
+    transitions = []
+    outputs = []
+    for t in range(n_chunks):
+        if cfg.cut_chunk is not None and t == cfg.cut_chunk:
+            for l in range(L):
+                if is_local[l]:
+                    hist_from[l] = cfg.chunk_start_frame(t)
+                is_local[l] = 0
+                W_cur[l] = W0[l].copy()
+                stats[l] = stats_init(cfg.D)
+            warm_start = t
+        in_warmup = warm_start <= t < warm_start + cfg.warmup_chunks
+        chunk_out = []
+        for l in range(L):
+            q = synth.chunk_q(cfg, l, t)
+            if is_local[l]:
+                frames = list(range(cfg.sink_frames)) + list(range(cfg.chunk_start_frame(t),
+                                                                    cfg.chunk_start_frame(t) + cfg.chunk_frames))
+                k = synth.kv_tensor(cfg, l, frames, "k")
+                v = synth.kv_tensor(cfg, l, frames, "v")
+                O, _ = local_attention(q, k, v, cfg.scale)
+            else:
+                frames = synth.cache_frames(cfg, t, hist_from[l])
+                lay = synth.chunk_layout(cfg, frames, t)
+                k = synth.kv_tensor(cfg, l, frames, "k")
+                v = synth.kv_tensor(cfg, l, frames, "v")
+                res = split_attention(q, k, v, (lay["sink_begin"], lay["sink_end"]),
+                                      (lay["chunk_begin"], lay["chunk_end"]), cfg.scale)
+                O = res["A_full"]
+                if in_warmup:
+                    stats_update(stats[l], res["A_loc"], res["A_full"], cfg.dtype)
+            if keep_outputs:
+                chunk_out.append(project(O, W_cur[l]))
+        if keep_outputs:
+            outputs.append(chunk_out)
+        if in_warmup and t == warm_start + cfg.warmup_chunks - 1:
+            dWs, errs = [], []
+            for l in range(L):
+                s = stats[l]
+                dW = absorb_solve(s["G"], s["C"], W0[l], cfg.lam)
+                dWs.append(dW)
+                errs.append(reconstruction_error(s["G"], s["C"], s["H"], W0[l], dW))
+            eps = [e["eps"] for e in errs]
+            idx, flags = select_layers(eps, K)
+            for l in idx:
+                W_cur[l] = W0[l] + dWs[l]
+            is_local = flags
+            transitions.append(dict(chunk=t, eps=eps, errs=errs, dW=dWs, idx=idx, is_local=flags,
+                                    stats=[dict(G=s["G"].copy(), C=s["C"].copy(), H=s["H"].copy(),
+                                                rows=s["rows"]) for s in stats]))
+    return dict(transitions=transitions, outputs=outputs)

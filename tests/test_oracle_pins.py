@@ -1,0 +1,324 @@
+"""Pins of the CPU oracle against facts fixed by the ISPA pages and by mathematics.
+
+Every check here compares the oracle with something other than itself: hand-derived
+worked examples (tests/golden), closed forms, brute-force loops written out in plain
+Python, library routines that reach the same result by another algorithm (least squares
+by QR/SVD instead of the normal equations; torch's bf16 cast), and invariants.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _rand(shape, seed, std=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * std
+
+
+# ---------------------------------------------------------------- bf16 rounding
+def test_bf16_round_matches_torch_cast():
+    x = np.random.default_rng(0).standard_normal(200000)
+    x *= np.exp(np.random.default_rng(1).uniform(-20, 20, x.shape))
+    x = x.astype(np.float32).astype(np.float64)        # float32-exact, so torch rounds once
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(oracle.bf16_round(x), ref)
+
+
+def test_bf16_round_ties_to_even():
+    # 1 + 2^-8 sits halfway between 1 and 1 + 2^-7: ties go to the even mantissa (1.0).
+    # 1 + 3*2^-8 sits halfway between 1 + 2^-7 and 1 + 2^-6: goes to 1 + 2^-6.
+    vals = np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -(1 + 2.0 ** -8), 1 + 2.0 ** -8 + 2.0 ** -40])
+    want = np.array([1.0, 1 + 2.0 ** -6, -1.0, 1 + 2.0 ** -7])
+    assert np.array_equal(oracle.bf16_round(vals), want)
+
+
+def test_synth_bf16_bits_match_torch():
+    x = np.random.default_rng(2).standard_normal(100000).astype(np.float32)
+    bits = synth.bf16_bits_from_f32(x)
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(bits, ref)
+
+
+# ---------------------------------------------------------------- attention (step a1)
+def test_attention_golden_two_keys():
+    g = _golden("attention_two_keys.json")
+    q, k, v = (np.array(g[n], dtype=np.float64) for n in ("q", "k", "v"))
+    res = oracle.split_attention(q, k, v, tuple(g["sink"]), tuple(g["chunk"]), 1 / math.sqrt(2))
+    for name in ("A_full", "lse_full", "A_loc", "lse_loc", "A_hist", "lse_hist"):
+        np.testing.assert_allclose(res[name], np.array(g[name]), rtol=0, atol=1e-12, err_msg=name)
+
+
+def _brute_attention(q, k, v, rows, scale):
+    """Per-query softmax with Python loops and math.exp (no max subtraction needed at these sizes)."""
+    n_q, h, d = q.shape
+    A = np.zeros((n_q, h, d))
+    lse = np.full((h, n_q), -np.inf)
+    for i in range(n_q):
+        for hh in range(h):
+            if not rows:
+                continue
+            ws = []
+            for j in rows:
+                s = scale * sum(q[i, hh, c] * k[j, hh, c] for c in range(d))
+                ws.append(math.exp(s))
+            tot = sum(ws)
+            for c in range(d):
+                A[i, hh, c] = sum(w * v[j, hh, c] for w, j in zip(ws, rows)) / tot
+            lse[hh, i] = math.log(tot)
+    return A, lse
+
+
+@pytest.mark.parametrize("sink,chunk", [((0, 2), (5, 7)), ((0, 1), (3, 7)), ((0, 7), (7, 7)), ((0, 0), (0, 0))])
+def test_attention_brute_force(sink, chunk):
+    q, k, v = _rand((3, 2, 4), 10), _rand((7, 2, 4), 11), _rand((7, 2, 4), 12)
+    scale = 0.5
+    res = oracle.split_attention(q, k, v, sink, chunk, scale)
+    local = sorted(set(range(*sink)) | set(range(*chunk)))
+    hist = [j for j in range(7) if j not in local]
+    for name, rows in (("full", list(range(7))), ("loc", local), ("hist", hist)):
+        A, lse = _brute_attention(q, k, v, rows, scale)
+        np.testing.assert_allclose(res["A_" + name], A, rtol=1e-12, atol=1e-13, err_msg=name)
+        np.testing.assert_allclose(res["lse_" + name], lse, rtol=1e-12, atol=1e-13, err_msg=name)
+
+
+def test_lse_merge_equals_full_softmax():
+    q, k, v = _rand((40, 3, 16), 20), _rand((300, 3, 16), 21), _rand((300, 3, 16), 22)
+    res = oracle.split_attention(q, k, v, (0, 50), (220, 300), 0.25)
+    A, lse = oracle.lse_merge(res["A_loc"], res["lse_loc"], res["A_hist"], res["lse_hist"])
+    np.testing.assert_allclose(A, res["A_full"], rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(lse, res["lse_full"], rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(res["lse_full"], np.logaddexp(res["lse_loc"], res["lse_hist"]), rtol=1e-13)
+
+
+def test_attention_closed_forms():
+    # zero keys: every score is 0, softmax is uniform, A = mean of the masked V rows, lse = ln(n)
+    q, v = _rand((5, 2, 8), 30), _rand((9, 2, 8), 31)
+    k = np.zeros((9, 2, 8))
+    res = oracle.split_attention(q, k, v, (0, 2), (6, 9), 0.3)
+    np.testing.assert_allclose(res["A_full"], np.broadcast_to(v.mean(0), (5, 2, 8)), atol=1e-13)
+    np.testing.assert_allclose(res["A_loc"], np.broadcast_to(v[[0, 1, 6, 7, 8]].mean(0), (5, 2, 8)), atol=1e-13)
+    np.testing.assert_allclose(res["lse_hist"], np.full((2, 5), math.log(4)), atol=1e-13)
+    # a single key row: A is that V row, lse = scale * q.k
+    k1 = _rand((1, 2, 8), 32)
+    v1 = _rand((1, 2, 8), 33)
+    A, lse = oracle.local_attention(q, k1, v1, 0.3)
+    np.testing.assert_allclose(A, np.broadcast_to(v1[0], (5, 2, 8)), atol=1e-13)
+    np.testing.assert_allclose(lse, 0.3 * np.einsum("ihd,hd->hi", q, k1[0]), atol=1e-12)
+
+
+def test_empty_history_partition():
+    q, k, v = _rand((6, 2, 8), 40), _rand((10, 2, 8), 41), _rand((10, 2, 8), 42)
+    res = oracle.split_attention(q, k, v, (0, 4), (4, 10), 0.35)
+    assert np.array_equal(res["A_full"], res["A_loc"])
+    assert np.all(np.isneginf(res["lse_hist"])) and np.all(res["A_hist"] == 0)
+
+
+def test_local_attention_gather_equals_mask():
+    q, k, v = _rand((7, 2, 8), 50), _rand((30, 2, 8), 51), _rand((30, 2, 8), 52)
+    res = oracle.split_attention(q, k, v, (0, 5), (22, 30), 0.35)
+    rows = list(range(5)) + list(range(22, 30))
+    A, lse = oracle.local_attention(q, k[rows], v[rows], 0.35)
+    np.testing.assert_allclose(A, res["A_loc"], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(lse, res["lse_loc"], rtol=1e-13)
+
+
+# ---------------------------------------------------------------- statistics (step a2)
+def test_stats_brute_force_and_invariants():
+    n, h, d = 9, 2, 3
+    D = h * d
+    A_loc = _rand((n, h, d), 60)
+    A_full = A_loc + 0.3 * _rand((n, h, d), 61)
+    st = oracle.stats_init(D)
+    oracle.stats_update(st, A_loc, A_full, "fp32")
+    a = A_loc.reshape(n, D)
+    r = A_full.reshape(n, D) - a
+    G = np.zeros((D, D)); C = np.zeros((D, D)); H = np.zeros((D, D))
+    for i in range(n):
+        for p in range(D):
+            for q_ in range(D):
+                G[p, q_] += a[i, p] * a[i, q_]
+                C[p, q_] += a[i, p] * r[i, q_]
+                H[p, q_] += r[i, p] * r[i, q_]
+    np.testing.assert_allclose(st["G"], G, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(st["C"], C, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(st["H"], H, rtol=1e-13, atol=1e-14)
+    assert st["rows"] == n
+    for M in (st["G"], st["H"]):
+        assert np.allclose(M, M.T)
+        assert np.linalg.eigvalsh(M).min() > -1e-12
+
+
+def test_stats_chunkwise_equals_one_shot():
+    A_loc = _rand((50, 2, 4), 70)
+    A_full = A_loc + _rand((50, 2, 4), 71)
+    one = oracle.stats_init(8)
+    oracle.stats_update(one, A_loc, A_full, "bf16")
+    parts = oracle.stats_init(8)
+    for s in (slice(0, 13), slice(13, 14), slice(14, 50)):
+        oracle.stats_update(parts, A_loc[s], A_full[s], "bf16")
+    for name in ("G", "C", "H"):
+        np.testing.assert_allclose(parts[name], one[name], rtol=1e-12, atol=1e-13)
+    assert parts["rows"] == one["rows"] == 50
+
+
+def test_stats_bf16_operands_are_rounded():
+    # bf16-grid inputs keep R = A_full - A_loc exact in float32, so torch's float32 -> bf16
+    # cast gives the correctly rounded operand to compare with.
+    bf = lambda x: torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    A_loc = bf(_rand((20, 1, 6), 72))
+    A_full = bf(A_loc + _rand((20, 1, 6), 73))
+    st = oracle.stats_init(6)
+    oracle.stats_update(st, A_loc, A_full, "bf16")
+    a = A_loc.reshape(20, 6)
+    r = bf((A_full - A_loc).reshape(20, 6))
+    assert not np.array_equal(r, (A_full - A_loc).reshape(20, 6))   # rounding did something
+    np.testing.assert_allclose(st["G"], a.T @ a, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(st["C"], a.T @ r, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(st["H"], r.T @ r, rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------- absorb solve (step a3)
+def test_ridge_golden_scalar():
+    g = _golden("ridge_scalar.json")
+    G, C, H, W = (np.array(g[n]) for n in ("G", "C", "H", "W"))
+    dW = oracle.absorb_solve(G, C, W, g["lambda"])
+    np.testing.assert_allclose(dW, np.array(g["dW"]), rtol=1e-15)
+    e = oracle.reconstruction_error(G, C, H, W, dW)
+    assert abs(e["E2"] - g["E2"]) < 1e-12 and abs(e["T2"] - g["T2"]) < 1e-12
+    assert abs(e["eps"] - g["eps"]) < 1e-15
+
+
+def test_empty_history_gives_zero_update_and_error():
+    q, k, v = _rand((12, 2, 4), 80), _rand((16, 2, 4), 81), _rand((16, 2, 4), 82)
+    res = oracle.split_attention(q, k, v, (0, 4), (4, 16), 0.5)   # local covers all rows
+    st = oracle.stats_init(8)
+    oracle.stats_update(st, res["A_loc"], res["A_full"], "fp32")
+    W = _rand((8, 8), 83, 1 / math.sqrt(8))
+    dW = oracle.absorb_solve(st["G"], st["C"], W, 1e-2)
+    assert np.all(dW == 0)
+    e = oracle.reconstruction_error(st["G"], st["C"], st["H"], W, dW)
+    assert e["eps"] == 0.0 and e["E2"] == 0.0
+
+
+def test_planted_linear_residual_recovered_as_lambda_vanishes():
+    n, D = 64, 8
+    a = _rand((n, D), 90)
+    P = _rand((D, D), 91)
+    W = _rand((D, D), 92)
+    A_loc = a.reshape(n, 2, 4)
+    A_full = (a + a @ P).reshape(n, 2, 4)                         # R = A_loc P exactly
+    st = oracle.stats_init(D)
+    oracle.stats_update(st, A_loc, A_full, "fp32")
+    dW = oracle.absorb_solve(st["G"], st["C"], W, 1e-10)
+    np.testing.assert_allclose(dW, P @ W, rtol=1e-7, atol=1e-9)
+    e = oracle.reconstruction_error(st["G"], st["C"], st["H"], W, dW)
+    assert abs(e["eps"]) < 1e-9
+
+
+def test_solve_agrees_with_least_squares():
+    n, D, lam = 40, 6, 0.3
+    a = _rand((n, D), 100)
+    r = _rand((n, D), 101)
+    W = _rand((D, D), 102)
+    st = oracle.stats_init(D)
+    oracle.stats_update(st, a.reshape(n, 2, 3), (a + r).reshape(n, 2, 3), "fp32")
+    dW = oracle.absorb_solve(st["G"], st["C"], W, lam)
+    Aaug = np.vstack([a, math.sqrt(lam) * np.eye(D)])
+    Baug = np.vstack([r @ W, np.zeros((D, D))])
+    ref = np.linalg.lstsq(Aaug, Baug, rcond=None)[0]
+    np.testing.assert_allclose(dW, ref, rtol=1e-10, atol=1e-12)
+    res = (st["G"] + lam * np.eye(D)) @ dW - st["C"] @ W
+    assert np.linalg.norm(res) / np.linalg.norm(st["C"] @ W) < 1e-12
+
+
+def test_error_traces_match_direct_norms():
+    n, D, lam = 50, 6, 0.05
+    a = _rand((n, D), 110)
+    r = 0.5 * a @ _rand((D, D), 111) + 0.2 * _rand((n, D), 112)
+    W = _rand((D, D), 113)
+    st = oracle.stats_init(D)
+    oracle.stats_update(st, a.reshape(n, 3, 2), (a + r).reshape(n, 3, 2), "fp32")
+    for dW in (oracle.absorb_solve(st["G"], st["C"], W, lam), _rand((D, D), 114)):
+        e = oracle.reconstruction_error(st["G"], st["C"], st["H"], W, dW)
+        E2 = np.sum((a @ (W + dW) - (a + r) @ W) ** 2)
+        T2 = np.sum(((a + r) @ W) ** 2)
+        assert abs(e["E2"] - E2) < 1e-9 * T2
+        assert abs(e["T2"] - T2) < 1e-10 * T2
+        assert abs(e["eps"] - E2 / T2) < 1e-9
+
+
+def test_solution_minimises_the_ridge_objective():
+    n, D, lam = 30, 5, 0.2
+    a = _rand((n, D), 120)
+    r = _rand((n, D), 121)
+    W = _rand((D, D), 122)
+    st = oracle.stats_init(D)
+    oracle.stats_update(st, a.reshape(n, 1, 5), (a + r).reshape(n, 1, 5), "fp32")
+    dW = oracle.absorb_solve(st["G"], st["C"], W, lam)
+
+    def obj(X):
+        return np.sum((a @ (W + X) - (a + r) @ W) ** 2) + lam * np.sum(X ** 2)
+
+    base = obj(dW)
+    rng = np.random.default_rng(123)
+    for _ in range(20):
+        assert obj(dW + 1e-3 * rng.standard_normal((D, D))) > base
+
+
+# ---------------------------------------------------------------- selection (step a5)
+def test_selection_golden():
+    g = _golden("selection_examples.json")
+    for case in g["cases"]:
+        eps = [float("nan") if e == "nan" else e for e in case["eps"]]
+        idx, flags = oracle.select_layers(eps, case["K"])
+        assert idx == case["idx"], case
+        assert flags == case["is_local"], case
+
+
+# ---------------------------------------------------------------- whole episodes
+def _small(structured=False, **kw):
+    base = dict(name="small", layers=4, heads=2, head_dim=16, tpf=24, chunk_frames=2, h_max=6,
+                warmup_chunks=3, lam=1e-2, K=2, dtype="fp32", structured=structured, planted_rank=4)
+    base.update(kw)
+    return synth.IspaConfig(**base)
+
+
+def test_episode_structured_layers_are_absorbable():
+    """The planted (rank-4 template + small drift) layers must reach a far lower error
+    than the i.i.d. layers, and be the ones selected."""
+    cfg = _small(structured=True)
+    out = oracle.run_episode(cfg, n_chunks=cfg.warmup_chunks)
+    eps = out["transitions"][0]["eps"]
+    planted = [eps[l] for l in range(cfg.layers) if cfg.planted(l)]
+    iid = [eps[l] for l in range(cfg.layers) if not cfg.planted(l)]
+    assert max(planted) < 0.25 * min(iid), eps
+    assert sorted(out["transitions"][0]["idx"]) == [0, 2]
+
+
+def test_episode_rewarmup_after_cut():
+    cfg = _small(structured=True, cut_chunk=5, total_chunks=8)
+    out = oracle.run_episode(cfg)
+    assert [tr["chunk"] for tr in out["transitions"]] == [2, 7]
+    for tr in out["transitions"]:
+        assert all(s["rows"] == cfg.warmup_chunks * cfg.n_q for s in tr["stats"])
+
+
+def test_episode_warmup_schedule_rows():
+    cfg = _small()
+    out = oracle.run_episode(cfg, n_chunks=cfg.warmup_chunks, keep_outputs=True)
+    tr = out["transitions"][0]
+    assert tr["chunk"] == cfg.warmup_chunks - 1 and len(tr["idx"]) == cfg.K
+    assert len(out["outputs"]) == cfg.warmup_chunks
