@@ -1,0 +1,178 @@
+/*
+ * ispa.h -- C ABI of libispa, the B200 (sm_100a) implementation of the warmup-phase hot
+ * path of Instance-Specific Parametric Absorption (ISPA).
+ *
+ * Source of the method: "Towards Memory-Efficient Autoregressive Video Generation via
+ * Instance-Specific Parametric Absorption", paper text (paperpeel.com/paper/2607.00712),
+ * cited as [ISPA §x]; the reading notes at paper.gecl.asia, section "Method", cited as
+ * [notes: Method]. The paper publishes no API; these calls follow its problem statement.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Memory: the caller owns every buffer. Pointers named "device" must be device memory
+ *    of the current CUDA device; "host" pointers are host memory. The library allocates
+ *    nothing; calls that need scratch space take a caller-provided workspace `ws` of at
+ *    least ispa_workspace_bytes(...) bytes (256-byte aligned).
+ *  - Layouts (row-major): Q, K, V, O are [rows, heads, head_dim]; KV rows are in time
+ *    order. An attention output seen as a matrix A is [n_q, D] with D = heads*head_dim and
+ *    column h*head_dim + j. W (the attention output projection) is stored [D_in, D_out]
+ *    so that y = A W; a torch nn.Linear weight is its transpose. The bias of the
+ *    projection cancels out of the residual and is not used.
+ *  - lse arrays are [heads, n_q] float32, natural logarithm of the softmax denominator of
+ *    scale * q.k over the partition; an empty partition has lse = -inf and output 0.
+ *  - dtype ISPA_BF16: Q/K/V/O/W in bf16, softmax and accumulation in float32, the
+ *    statistics operands A_loc and R rounded to bf16, statistics in float32.
+ *    dtype ISPA_FP32: everything in float32.
+ *  - Asynchrony: every device call is enqueued on `stream` (NULL = legacy default
+ *    stream) and returns before the GPU finishes. Argument errors are reported before
+ *    anything is enqueued; a launch failure returns ISPA_ERR_CUDA. Errors found on the
+ *    device (a bounded wait that ran out) are latched in a per-device flag that
+ *    ispa_device_status() reads and clears.
+ *  - Threading: calls may come from several host threads; ispa_last_error() is
+ *    per-thread.
+ */
+#ifndef ISPA_H
+#define ISPA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *ispa_stream_t; /* a cudaStream_t */
+
+typedef enum {
+    ISPA_OK = 0,
+    ISPA_ERR_INVALID_ARG = -1,  /* bad pointer, size, range or dtype; nothing enqueued  */
+    ISPA_ERR_UNSUPPORTED = -2,  /* valid but not implemented (e.g. head_dim not 64/128) */
+    ISPA_ERR_CUDA = -3,         /* a CUDA runtime/driver call failed                     */
+    ISPA_ERR_NOT_SPD = -4,      /* G + lambda*I was not positive definite for a layer    */
+    ISPA_ERR_TIMEOUT = -5,      /* a bounded device-side wait ran out (device flag)      */
+    ISPA_ERR_WORKSPACE = -6     /* ws is NULL, misaligned or smaller than required       */
+} ispa_status;
+
+typedef enum { ISPA_BF16 = 0, ISPA_FP32 = 1 } ispa_dtype;
+
+/* One layer's attention call. The KV rows [0, n_kv) split into two partitions
+ * [ISPA §3.1 step 1]: the local partition = [sink_begin, sink_end) U [chunk_begin,
+ * chunk_end) (sink frame + current chunk), and the history partition = every other row.
+ * Ranges may be empty; they must lie inside [0, n_kv) and must not overlap. */
+typedef struct {
+    int n_q;          /* query rows (tokens of the chunk)                  */
+    int n_kv;         /* cached KV rows, sink and chunk included           */
+    int heads;        /* attention heads                                   */
+    int head_dim;     /* 64 or 128                                         */
+    int sink_begin, sink_end;
+    int chunk_begin, chunk_end;
+    float scale;      /* softmax scale, normally 1/sqrt(head_dim)          */
+    ispa_dtype dtype;
+} ispa_attn_desc;
+
+/* Ridge statistics of one layer [ISPA §3.2; notes: Method], all device memory:
+ * G = sum A_loc^T A_loc, C = sum A_loc^T R, H = sum R^T R (R = A_full - A_loc), each
+ * [D, D] float32 row-major, and rows = number of token rows accumulated. */
+typedef struct {
+    int D;
+    float *G;
+    float *C;
+    float *H;
+    long long *rows;
+} ispa_stats;
+
+/* ispa_attn_split -- decomposable attention [ISPA §3.1 step 1 "Dual-Stream Warmup",
+ * §3.4 "Decomposable Attention"]: one pass over the KV rows gives the local output
+ * (O_loc, lse_loc) and the history output (O_hist, lse_hist), merged by their
+ * log-sum-exps into the full output: lse_full = logaddexp(lse_loc, lse_hist),
+ * O_full = e^(lse_loc-lse_full) O_loc + e^(lse_hist-lse_full) O_hist.
+ *   q [n_q, heads, head_dim], k/v [n_kv, heads, head_dim]     (device, dtype)
+ *   o_full [n_q, heads, head_dim] (device, dtype), lse_full [heads, n_q] (device)
+ *   o_loc/lse_loc/o_hist/lse_hist: optional outputs (NULL to skip)
+ *   stats: optional; when given, R = O_full - O_loc is formed on chip and
+ *     G += A_loc^T A_loc, C += A_loc^T R, H += R^T R, rows += n_q (fused accumulation,
+ *     [ISPA §3.2]); stats->D must equal heads*head_dim. With stats == NULL the call is
+ *     plain full attention (an F-layer after the switch [ISPA §3.1 step 3]).
+ *   ws: workspace of ispa_workspace_bytes(desc, 1, D) bytes when stats != NULL
+ *     (may be NULL otherwise). */
+int ispa_attn_split(const ispa_attn_desc *desc, const void *q, const void *k, const void *v,
+                    void *o_full, float *lse_full, void *o_loc, float *lse_loc, void *o_hist,
+                    float *lse_hist, const ispa_stats *stats, void *ws, size_t ws_bytes,
+                    ispa_stream_t stream);
+
+/* ispa_accum_stats -- the statistics of [ISPA §3.2] from attention outputs that were
+ * computed elsewhere (unfused path): R = a_full - a_loc (then rounded to bf16 in bf16
+ * mode), G += A_loc^T A_loc, C += A_loc^T R, H += R^T R, rows += n_rows.
+ *   a_loc, a_full: [n_rows, D] device, dtype. ws: ispa_workspace_bytes(NULL, n_rows, D). */
+int ispa_accum_stats(const ispa_stats *stats, const void *a_loc, const void *a_full, int n_rows,
+                     ispa_dtype dtype, void *ws, size_t ws_bytes, ispa_stream_t stream);
+
+/* ispa_stats_reset -- zero G, C, H and rows (start of a warmup, or a re-warmup after a
+ * scene change [ISPA §3.1, §3.3]). */
+int ispa_stats_reset(const ispa_stats *stats, ispa_stream_t stream);
+
+/* ispa_solve_absorb -- Layer Absorb [ISPA §3.1 step 2, §3.2, §4.1 "Eq. 5"] and the
+ * per-layer reconstruction error [ISPA §3.3], batched over layers:
+ *   (G + lambda I) dW = C W, solved by a blocked Cholesky factorisation in float32;
+ *   eps = E^2 / T^2 with E^2 = tr(dW^T G dW) - 2 tr(dW^T C W) + tr(W^T H W) and
+ *   T^2 = tr(W^T (G + C + C^T + H) W) (relative squared error of the reconstructed
+ *   projected output; eps = 0 when T^2 = 0).
+ *   per_layer: host array of n_layers stats (device buffers, all with the same D).
+ *   w_o: host array of n_layers device pointers to W [D, D] of w_dtype.
+ *   dW: device [n_layers, D, D] float32.  eps: device [n_layers] float32.
+ *   err_terms: optional device [n_layers, 2] double (E^2, T^2).
+ *   w_new: optional host array of n_layers device pointers [D, D] w_dtype, written with
+ *     W + dW (rounded to bf16 in bf16 mode) [ISPA §3.1 step 3].
+ *   layer_status: device [n_layers] int, ISPA_OK or ISPA_ERR_NOT_SPD per layer (dW and
+ *     eps of such a layer are NaN).
+ *   ws: ispa_workspace_bytes(NULL, n_layers, D) bytes. */
+int ispa_solve_absorb(const ispa_stats *per_layer, int n_layers, const void *const *w_o,
+                      ispa_dtype w_dtype, float lambda, float *dW, float *eps, double *err_terms,
+                      void *const *w_new, int *layer_status, void *ws, size_t ws_bytes,
+                      ispa_stream_t stream);
+
+/* ispa_select_layers -- Dynamic Layer Selection [ISPA §3.3], host only: rank layers by
+ * eps ascending (ties: lower layer index first; NaN last) and take the first K.
+ *   eps_host [n_layers] (host), idx_out [min(K, n_layers)] (host, rank order),
+ *   is_local [n_layers] (host, 1 for a selected layer), either output may be NULL. */
+int ispa_select_layers(const float *eps_host, int n_layers, int K, int *idx_out,
+                       unsigned char *is_local);
+
+/* ispa_local_attn -- an L-layer after the switch [ISPA §3.1 step 3, §3.3]: attention
+ * over the local rows only (every one of desc->n_kv rows of k_loc/v_loc, i.e. the sink
+ * frame + current chunk; desc's range fields are ignored), and optionally the output
+ * projection with the updated weights, y = O W_new.
+ *   o [n_q, heads, head_dim] (device, dtype), lse [heads, n_q] (device, optional)
+ *   w_new [D, D] (device, dtype, optional), y [n_q, D] (device, dtype; required iff
+ *   w_new is given). ws: ispa_workspace_bytes(desc, 1, D) when w_new != NULL. */
+int ispa_local_attn(const ispa_attn_desc *desc, const void *q, const void *k_loc,
+                    const void *v_loc, void *o, float *lse, const void *w_new, void *y, void *ws,
+                    size_t ws_bytes, ispa_stream_t stream);
+
+/* ispa_workspace_bytes -- bytes of workspace that suffice for every call above with
+ * these shapes: attention calls described by `desc` (may be NULL), ispa_accum_stats
+ * with n_rows = n (when desc is NULL) and ispa_solve_absorb over n layers of size D. */
+size_t ispa_workspace_bytes(const ispa_attn_desc *desc, int n, int D);
+
+/* ispa_device_status -- synchronise `stream`, read and clear the current device's
+ * error flag. Returns ISPA_OK, ISPA_ERR_TIMEOUT (a kernel's bounded wait ran out and the
+ * kernel returned early; its outputs are not valid) or ISPA_ERR_CUDA. */
+int ispa_device_status(ispa_stream_t stream);
+
+/* ispa_selftest_bounded_wait -- test hook for the failure path: launches one kernel that
+ * waits on an mbarrier nothing ever arrives on, with a limit of `limit_us` microseconds
+ * (1..1000000), after which the kernel records ISPA_ERR_TIMEOUT in the device flag and
+ * returns. The GPU context stays usable. */
+int ispa_selftest_bounded_wait(unsigned limit_us, ispa_stream_t stream);
+
+/* ispa_last_error -- message of the last failing call on this host thread ("" if none). */
+const char *ispa_last_error(void);
+
+/* ispa_version -- library version string. */
+const char *ispa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ISPA_H */

@@ -1,0 +1,452 @@
+// C-ABI entry points of libispa: argument checks, workspace layout and dispatch to the
+// kernels. Every call enqueues on the caller's stream and allocates nothing.
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace ispa {
+cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H, const PtrBatch &W, ElemType wt,
+                        const PtrBatch &dW, const PtrBatch &M, const PtrBatch &Y, const PtrBatch &P, double *terms,
+                        int nparts, int *status, float *eps, double *err_terms, const PtrBatch *w_new, int D,
+                        float lambda, int batch, cudaStream_t s);
+}
+
+using namespace ispa;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *where) {
+    return fail(ISPA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+#define CUDA_CHECK_RET(x, where)                     \
+    do {                                             \
+        cudaError_t e_ = (x);                        \
+        if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+    } while (0)
+
+// Per-device error flag, shared by every kernel of the library. Host code never touches
+// the symbol directly: its device address is looked up once per device.
+__device__ int g_device_error_flag;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_flag_mutex;
+int *g_flag_ptr[kMaxDevices] = {nullptr};
+
+int device_error_flag(int **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(ISPA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+    std::lock_guard<std::mutex> lk(g_flag_mutex);
+    if (!g_flag_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_device_error_flag);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(error flag)");
+        g_flag_ptr[dev] = static_cast<int *>(p);
+    }
+    *out = g_flag_ptr[dev];
+    return ISPA_OK;
+}
+
+size_t elem_size(ispa_dtype t) { return t == ISPA_BF16 ? 2 : 4; }
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Workspace of one attention call with fused statistics: A_loc and R operands.
+size_t attn_ws_bytes(const ispa_attn_desc *d) {
+    const size_t D = (size_t)d->heads * d->head_dim;
+    return 2 * align_up((size_t)d->n_q * D * elem_size(d->dtype), 256);
+}
+
+size_t accum_ws_bytes(int n_rows, int D, ispa_dtype t) {
+    return align_up((size_t)n_rows * D * elem_size(t), 256);
+}
+
+constexpr int kEpsParts = 64;
+
+size_t solve_ws_bytes(int n_layers, int D) {
+    const size_t b = (size_t)std::min(n_layers, kMaxBatch);
+    const size_t mat = align_up((size_t)D * D * sizeof(float), 256);
+    return b * 3 * mat + align_up(5 * b * kEpsParts * sizeof(double), 256);
+}
+
+int check_desc(const ispa_attn_desc *d, bool need_ranges) {
+    if (!d) return fail(ISPA_ERR_INVALID_ARG, "desc is NULL");
+    if (d->n_q < 0 || d->n_kv < 0 || d->heads <= 0) return fail(ISPA_ERR_INVALID_ARG, "bad sizes n_q=%d n_kv=%d heads=%d", d->n_q, d->n_kv, d->heads);
+    if (d->head_dim != 64 && d->head_dim != 128) return fail(ISPA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", d->head_dim);
+    if (d->dtype != ISPA_BF16 && d->dtype != ISPA_FP32) return fail(ISPA_ERR_INVALID_ARG, "bad dtype %d", (int)d->dtype);
+    if (!(d->scale > 0.f) || !(d->scale < 1e30f)) return fail(ISPA_ERR_INVALID_ARG, "bad scale");
+    if ((long long)d->n_kv * d->heads * d->head_dim >= (1ll << 40)) return fail(ISPA_ERR_UNSUPPORTED, "KV too large");
+    if (need_ranges) {
+        auto okr = [&](int b, int e) { return 0 <= b && b <= e && e <= d->n_kv; };
+        if (!okr(d->sink_begin, d->sink_end)) return fail(ISPA_ERR_INVALID_ARG, "sink range [%d,%d) outside [0,%d)", d->sink_begin, d->sink_end, d->n_kv);
+        if (!okr(d->chunk_begin, d->chunk_end)) return fail(ISPA_ERR_INVALID_ARG, "chunk range [%d,%d) outside [0,%d)", d->chunk_begin, d->chunk_end, d->n_kv);
+        const bool se = d->sink_begin == d->sink_end, ce = d->chunk_begin == d->chunk_end;
+        if (!se && !ce && d->sink_begin < d->chunk_end && d->chunk_begin < d->sink_end)
+            return fail(ISPA_ERR_INVALID_ARG, "sink and chunk ranges overlap");
+    }
+    return ISPA_OK;
+}
+
+// Local segments first (in row order), then the history gaps.
+SegmentList make_segments(const ispa_attn_desc *d, bool local_only) {
+    SegmentList L;
+    L.count = 0;
+    if (local_only) {
+        if (d->n_kv > 0) L.seg[L.count++] = {0, d->n_kv, 0};
+        return L;
+    }
+    std::vector<std::pair<int, int>> loc;
+    if (d->sink_end > d->sink_begin) loc.push_back({d->sink_begin, d->sink_end});
+    if (d->chunk_end > d->chunk_begin) loc.push_back({d->chunk_begin, d->chunk_end});
+    std::sort(loc.begin(), loc.end());
+    for (auto &r : loc) L.seg[L.count++] = {r.first, r.second, 0};
+    int cur = 0;
+    for (auto &r : loc) {
+        if (r.first > cur) L.seg[L.count++] = {cur, r.first, 1};
+        cur = std::max(cur, r.second);
+    }
+    if (cur < d->n_kv) L.seg[L.count++] = {cur, d->n_kv, 1};
+    return L;
+}
+
+__global__ void add_rows_kernel(long long *rows, long long n) { *rows += n; }
+
+template <typename T>
+__global__ void residual_kernel(const T *a_loc, const T *a_full, T *r, size_t n) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        r[i] = from_f32<T>(to_f32(a_full[i]) - to_f32(a_loc[i]));
+}
+
+// G += A^T A, C += A^T R, H += R^T R, rows += n, for operands [n, D] of type t.
+int accumulate(const ispa_stats *st, const void *a_ops, const void *r_ops, int n, ispa_dtype t, int *flag,
+               cudaStream_t s) {
+    const int D = st->D;
+    if (n > 0) {
+        if (t == ISPA_BF16) {
+            CUDA_CHECK_RET(launch_stats_bf16(a_ops, r_ops, n, D, st->G, st->C, st->H, flag, s), "stats GEMM (bf16)");
+        } else {
+            const ElemType et = ElemType::F32;
+            GemmDesc g{D, D, n, D, D, D, false, false, et, et, ElemType::F32, 1.f, 1.f, false, 1};
+            GemmBatch b;
+            b.A[0] = a_ops; b.B[0] = a_ops; b.C[0] = st->G;
+            CUDA_CHECK_RET(launch_gemm_simt(g, b, s), "stats GEMM G");
+            b.A[0] = a_ops; b.B[0] = r_ops; b.C[0] = st->C;
+            CUDA_CHECK_RET(launch_gemm_simt(g, b, s), "stats GEMM C");
+            b.A[0] = r_ops; b.B[0] = r_ops; b.C[0] = st->H;
+            CUDA_CHECK_RET(launch_gemm_simt(g, b, s), "stats GEMM H");
+        }
+    }
+    add_rows_kernel<<<1, 1, 0, s>>>(st->rows, n);
+    CUDA_CHECK_RET(cudaGetLastError(), "rows counter");
+    return ISPA_OK;
+}
+
+int check_stats(const ispa_stats *st, int D) {
+    if (!st) return fail(ISPA_ERR_INVALID_ARG, "stats is NULL");
+    if (st->D != D) return fail(ISPA_ERR_INVALID_ARG, "stats D=%d but the attention has D=%d", st->D, D);
+    if (!st->G || !st->C || !st->H || !st->rows) return fail(ISPA_ERR_INVALID_ARG, "stats has a NULL buffer");
+    if (!aligned(st->G, 16) || !aligned(st->C, 16) || !aligned(st->H, 16)) return fail(ISPA_ERR_INVALID_ARG, "stats buffers must be 16-byte aligned");
+    return ISPA_OK;
+}
+
+int check_ws(void *ws, size_t have, size_t need) {
+    if (need == 0) return ISPA_OK;
+    if (!ws) return fail(ISPA_ERR_WORKSPACE, "workspace of %zu bytes required, got NULL", need);
+    if (!aligned(ws, 256)) return fail(ISPA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    if (have < need) return fail(ISPA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", have, need);
+    return ISPA_OK;
+}
+
+int run_attention(const ispa_attn_desc *d, const void *q, const void *k, const void *v, void *o_full, float *lse_full,
+                  void *o_loc, float *lse_loc, void *o_hist, float *lse_hist, void *a_ops, void *r_ops,
+                  bool local_only, cudaStream_t s) {
+    int *flag = nullptr;
+    int rc = device_error_flag(&flag);
+    if (rc != ISPA_OK) return rc;
+    AttnArgs a;
+    a.q = q; a.k = k; a.v = v;
+    a.o_full = o_full; a.lse_full = lse_full;
+    a.o_loc = o_loc; a.lse_loc = lse_loc;
+    a.o_hist = o_hist; a.lse_hist = lse_hist;
+    a.a_loc_ops = a_ops; a.r_ops = r_ops;
+    a.n_q = d->n_q; a.n_kv = d->n_kv; a.heads = d->heads; a.head_dim = d->head_dim;
+    a.scale = d->scale;
+    a.segs = make_segments(d, local_only);
+    a.err_flag = flag;
+    cudaError_t e = d->dtype == ISPA_FP32 ? launch_attn_simt_f32(a, s) : launch_attn_bf16(a, s);
+    if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
+    return ISPA_OK;
+}
+
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns, int *flag) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(&bar, 1);
+        ptx::fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        // Nothing ever arrives on `bar`: the wait must run out and record the timeout.
+        ptx::mbar_wait_bounded(&bar, 0, limit_ns, flag, nullptr);
+    }
+    __syncthreads();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *ispa_last_error(void) { return g_last_error.c_str(); }
+
+const char *ispa_version(void) { return "ispa-b200 0.1 (sm_100a)"; }
+
+size_t ispa_workspace_bytes(const ispa_attn_desc *desc, int n, int D) {
+    size_t need = 0;
+    if (desc) {
+        need = std::max(need, attn_ws_bytes(desc));
+        const size_t Dd = (size_t)desc->heads * desc->head_dim;
+        need = std::max(need, align_up((size_t)desc->n_q * Dd * elem_size(desc->dtype), 256));
+    } else if (n > 0 && D > 0) {
+        need = std::max(need, accum_ws_bytes(n, D, ISPA_FP32));
+    }
+    if (n > 0 && D > 0) need = std::max(need, solve_ws_bytes(n, D));
+    return need;
+}
+
+int ispa_attn_split(const ispa_attn_desc *desc, const void *q, const void *k, const void *v, void *o_full,
+                    float *lse_full, void *o_loc, float *lse_loc, void *o_hist, float *lse_hist,
+                    const ispa_stats *stats, void *ws, size_t ws_bytes, ispa_stream_t stream) {
+    g_last_error.clear();
+    int rc = check_desc(desc, true);
+    if (rc != ISPA_OK) return rc;
+    if (desc->n_q > 0 && (!q || !o_full || !lse_full)) return fail(ISPA_ERR_INVALID_ARG, "q, o_full and lse_full are required");
+    if (desc->n_kv > 0 && (!k || !v)) return fail(ISPA_ERR_INVALID_ARG, "k and v are required");
+    for (const void *p : {q, k, v, (const void *)o_full, (const void *)o_loc, (const void *)o_hist})
+        if (p && !aligned(p, 16)) return fail(ISPA_ERR_INVALID_ARG, "q/k/v/o buffers must be 16-byte aligned");
+    const int D = desc->heads * desc->head_dim;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    void *a_ops = nullptr, *r_ops = nullptr;
+    if (stats) {
+        rc = check_stats(stats, D);
+        if (rc != ISPA_OK) return rc;
+        rc = check_ws(ws, ws_bytes, attn_ws_bytes(desc));
+        if (rc != ISPA_OK) return rc;
+        a_ops = ws;
+        r_ops = static_cast<char *>(ws) + align_up((size_t)desc->n_q * D * elem_size(desc->dtype), 256);
+    }
+    if (desc->n_q > 0) {
+        rc = run_attention(desc, q, k, v, o_full, lse_full, o_loc, lse_loc, o_hist, lse_hist, a_ops, r_ops, false, s);
+        if (rc != ISPA_OK) return rc;
+    }
+    if (stats) {
+        int *flag = nullptr;
+        rc = device_error_flag(&flag);
+        if (rc != ISPA_OK) return rc;
+        return accumulate(stats, a_ops, r_ops, desc->n_q, desc->dtype, flag, s);
+    }
+    return ISPA_OK;
+}
+
+int ispa_accum_stats(const ispa_stats *stats, const void *a_loc, const void *a_full, int n_rows, ispa_dtype dtype,
+                     void *ws, size_t ws_bytes, ispa_stream_t stream) {
+    g_last_error.clear();
+    if (!stats) return fail(ISPA_ERR_INVALID_ARG, "stats is NULL");
+    if (dtype != ISPA_BF16 && dtype != ISPA_FP32) return fail(ISPA_ERR_INVALID_ARG, "bad dtype");
+    if (n_rows < 0) return fail(ISPA_ERR_INVALID_ARG, "n_rows < 0");
+    int rc = check_stats(stats, stats->D);
+    if (rc != ISPA_OK) return rc;
+    if (stats->D <= 0) return fail(ISPA_ERR_INVALID_ARG, "D <= 0");
+    if (n_rows > 0 && (!a_loc || !a_full)) return fail(ISPA_ERR_INVALID_ARG, "a_loc and a_full are required");
+    if ((a_loc && !aligned(a_loc, 16)) || (a_full && !aligned(a_full, 16))) return fail(ISPA_ERR_INVALID_ARG, "a_loc/a_full must be 16-byte aligned");
+    if (dtype == ISPA_BF16 && stats->D % 64 != 0) return fail(ISPA_ERR_UNSUPPORTED, "bf16 statistics need D %% 64 == 0");
+    rc = check_ws(ws, ws_bytes, n_rows > 0 ? accum_ws_bytes(n_rows, stats->D, dtype) : 0);
+    if (rc != ISPA_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int *flag = nullptr;
+    rc = device_error_flag(&flag);
+    if (rc != ISPA_OK) return rc;
+    const size_t n = (size_t)n_rows * stats->D;
+    if (n > 0) {
+        const int blocks = (int)std::min<size_t>((n + 255) / 256, 4096);
+        if (dtype == ISPA_BF16)
+            residual_kernel<bf16><<<blocks, 256, 0, s>>>((const bf16 *)a_loc, (const bf16 *)a_full, (bf16 *)ws, n);
+        else
+            residual_kernel<float><<<blocks, 256, 0, s>>>((const float *)a_loc, (const float *)a_full, (float *)ws, n);
+        CUDA_CHECK_RET(cudaGetLastError(), "residual kernel");
+    }
+    return accumulate(stats, a_loc, ws, n_rows, dtype, flag, s);
+}
+
+int ispa_stats_reset(const ispa_stats *stats, ispa_stream_t stream) {
+    g_last_error.clear();
+    if (!stats) return fail(ISPA_ERR_INVALID_ARG, "stats is NULL");
+    int rc = check_stats(stats, stats->D);
+    if (rc != ISPA_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t b = (size_t)stats->D * stats->D * sizeof(float);
+    CUDA_CHECK_RET(cudaMemsetAsync(stats->G, 0, b, s), "memset G");
+    CUDA_CHECK_RET(cudaMemsetAsync(stats->C, 0, b, s), "memset C");
+    CUDA_CHECK_RET(cudaMemsetAsync(stats->H, 0, b, s), "memset H");
+    CUDA_CHECK_RET(cudaMemsetAsync(stats->rows, 0, sizeof(long long), s), "memset rows");
+    return ISPA_OK;
+}
+
+int ispa_solve_absorb(const ispa_stats *per_layer, int n_layers, const void *const *w_o, ispa_dtype w_dtype,
+                      float lambda, float *dW, float *eps, double *err_terms, void *const *w_new, int *layer_status,
+                      void *ws, size_t ws_bytes, ispa_stream_t stream) {
+    g_last_error.clear();
+    if (n_layers < 0) return fail(ISPA_ERR_INVALID_ARG, "n_layers < 0");
+    if (n_layers == 0) return ISPA_OK;
+    if (!per_layer || !w_o || !dW || !eps || !layer_status) return fail(ISPA_ERR_INVALID_ARG, "per_layer, w_o, dW, eps and layer_status are required");
+    if (w_dtype != ISPA_BF16 && w_dtype != ISPA_FP32) return fail(ISPA_ERR_INVALID_ARG, "bad w_dtype");
+    if (!(lambda >= 0.f) || !(lambda < 1e30f)) return fail(ISPA_ERR_INVALID_ARG, "lambda must be finite and >= 0");
+    const int D = per_layer[0].D;
+    if (D <= 0 || D % 64 != 0) return fail(ISPA_ERR_UNSUPPORTED, "D=%d: the solve needs D %% 64 == 0", D);
+    for (int l = 0; l < n_layers; ++l) {
+        int rc = check_stats(&per_layer[l], D);
+        if (rc != ISPA_OK) return fail(rc, "layer %d: %s", l, g_last_error.c_str());
+        if (!w_o[l]) return fail(ISPA_ERR_INVALID_ARG, "w_o[%d] is NULL", l);
+        if (w_new && !w_new[l]) return fail(ISPA_ERR_INVALID_ARG, "w_new[%d] is NULL", l);
+    }
+    if (!aligned(dW, 16)) return fail(ISPA_ERR_INVALID_ARG, "dW must be 16-byte aligned");
+    int rc = check_ws(ws, ws_bytes, solve_ws_bytes(n_layers, D));
+    if (rc != ISPA_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    CUDA_CHECK_RET(cudaMemsetAsync(layer_status, 0, sizeof(int) * n_layers, s), "memset layer_status");
+
+    const size_t mat = align_up((size_t)D * D * sizeof(float), 256);
+    const int bmax = std::min(n_layers, kMaxBatch);
+    char *wsb = static_cast<char *>(ws);
+    double *terms = reinterpret_cast<double *>(wsb + (size_t)bmax * 3 * mat);
+    for (int l0 = 0; l0 < n_layers; l0 += kMaxBatch) {
+        const int b = std::min(kMaxBatch, n_layers - l0);
+        PtrBatch G, C, H, W, DW, M, Y, P, WN;
+        for (int z = 0; z < b; ++z) {
+            const ispa_stats &st = per_layer[l0 + z];
+            G.p[z] = st.G; C.p[z] = st.C; H.p[z] = st.H;
+            W.p[z] = const_cast<void *>(w_o[l0 + z]);
+            DW.p[z] = dW + (size_t)(l0 + z) * D * D;
+            M.p[z] = wsb + (size_t)z * 3 * mat;
+            Y.p[z] = wsb + (size_t)z * 3 * mat + mat;
+            P.p[z] = wsb + (size_t)z * 3 * mat + 2 * mat;
+            if (w_new) WN.p[z] = w_new[l0 + z];
+        }
+        cudaError_t e = solve_batch(G, C, H, W, w_dtype == ISPA_BF16 ? ElemType::BF16 : ElemType::F32, DW, M, Y, P,
+                                    terms, kEpsParts, layer_status + l0, eps + l0,
+                                    err_terms ? err_terms + 2 * (size_t)l0 : nullptr, w_new ? &WN : nullptr, D, lambda,
+                                    b, s);
+        if (e != cudaSuccess) return cuda_fail(e, "absorb solve");
+    }
+    return ISPA_OK;
+}
+
+int ispa_select_layers(const float *eps_host, int n_layers, int K, int *idx_out, unsigned char *is_local) {
+    g_last_error.clear();
+    if (n_layers < 0) return fail(ISPA_ERR_INVALID_ARG, "n_layers < 0");
+    if (K < 0) return fail(ISPA_ERR_INVALID_ARG, "K < 0");
+    if (n_layers > 0 && !eps_host) return fail(ISPA_ERR_INVALID_ARG, "eps_host is NULL");
+    std::vector<int> order(n_layers);
+    for (int l = 0; l < n_layers; ++l) order[l] = l;
+    auto key = [&](int l) {
+        const float e = eps_host[l];
+        return e != e ? INFINITY : e;   // NaN ranks last
+    };
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
+        const float ka = key(a), kb = key(b);
+        if (ka < kb) return true;
+        if (kb < ka) return false;
+        return a < b;
+    });
+    const int k = std::min(K, n_layers);
+    if (idx_out)
+        for (int i = 0; i < k; ++i) idx_out[i] = order[i];
+    if (is_local) {
+        for (int l = 0; l < n_layers; ++l) is_local[l] = 0;
+        for (int i = 0; i < k; ++i) is_local[order[i]] = 1;
+    }
+    return ISPA_OK;
+}
+
+int ispa_local_attn(const ispa_attn_desc *desc, const void *q, const void *k_loc, const void *v_loc, void *o,
+                    float *lse, const void *w_new, void *y, void *ws, size_t ws_bytes, ispa_stream_t stream) {
+    g_last_error.clear();
+    int rc = check_desc(desc, false);
+    if (rc != ISPA_OK) return rc;
+    if (desc->n_q > 0 && (!q || !o)) return fail(ISPA_ERR_INVALID_ARG, "q and o are required");
+    if (desc->n_kv > 0 && (!k_loc || !v_loc)) return fail(ISPA_ERR_INVALID_ARG, "k_loc and v_loc are required");
+    if ((w_new == nullptr) != (y == nullptr)) return fail(ISPA_ERR_INVALID_ARG, "w_new and y go together");
+    for (const void *p : {q, k_loc, v_loc, (const void *)o, w_new, (const void *)y})
+        if (p && !aligned(p, 16)) return fail(ISPA_ERR_INVALID_ARG, "buffers must be 16-byte aligned");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int D = desc->heads * desc->head_dim;
+    // lse is optional for the caller but the kernels always write one: park it in ws.
+    float *lse_out = lse;
+    size_t need = 0;
+    if (!lse) need += align_up((size_t)desc->heads * desc->n_q * sizeof(float), 256);
+    rc = check_ws(ws, ws_bytes, need);
+    if (rc != ISPA_OK) return rc;
+    if (!lse) lse_out = static_cast<float *>(ws);
+    if (desc->n_q == 0) return ISPA_OK;
+    rc = run_attention(desc, q, k_loc, v_loc, o, lse_out, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, true, s);
+    if (rc != ISPA_OK) return rc;
+    if (w_new) {
+        const ElemType t = desc->dtype == ISPA_BF16 ? ElemType::BF16 : ElemType::F32;
+        GemmDesc g{desc->n_q, D, D, D, D, D, true, false, t, t, t, 1.f, 0.f, false, 1};
+        GemmBatch b;
+        b.A[0] = o; b.B[0] = w_new; b.C[0] = y;
+        CUDA_CHECK_RET(launch_gemm_simt(g, b, s), "projection GEMM");
+    }
+    return ISPA_OK;
+}
+
+int ispa_device_status(ispa_stream_t stream) {
+    g_last_error.clear();
+    int *flag = nullptr;
+    int rc = device_error_flag(&flag);
+    if (rc != ISPA_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    CUDA_CHECK_RET(cudaStreamSynchronize(s), "cudaStreamSynchronize");
+    int v = 0;
+    CUDA_CHECK_RET(cudaMemcpy(&v, flag, sizeof(int), cudaMemcpyDeviceToHost), "read device flag");
+    if (v != 0) {
+        const int zero = 0;
+        CUDA_CHECK_RET(cudaMemcpy(flag, &zero, sizeof(int), cudaMemcpyHostToDevice), "clear device flag");
+        return fail(v, "a kernel reported device error %d", v);
+    }
+    return ISPA_OK;
+}
+
+int ispa_selftest_bounded_wait(unsigned limit_us, ispa_stream_t stream) {
+    g_last_error.clear();
+    if (limit_us < 1 || limit_us > 1000000) return fail(ISPA_ERR_INVALID_ARG, "limit_us must be in [1, 1e6]");
+    int *flag = nullptr;
+    int rc = device_error_flag(&flag);
+    if (rc != ISPA_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    bounded_wait_selftest_kernel<<<1, 32, 0, s>>>((uint64_t)limit_us * 1000ull, flag);
+    CUDA_CHECK_RET(cudaGetLastError(), "selftest launch");
+    return ISPA_OK;
+}
+
+}  // extern "C"

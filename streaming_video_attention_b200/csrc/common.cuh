@@ -1,0 +1,104 @@
+// Shared definitions of the libispa CUDA sources (internal; not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/ispa.h"
+
+namespace ispa {
+
+typedef __nv_bfloat16 bf16;
+
+constexpr int kMaxBatch = 48;      // layers per batched launch of the solve kernels
+constexpr int kMaxSegments = 6;    // KV row segments of one attention call
+
+// A run of KV rows [begin, end) that belongs to one partition (0 = local, 1 = history).
+struct Segment {
+    int begin, end, part;
+};
+
+struct SegmentList {
+    Segment seg[kMaxSegments];
+    int count;
+};
+
+__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(bf16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ bf16 from_f32<bf16>(float x) { return __float2bfloat16_rn(x); }
+
+// Latch a device-side error code (first writer wins) into the per-device flag.
+__device__ __forceinline__ void raise_device_error(int *flag, int code) {
+    if (flag) atomicCAS(flag, 0, code);
+}
+
+// ---- launchers implemented in the .cu files ------------------------------------------
+
+struct AttnArgs {
+    const void *q, *k, *v;
+    void *o_full;
+    float *lse_full;
+    void *o_loc;
+    float *lse_loc;
+    void *o_hist;
+    float *lse_hist;
+    void *a_loc_ops;   // statistics operand A_loc [n_q, D] (bf16 or fp32), or null
+    void *r_ops;       // statistics operand R [n_q, D], or null
+    int n_q, n_kv, heads, head_dim;
+    float scale;
+    SegmentList segs;
+    int *err_flag;
+};
+
+cudaError_t launch_attn_simt_f32(const AttnArgs &a, cudaStream_t s);
+cudaError_t launch_attn_simt_bf16(const AttnArgs &a, cudaStream_t s);
+cudaError_t launch_attn_bf16(const AttnArgs &a, cudaStream_t s);   // tcgen05 path
+
+// Batched SIMT GEMM: C_z[m][n] = alpha * sum_k A_z(m,k) B_z(k,n) + beta * C_z[m][n].
+// A_z(m,k) = A[m*lda + k] if a_kcontig else A[k*lda + m]; B_z(k,n) = B[n*ldb + k] if
+// b_kcontig else B[k*ldb + n]. lower_only restricts the update to tiles touching m >= n.
+enum class ElemType { F32 = 0, BF16 = 1 };
+struct GemmBatch {
+    const void *A[kMaxBatch];
+    const void *B[kMaxBatch];
+    void *C[kMaxBatch];
+};
+struct GemmDesc {
+    int M, N, K;
+    int lda, ldb, ldc;
+    bool a_kcontig, b_kcontig;
+    ElemType a_type, b_type, c_type;
+    float alpha, beta;
+    bool lower_only;
+    int batch;
+};
+cudaError_t launch_gemm_simt(const GemmDesc &d, const GemmBatch &b, cudaStream_t s);
+
+// Ridge statistics from bf16 operands [n, D] row-major, float32 G/C/H updated in place.
+cudaError_t launch_stats_bf16(const void *a_loc, const void *r, int n, int D, float *G, float *C,
+                               float *H, int *err_flag, cudaStream_t s);
+
+// Solve-phase kernels (float32, batched over layers).
+struct PtrBatch {
+    void *p[kMaxBatch];
+};
+cudaError_t launch_fill_shifted(const PtrBatch &src, const PtrBatch &dst, int D, float lambda, int batch,
+                                cudaStream_t s);
+cudaError_t launch_potrf_diag(const PtrBatch &M, int D, int k0, int nb, int *status, int batch, cudaStream_t s);
+cudaError_t launch_trsm_panel(const PtrBatch &M, int D, int k0, int nb, int batch, cudaStream_t s);
+cudaError_t launch_trsv_block(const PtrBatch &L, const PtrBatch &X, int D, int k0, int nb, bool transpose,
+                              int batch, cudaStream_t s);
+cudaError_t launch_trace_terms(const PtrBatch &X, const PtrBatch &P, int D, int which, int ncols_x_is_w_bf16,
+                               double *partials, int nparts, int batch, cudaStream_t s);
+cudaError_t launch_copy_f32(const PtrBatch &src, const PtrBatch &dst, size_t n, int batch, cudaStream_t s);
+cudaError_t launch_convert_w(const PtrBatch &w, ElemType t, const PtrBatch &out, size_t n, int batch,
+                             cudaStream_t s);
+
+}  // namespace ispa

@@ -1,0 +1,318 @@
+// Absorb solve and reconstruction error, float32, batched over layers
+// [ISPA §3.1 step 2, §3.2, §3.3, §4.1 "Eq. 5"].
+//
+//   M = G + lambda I                          fill_shifted
+//   M = L L^T (blocked, right-looking)        potrf_diag + trsm_panel + GEMM trailing update
+//   dW = L^-T L^-1 (C W)                      GEMM, then trsv_block + GEMM per block, both ways
+//   five traces -> E^2, T^2, eps              GEMMs G dW, H W, G W, then dot_partials
+//
+// Block size nb = 64 (D must be a multiple of 64). The diagonal blocks are factored and
+// solved by one CTA each in shared memory; everything of order D^3 runs in the batched
+// GEMM. A non-positive pivot marks the layer ISPA_ERR_NOT_SPD and turns its results to
+// NaN; nothing traps.
+#include "common.cuh"
+
+namespace ispa {
+namespace {
+
+constexpr int NB = 64;
+
+__global__ void fill_shifted_kernel(PtrBatch src, PtrBatch dst, int D, float lambda) {
+    const int z = blockIdx.y;
+    const float *S = static_cast<const float *>(src.p[z]);
+    float *Dst = static_cast<float *>(dst.p[z]);
+    const size_t n = (size_t)D * D;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        float v = S[i];
+        if (i / D == i % D) v += lambda;
+        Dst[i] = v;
+    }
+}
+
+__global__ void potrf_diag_kernel(PtrBatch M, int D, int k0, int *status) {
+    __shared__ float A[NB][NB + 1];
+    const int z = blockIdx.x;
+    float *Mz = static_cast<float *>(M.p[z]);
+    const int tid = threadIdx.x, nt = blockDim.x;
+    for (int idx = tid; idx < NB * NB; idx += nt) {
+        const int i = idx / NB, j = idx % NB;
+        A[i][j] = Mz[(size_t)(k0 + i) * D + k0 + j];
+    }
+    __syncthreads();
+    for (int j = 0; j < NB; ++j) {
+        if (tid == 0) {
+            float d = A[j][j];
+            if (!(d > 0.f)) {
+                status[z] = ISPA_ERR_NOT_SPD;
+                d = __int_as_float(0x7fc00000);
+            } else {
+                d = sqrtf(d);
+            }
+            A[j][j] = d;
+        }
+        __syncthreads();
+        for (int i = j + 1 + tid; i < NB; i += nt) A[i][j] = A[i][j] / A[j][j];
+        __syncthreads();
+        const int w = NB - j - 1;
+        for (int idx = tid; idx < w * w; idx += nt) {
+            const int r = j + 1 + idx / w, c = j + 1 + idx % w;
+            if (c <= r) A[r][c] -= A[r][j] * A[c][j];
+        }
+        __syncthreads();
+    }
+    for (int idx = tid; idx < NB * NB; idx += nt) {
+        const int i = idx / NB, j = idx % NB;
+        if (j <= i) Mz[(size_t)(k0 + i) * D + k0 + j] = A[i][j];
+    }
+}
+
+// Rows below the diagonal block: L21 = A21 L11^-T (row-wise forward substitution).
+__global__ void trsm_panel_kernel(PtrBatch M, int D, int k0) {
+    __shared__ float Lk[NB][NB + 1];
+    __shared__ float Xs[NB][NB + 1];
+    const int z = blockIdx.y;
+    float *Mz = static_cast<float *>(M.p[z]);
+    const int r0 = k0 + NB + blockIdx.x * NB;
+    const int tid = threadIdx.x, nt = blockDim.x;
+    for (int idx = tid; idx < NB * NB; idx += nt) {
+        const int i = idx / NB, j = idx % NB;
+        Lk[i][j] = j <= i ? Mz[(size_t)(k0 + i) * D + k0 + j] : 0.f;
+        Xs[i][j] = (r0 + i < D) ? Mz[(size_t)(r0 + i) * D + k0 + j] : 0.f;
+    }
+    __syncthreads();
+    if (tid < NB && r0 + tid < D) {
+        const int row = tid;
+        for (int j = 0; j < NB; ++j) {
+            float x = Xs[row][j];
+            for (int c = 0; c < j; ++c) x -= Xs[row][c] * Lk[j][c];
+            Xs[row][j] = x / Lk[j][j];
+        }
+    }
+    __syncthreads();
+    for (int idx = tid; idx < NB * NB; idx += nt) {
+        const int i = idx / NB, j = idx % NB;
+        if (r0 + i < D) Mz[(size_t)(r0 + i) * D + k0 + j] = Xs[i][j];
+    }
+}
+
+// X_k = L_kk^-1 X_k (forward) or L_kk^-T X_k (backward) for the NB rows of block k,
+// every column of X at once (one thread per column).
+template <bool TRANS>
+__global__ void __launch_bounds__(128) trsv_block_kernel(PtrBatch L, PtrBatch X, int D, int k0) {
+    __shared__ float Lk[NB][NB + 1];
+    const int z = blockIdx.y;
+    const float *Lz = static_cast<const float *>(L.p[z]);
+    float *Xz = static_cast<float *>(X.p[z]);
+    for (int idx = threadIdx.x; idx < NB * NB; idx += blockDim.x) {
+        const int i = idx / NB, j = idx % NB;
+        Lk[i][j] = j <= i ? Lz[(size_t)(k0 + i) * D + k0 + j] : 0.f;
+    }
+    __syncthreads();
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= D) return;
+    float x[NB];
+#pragma unroll
+    for (int j = 0; j < NB; ++j) x[j] = Xz[(size_t)(k0 + j) * D + c];
+    if (!TRANS) {
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+            float v = x[j];
+#pragma unroll
+            for (int i = 0; i < j; ++i) v -= Lk[j][i] * x[i];
+            x[j] = v / Lk[j][j];
+        }
+    } else {
+#pragma unroll
+        for (int j = NB - 1; j >= 0; --j) {
+            float v = x[j];
+#pragma unroll
+            for (int i = j + 1; i < NB; ++i) v -= Lk[i][j] * x[i];
+            x[j] = v / Lk[j][j];
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < NB; ++j) Xz[(size_t)(k0 + j) * D + c] = x[j];
+}
+
+// partial[z][blockIdx.x] = sum over a strided share of i of X_z[i] * P_z[i] (double).
+template <typename TX>
+__global__ void __launch_bounds__(256) dot_partials_kernel(PtrBatch X, PtrBatch P, size_t n, double *partials) {
+    const int z = blockIdx.y;
+    const TX *Xz = static_cast<const TX *>(X.p[z]);
+    const float *Pz = static_cast<const float *>(P.p[z]);
+    double s = 0.0;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        s += (double)to_f32(Xz[i]) * (double)Pz[i];
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_down_sync(0xffffffffu, s, o);
+    __shared__ double red[8];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double t = 0.0;
+        for (int w = 0; w < 8; ++w) t += red[w];
+        partials[(size_t)z * gridDim.x + blockIdx.x] = t;
+    }
+}
+
+// terms[k][z][p] for k = 0..4: tr(dW^T G dW), tr(dW^T C W), tr(W^T H W), tr(W^T G W), tr(W^T C W)
+__global__ void finalize_eps_kernel(const double *terms, int nparts, int batch, const int *status, float *eps,
+                                    double *err_terms) {
+    const int z = blockIdx.x * blockDim.x + threadIdx.x;
+    if (z >= batch) return;
+    double t[5];
+    for (int k = 0; k < 5; ++k) {
+        double s = 0.0;
+        for (int p = 0; p < nparts; ++p) s += terms[((size_t)k * batch + z) * nparts + p];
+        t[k] = s;
+    }
+    const double E2 = t[0] - 2.0 * t[1] + t[2];
+    const double T2 = t[3] + 2.0 * t[4] + t[2];
+    float e = T2 == 0.0 ? 0.f : (float)(E2 / T2);
+    if (status[z] != ISPA_OK) e = __int_as_float(0x7fc00000);
+    eps[z] = e;
+    if (err_terms) {
+        err_terms[2 * z] = E2;
+        err_terms[2 * z + 1] = T2;
+    }
+}
+
+template <typename TW>
+__global__ void add_delta_kernel(PtrBatch W, PtrBatch dW, PtrBatch out, size_t n) {
+    const int z = blockIdx.y;
+    const TW *Wz = static_cast<const TW *>(W.p[z]);
+    const float *dz = static_cast<const float *>(dW.p[z]);
+    TW *oz = static_cast<TW *>(out.p[z]);
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        oz[i] = from_f32<TW>(to_f32(Wz[i]) + dz[i]);
+}
+
+__global__ void copy_f32_kernel(PtrBatch src, PtrBatch dst, size_t n) {
+    const int z = blockIdx.y;
+    const float4 *s = static_cast<const float4 *>(src.p[z]);
+    float4 *d = static_cast<float4 *>(dst.p[z]);
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n / 4; i += (size_t)gridDim.x * blockDim.x)
+        d[i] = s[i];
+}
+
+}  // namespace
+
+// ---- host side ----------------------------------------------------------------------
+
+static GemmBatch make_gemm_batch(const PtrBatch &A, size_t offA, const PtrBatch &B, size_t offB, const PtrBatch &C,
+                                 size_t offC, int batch, size_t eA, size_t eB) {
+    GemmBatch g;
+    for (int z = 0; z < batch; ++z) {
+        g.A[z] = static_cast<const char *>(A.p[z]) + offA * eA;
+        g.B[z] = static_cast<const char *>(B.p[z]) + offB * eB;
+        g.C[z] = static_cast<char *>(C.p[z]) + offC * sizeof(float);
+    }
+    return g;
+}
+
+#define ISPA_TRY(x)                          \
+    do {                                     \
+        cudaError_t e_ = (x);                \
+        if (e_ != cudaSuccess) return e_;    \
+    } while (0)
+
+// Solve for one batch of layers. All pointers are device pointers, one per layer.
+//   G, C, H: statistics; W: weights of type wt; dW: output; M, Y: D*D float scratch each;
+//   P: D*D float scratch; terms: 5 * batch * nparts doubles; status: batch ints (zeroed).
+cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H, const PtrBatch &W, ElemType wt,
+                        const PtrBatch &dW, const PtrBatch &M, const PtrBatch &Y, const PtrBatch &P, double *terms,
+                        int nparts, int *status, float *eps, double *err_terms, const PtrBatch *w_new, int D,
+                        float lambda, int batch, cudaStream_t s) {
+    const size_t n = (size_t)D * D;
+    const size_t ew = wt == ElemType::BF16 ? 2 : 4;
+    const int fill_blocks = (int)std::min<size_t>((n + 255) / 256, 1024);
+
+    // M = G + lambda I
+    fill_shifted_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(G, M, D, lambda);
+    ISPA_TRY(cudaGetLastError());
+
+    // Y = C W, and dW <- Y (solved in place below)
+    {
+        GemmDesc d{D, D, D, D, D, D, true, false, ElemType::F32, wt, ElemType::F32, 1.f, 0.f, false, batch};
+        ISPA_TRY(launch_gemm_simt(d, make_gemm_batch(C, 0, W, 0, Y, 0, batch, 4, ew), s));
+        copy_f32_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(Y, dW, n);
+        ISPA_TRY(cudaGetLastError());
+    }
+
+    // Cholesky factorisation, blocked
+    const int nblk = D / NB;
+    for (int kb = 0; kb < nblk; ++kb) {
+        const int k0 = kb * NB;
+        potrf_diag_kernel<<<batch, 256, 0, s>>>(M, D, k0, status);
+        ISPA_TRY(cudaGetLastError());
+        const int rest = D - k0 - NB;
+        if (rest <= 0) break;
+        trsm_panel_kernel<<<dim3((rest + NB - 1) / NB, batch), 256, 0, s>>>(M, D, k0);
+        ISPA_TRY(cudaGetLastError());
+        GemmDesc d{rest, rest, NB, D, D, D, true, true, ElemType::F32, ElemType::F32, ElemType::F32, -1.f, 1.f,
+                   true, batch};
+        const size_t offA = (size_t)(k0 + NB) * D + k0;
+        const size_t offC = (size_t)(k0 + NB) * D + k0 + NB;
+        ISPA_TRY(launch_gemm_simt(d, make_gemm_batch(M, offA, M, offA, M, offC, batch, 4, 4), s));
+    }
+
+    // Forward substitution L Z = Y (in dW)
+    const dim3 tgrid((D + 127) / 128, batch);
+    for (int kb = 0; kb < nblk; ++kb) {
+        const int k0 = kb * NB;
+        trsv_block_kernel<false><<<tgrid, 128, 0, s>>>(M, dW, D, k0);
+        ISPA_TRY(cudaGetLastError());
+        const int rest = D - k0 - NB;
+        if (rest <= 0) break;
+        GemmDesc d{rest, D, NB, D, D, D, true, false, ElemType::F32, ElemType::F32, ElemType::F32, -1.f, 1.f,
+                   false, batch};
+        ISPA_TRY(launch_gemm_simt(
+            d, make_gemm_batch(M, (size_t)(k0 + NB) * D + k0, dW, (size_t)k0 * D, dW, (size_t)(k0 + NB) * D, batch, 4, 4),
+            s));
+    }
+    // Backward substitution L^T X = Z
+    for (int kb = nblk - 1; kb >= 0; --kb) {
+        const int k0 = kb * NB;
+        trsv_block_kernel<true><<<tgrid, 128, 0, s>>>(M, dW, D, k0);
+        ISPA_TRY(cudaGetLastError());
+        if (k0 == 0) break;
+        // X[0:k0, :] -= (L[k0:k0+NB, 0:k0])^T X_k
+        GemmDesc d{k0, D, NB, D, D, D, false, false, ElemType::F32, ElemType::F32, ElemType::F32, -1.f, 1.f, false,
+                   batch};
+        ISPA_TRY(launch_gemm_simt(d, make_gemm_batch(M, (size_t)k0 * D, dW, (size_t)k0 * D, dW, 0, batch, 4, 4), s));
+    }
+
+    // Reconstruction error terms
+    const dim3 rgrid(nparts, batch);
+    GemmDesc full{D, D, D, D, D, D, true, false, ElemType::F32, ElemType::F32, ElemType::F32, 1.f, 0.f, false, batch};
+    // t0 = tr(dW^T G dW)
+    ISPA_TRY(launch_gemm_simt(full, make_gemm_batch(G, 0, dW, 0, P, 0, batch, 4, 4), s));
+    dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, P, n, terms + 0 * (size_t)batch * nparts);
+    // t1 = tr(dW^T C W)
+    dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, Y, n, terms + 1 * (size_t)batch * nparts);
+    // t2 = tr(W^T H W), t3 = tr(W^T G W), t4 = tr(W^T C W)
+    GemmDesc fw = full;
+    fw.b_type = wt;
+    ISPA_TRY(launch_gemm_simt(fw, make_gemm_batch(H, 0, W, 0, P, 0, batch, 4, ew), s));
+    if (wt == ElemType::BF16) dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, P, n, terms + 2 * (size_t)batch * nparts);
+    else dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, P, n, terms + 2 * (size_t)batch * nparts);
+    ISPA_TRY(launch_gemm_simt(fw, make_gemm_batch(G, 0, W, 0, P, 0, batch, 4, ew), s));
+    if (wt == ElemType::BF16) {
+        dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, P, n, terms + 3 * (size_t)batch * nparts);
+        dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, Y, n, terms + 4 * (size_t)batch * nparts);
+    } else {
+        dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, P, n, terms + 3 * (size_t)batch * nparts);
+        dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, Y, n, terms + 4 * (size_t)batch * nparts);
+    }
+    ISPA_TRY(cudaGetLastError());
+    finalize_eps_kernel<<<(batch + 63) / 64, 64, 0, s>>>(terms, nparts, batch, status, eps, err_terms);
+    ISPA_TRY(cudaGetLastError());
+
+    if (w_new) {
+        if (wt == ElemType::BF16) add_delta_kernel<bf16><<<dim3(fill_blocks, batch), 256, 0, s>>>(W, dW, *w_new, n);
+        else add_delta_kernel<float><<<dim3(fill_blocks, batch), 256, 0, s>>>(W, dW, *w_new, n);
+        ISPA_TRY(cudaGetLastError());
+    }
+    return cudaSuccess;
+}
+
+}  // namespace ispa

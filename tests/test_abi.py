@@ -1,0 +1,82 @@
+"""The C-ABI library: it loads, exports every symbol the header declares, and its host-only
+logic (argument checks, workspace sizing, layer selection) behaves. No GPU is touched."""
+import ctypes
+import json
+import math
+import os
+import re
+
+import pytest
+
+from streaming_video_attention_b200 import ispa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(ispa_[a-z_0-9]+)\s*\(", src))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_symbol():
+    L = ispa.lib()
+    declared = _declared_symbols()
+    assert len(declared) >= 11
+    for name in declared:
+        assert hasattr(L, name), name
+    assert set(declared) == set(ispa.EXPORTS)
+    assert b"sm_100a" in L.ispa_version()
+
+
+def test_invalid_arguments_are_rejected_before_any_launch():
+    L = ispa.lib()
+    assert L.ispa_attn_split(None, None, None, None, None, None, None, None, None, None, None, None, 0,
+                             None) == ispa.ISPA_ERR_INVALID_ARG
+    assert b"desc" in L.ispa_last_error()
+    d = ispa.make_desc(128, 64, 2, 96)
+    assert L.ispa_attn_split(ctypes.byref(d), None, None, None, None, None, None, None, None, None, None, None, 0,
+                             None) == ispa.ISPA_ERR_UNSUPPORTED
+    d = ispa.make_desc(128, 64, 2, 64, sink=(0, 40), chunk=(30, 64))
+    assert L.ispa_attn_split(ctypes.byref(d), None, None, None, None, None, None, None, None, None, None, None, 0,
+                             None) == ispa.ISPA_ERR_INVALID_ARG
+    assert b"overlap" in L.ispa_last_error()
+    d = ispa.make_desc(128, 64, 2, 64, sink=(0, 70), chunk=(0, 0))
+    assert L.ispa_attn_split(ctypes.byref(d), None, None, None, None, None, None, None, None, None, None, None, 0,
+                             None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_select_layers(None, 3, 1, None, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_selftest_bounded_wait(0, None) == ispa.ISPA_ERR_INVALID_ARG
+
+
+def test_workspace_sizes():
+    d = ispa.make_desc(4680, 37440, 12, 128, dtype=ispa.ISPA_BF16)
+    # fused statistics need the A_loc and R operands: 2 * n_q * D bf16
+    assert ispa.workspace_bytes(d, 0, 0) >= 2 * 4680 * 1536 * 2
+    # the solve needs three D x D float32 matrices per layer in a batch
+    assert ispa.workspace_bytes(None, 30, 1536) >= 30 * 3 * 1536 * 1536 * 4
+
+
+def test_select_layers_golden():
+    with open(os.path.join(ROOT, "tests", "golden", "selection_examples.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        eps = [math.nan if e == "nan" else e for e in c["eps"]]
+        idx, flags = ispa.ispa_select_layers(eps, c["K"])
+        assert idx == c["idx"], c
+        assert flags == c["is_local"], c
+
+
+def test_select_layers_matches_oracle_on_random_errors():
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(5)
+    for trial in range(50):
+        L = int(rng.integers(1, 60))
+        eps = rng.choice([0.1, 0.2, 0.3], size=L) if trial % 2 else rng.random(L)
+        eps = eps.astype(np.float32).tolist()
+        K = int(rng.integers(0, L + 2))
+        assert ispa.ispa_select_layers(eps, K) == oracle.select_layers(eps, K)

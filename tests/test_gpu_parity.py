@@ -1,0 +1,257 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the CPU oracle on the same
+seeded inputs.
+
+Tolerances (written per check below):
+  * float32 workloads: 1e-5 relative Frobenius norm per tensor (attention, statistics);
+    the absorb solve 1e-3 relative Frobenius (the float32 Cholesky against a float64 LU).
+  * bf16 workloads: attention outputs 2e-2 relative Frobenius per tensor, lse within
+    2e-2 absolute; statistics from identical bf16 operands 1e-5 relative; statistics
+    fused behind bf16 attention 2e-2 relative (they inherit the attention's rounding).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from streaming_video_attention_b200 import ispa
+from tests.helpers import rel_fro, to_device, to_numpy, torch_dtype
+
+pytestmark = pytest.mark.gpu
+
+ATTN_TOL = {"fp32": 1e-5, "bf16": 2e-2}
+LSE_TOL = {"fp32": 1e-5, "bf16": 2e-2}
+
+
+def _attn_case(seed, n_q, n_kv, heads, hd, dtype):
+    q = synth.normal_tensor(seed, (1,), (n_q, heads, hd), dtype)
+    k = synth.normal_tensor(seed, (2,), (n_kv, heads, hd), dtype)
+    v = synth.normal_tensor(seed, (3,), (n_kv, heads, hd), dtype)
+    return q, k, v
+
+
+def _run_split(q, k, v, sink, chunk, dtype, stats=None):
+    n_q, heads, hd = q.shape
+    n_kv = k.shape[0]
+    td = torch_dtype(dtype)
+    code = ispa.ISPA_BF16 if dtype == "bf16" else ispa.ISPA_FP32
+    desc = ispa.make_desc(n_q, n_kv, heads, hd, sink, chunk, dtype=code)
+    Q, K, V = to_device(q, dtype), to_device(k, dtype), to_device(v, dtype)
+    outs = {n: torch.full((n_q, heads, hd), float("nan"), dtype=td, device="cuda") for n in ("full", "loc", "hist")}
+    lses = {n: torch.full((heads, n_q), float("nan"), dtype=torch.float32, device="cuda") for n in ("full", "loc", "hist")}
+    ws = ispa.alloc_workspace(ispa.workspace_bytes(desc, 0, 0)) if stats is not None else None
+    ispa.ispa_attn_split(desc, Q, K, V, outs["full"], lses["full"], outs["loc"], lses["loc"], outs["hist"],
+                         lses["hist"], stats=stats, ws=ws)
+    torch.cuda.synchronize()
+    assert ispa.ispa_device_status() == ispa.ISPA_OK
+    return {("A_" + n): to_numpy(outs[n]) for n in outs} | {("lse_" + n): to_numpy(lses[n]) for n in lses}
+
+
+def _check_attn(got, want, dtype, names=("full", "loc", "hist")):
+    for n in names:
+        err = rel_fro(got["A_" + n], want["A_" + n])
+        assert err < ATTN_TOL[dtype], (n, err)
+        lw, lg = want["lse_" + n], got["lse_" + n]
+        fin = np.isfinite(lw)
+        assert np.array_equal(fin, np.isfinite(lg)), n
+        if fin.any():
+            assert np.max(np.abs(lg[fin] - lw[fin])) < LSE_TOL[dtype], n
+        assert np.all(lg[~fin] == -np.inf), n
+
+
+# ------------------------------------------------------------------ attention (a1)
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("hd", [64, 128])
+@pytest.mark.parametrize("layout", ["sink_hist_chunk", "no_history", "no_sink", "chunk_inside"])
+def test_split_attention_matches_oracle(dtype, hd, layout):
+    tpf, heads = 200, 2
+    n_q = 3 * tpf                                   # 600 = 4 full 128-row tiles + a ragged 88
+    if layout == "sink_hist_chunk":
+        n_kv, sink, chunk = 8 * tpf, (0, tpf), (5 * tpf, 8 * tpf)
+    elif layout == "no_history":
+        n_kv, sink, chunk = 4 * tpf, (0, tpf), (tpf, 4 * tpf)
+    elif layout == "no_sink":
+        n_kv, sink, chunk = 7 * tpf + 37, (0, 0), (4 * tpf + 37, 7 * tpf + 37)
+    else:
+        n_kv, sink, chunk = 9 * tpf + 5, (3, 3 + tpf), (2 * tpf + 50, 5 * tpf + 50)
+    q, k, v = _attn_case(11 + hd, n_q, n_kv, heads, hd, dtype)
+    got = _run_split(q, k, v, sink, chunk, dtype)
+    want = oracle.split_attention(q, k, v, sink, chunk, 1 / math.sqrt(hd))
+    _check_attn(got, want, dtype)
+
+
+def test_split_attention_edge_sizes():
+    # a single query row, a single history row, and one KV tile with a 1-row tail
+    for (n_q, n_kv, sink, chunk) in [(1, 130, (0, 1), (2, 130)), (129, 129, (0, 64), (65, 129)), (5, 3, (0, 1), (1, 3))]:
+        q, k, v = _attn_case(99, n_q, n_kv, 2, 128, "bf16")
+        got = _run_split(q, k, v, sink, chunk, "bf16")
+        want = oracle.split_attention(q, k, v, sink, chunk, 1 / math.sqrt(128))
+        _check_attn(got, want, "bf16")
+
+
+# ------------------------------------------------------------------ statistics (a2)
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_accum_stats_matches_oracle_on_identical_operands(dtype):
+    n, D = 777, 256
+    a_loc = synth.normal_tensor(7, (10,), (n, D), dtype, std=0.05)
+    a_full = synth.normal_tensor(7, (11,), (n, D), dtype, std=0.05)
+    st = ispa.Stats(D)
+    ws = ispa.alloc_workspace(ispa.workspace_bytes(None, n, D))
+    code = ispa.ISPA_BF16 if dtype == "bf16" else ispa.ISPA_FP32
+    A, F = to_device(a_loc, dtype), to_device(a_full, dtype)
+    # two calls: accumulation adds up
+    ispa.ispa_accum_stats(st, A[:400], F[:400], 400, code, ws=ws)
+    ispa.ispa_accum_stats(st, A[400:], F[400:], n - 400, code, ws=ws)
+    torch.cuda.synchronize()
+    ref = oracle.stats_init(D)
+    oracle.stats_update(ref, a_loc.astype(np.float64), a_full.astype(np.float64), dtype)
+    for name in ("G", "C", "H"):
+        assert rel_fro(to_numpy(getattr(st, name)), ref[name]) < 1e-5, name
+    assert int(st.rows.item()) == n
+    ispa.ispa_stats_reset(st)
+    torch.cuda.synchronize()
+    assert float(st.G.abs().sum()) == 0 and int(st.rows.item()) == 0
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_fused_stats_match_oracle(dtype):
+    tpf, heads, hd = 200, 2, 128
+    n_q, n_kv, sink, chunk = 3 * tpf, 8 * tpf, (0, tpf), (5 * tpf, 8 * tpf)
+    q, k, v = _attn_case(5, n_q, n_kv, heads, hd, dtype)
+    st = ispa.Stats(heads * hd)
+    got = _run_split(q, k, v, sink, chunk, dtype, stats=st)
+    want = oracle.split_attention(q, k, v, sink, chunk, 1 / math.sqrt(hd))
+    _check_attn(got, want, dtype)
+    ref = oracle.stats_init(heads * hd)
+    oracle.stats_update(ref, want["A_loc"], want["A_full"], dtype)
+    tol = 1e-5 if dtype == "fp32" else 2e-2
+    for name in ("G", "C", "H"):
+        assert rel_fro(to_numpy(getattr(st, name)), ref[name]) < tol, name
+    assert int(st.rows.item()) == n_q
+
+
+# ------------------------------------------------------------------ solve, error, selection (a3-a5)
+def _oracle_stats_for(cfg_dtype, seed, n, D, planted=False):
+    a = synth.normal_tensor(seed, (20,), (n, D), cfg_dtype, std=0.05).astype(np.float64)
+    if planted:
+        P = synth.normal_tensor(seed, (21,), (D, D), "fp32", std=1.0 / math.sqrt(D)).astype(np.float64)
+        r = a @ P + 0.01 * synth.normal_tensor(seed, (22,), (n, D), cfg_dtype, std=0.05)
+    else:
+        r = synth.normal_tensor(seed, (23,), (n, D), cfg_dtype, std=0.05).astype(np.float64)
+    st = oracle.stats_init(D)
+    oracle.stats_update(st, a.reshape(n, -1, 64), (a + r).reshape(n, -1, 64), cfg_dtype)
+    return st
+
+
+@pytest.mark.parametrize("dtype,D,L", [("fp32", 128, 1), ("bf16", 256, 3), ("bf16", 1536, 2)])
+def test_solve_absorb_matches_oracle(dtype, D, L):
+    lam = 1e-2
+    n = max(2 * D, 512)
+    stats_np = [_oracle_stats_for(dtype, 40 + l, n, D, planted=(l % 2 == 0)) for l in range(L)]
+    W_np = [synth.normal_tensor(50 + l, (30,), (D, D), dtype, std=1 / math.sqrt(D)) for l in range(L)]
+    stats = []
+    for s in stats_np:
+        st = ispa.Stats(D)
+        st.G.copy_(torch.from_numpy(s["G"].astype(np.float32)))
+        st.C.copy_(torch.from_numpy(s["C"].astype(np.float32)))
+        st.H.copy_(torch.from_numpy(s["H"].astype(np.float32)))
+        st.rows.fill_(s["rows"])
+        stats.append(st)
+    Ws = [to_device(w, dtype) for w in W_np]
+    W_new = [torch.empty_like(w) for w in Ws]
+    dW = torch.full((L, D, D), float("nan"), device="cuda")
+    eps = torch.full((L,), float("nan"), device="cuda")
+    terms = torch.zeros((L, 2), dtype=torch.float64, device="cuda")
+    status = torch.full((L,), 7, dtype=torch.int32, device="cuda")
+    ws = ispa.alloc_workspace(ispa.workspace_bytes(None, L, D))
+    code = ispa.ISPA_BF16 if dtype == "bf16" else ispa.ISPA_FP32
+    ispa.ispa_solve_absorb(stats, Ws, code, lam, dW, eps, terms, W_new, status, ws)
+    torch.cuda.synchronize()
+    assert status.tolist() == [0] * L
+    eps_ref = []
+    for l in range(L):
+        # the oracle solves from the float32 statistics the GPU was given
+        G = stats_np[l]["G"].astype(np.float32).astype(np.float64)
+        C = stats_np[l]["C"].astype(np.float32).astype(np.float64)
+        H = stats_np[l]["H"].astype(np.float32).astype(np.float64)
+        dW_ref = oracle.absorb_solve(G, C, W_np[l], lam)
+        assert rel_fro(to_numpy(dW[l]), dW_ref) < 1e-3, l
+        e = oracle.reconstruction_error(G, C, H, W_np[l], dW_ref)
+        eps_ref.append(e["eps"])
+        assert abs(float(eps[l]) - e["eps"]) <= 1e-3 * abs(e["eps"]) + 1e-6, (l, float(eps[l]), e["eps"])
+        assert abs(float(terms[l, 1]) - e["T2"]) <= 1e-4 * abs(e["T2"])
+        wn_ref = W_np[l].astype(np.float64) + dW_ref
+        assert rel_fro(to_numpy(W_new[l]), wn_ref) < (1e-5 if dtype == "fp32" else 1e-2)
+    # selection: identical on the same eps, and on the oracle's own eps
+    eps_gpu = eps.cpu().tolist()
+    assert ispa.ispa_select_layers(eps_gpu, 1) == oracle.select_layers(eps_gpu, 1)
+    assert ispa.ispa_select_layers(eps_gpu, 1)[0] == oracle.select_layers(eps_ref, 1)[0]
+
+
+def test_solve_reports_non_spd_layers():
+    D = 128
+    st_bad, st_ok = ispa.Stats(D), ispa.Stats(D)
+    st_bad.G.copy_(-torch.eye(D))
+    st_ok.G.copy_(torch.eye(D))
+    W = [torch.eye(D, device="cuda"), torch.eye(D, device="cuda")]
+    dW = torch.zeros((2, D, D), device="cuda")
+    eps = torch.zeros(2, device="cuda")
+    status = torch.zeros(2, dtype=torch.int32, device="cuda")
+    ws = ispa.alloc_workspace(ispa.workspace_bytes(None, 2, D))
+    ispa.ispa_solve_absorb([st_bad, st_ok], W, ispa.ISPA_FP32, 0.0, dW, eps, None, None, status, ws)
+    torch.cuda.synchronize()
+    assert status.tolist() == [ispa.ISPA_ERR_NOT_SPD, 0]
+    assert math.isnan(float(eps[0])) and float(eps[1]) == 0.0
+    assert bool(torch.isnan(dW[0]).all()) and float(dW[1].abs().max()) == 0.0
+
+
+# ------------------------------------------------------------------ local attention (a6)
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_local_attention_and_projection(dtype):
+    n_q, n_loc, heads, hd = 600, 800, 2, 128
+    q, k, v = _attn_case(77, n_q, n_loc, heads, hd, dtype)
+    D = heads * hd
+    W = synth.normal_tensor(78, (1,), (D, D), dtype, std=1 / math.sqrt(D))
+    code = ispa.ISPA_BF16 if dtype == "bf16" else ispa.ISPA_FP32
+    desc = ispa.make_desc(n_q, n_loc, heads, hd, dtype=code)
+    td = torch_dtype(dtype)
+    o = torch.empty((n_q, heads, hd), dtype=td, device="cuda")
+    lse = torch.empty((heads, n_q), device="cuda")
+    y = torch.empty((n_q, D), dtype=td, device="cuda")
+    Wd = to_device(W, dtype)
+    ispa.ispa_local_attn(desc, to_device(q, dtype), to_device(k, dtype), to_device(v, dtype), o, lse, Wd, y)
+    torch.cuda.synchronize()
+    A, L = oracle.local_attention(q, k, v, 1 / math.sqrt(hd))
+    assert rel_fro(to_numpy(o), A) < ATTN_TOL[dtype]
+    assert np.max(np.abs(to_numpy(lse) - L)) < LSE_TOL[dtype]
+    assert rel_fro(to_numpy(y), oracle.project(A, W)) < ATTN_TOL[dtype]
+
+
+# ------------------------------------------------------------------ full size, sampled rows
+def test_full_size_1p3b_layer_sampled_rows():
+    """One 1.3B-shaped layer call at the last warmup chunk (n_q 4680, n_kv 37440, 12 heads),
+    in the launch configuration the benchmark times (fused statistics). Sampled query rows
+    go to the oracle; the statistics are checked by properties that hold at any size."""
+    cfg = synth.CONFIGS["1p3b_bf16"]
+    t, layer = cfg.warmup_chunks - 1, 3
+    frames = synth.cache_frames(cfg, t)
+    lay = synth.chunk_layout(cfg, frames, t)
+    q = synth.chunk_q(cfg, layer, t)
+    k = synth.kv_tensor(cfg, layer, frames, "k")
+    v = synth.kv_tensor(cfg, layer, frames, "v")
+    assert k.shape[0] == 37440
+    st = ispa.Stats(cfg.D)
+    sink, chunk = (lay["sink_begin"], lay["sink_end"]), (lay["chunk_begin"], lay["chunk_end"])
+    got = _run_split(q, k, v, sink, chunk, "bf16", stats=st)
+    rows = np.unique(np.concatenate([np.arange(0, 4680, 97), np.arange(4600, 4680, 7), [127, 128, 4679]]))
+    want = oracle.split_attention(q[rows], k, v, sink, chunk, cfg.scale)
+    sub = {n: (got[n][rows] if n.startswith("A_") else got[n][:, rows]) for n in got}
+    _check_attn(sub, want, "bf16")
+    G, H = to_numpy(st.G), to_numpy(st.H)
+    assert int(st.rows.item()) == cfg.n_q
+    assert rel_fro(G, G.T) < 1e-6 and rel_fro(H, H.T) < 1e-6
+    assert np.all(np.diag(G) >= 0) and np.all(np.diag(H) >= 0)
+    a = got["A_loc"].reshape(cfg.n_q, -1)
+    assert abs(np.trace(G) - np.sum(a * a)) < 1e-4 * np.sum(a * a)
