@@ -70,6 +70,14 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
 }
 
 // ---- misc ---------------------------------------------------------------------------
+// 2^x with the hardware approximation (MUFU.EX2), flush-to-zero; used for softmax weights
+// that are rounded to bf16 right after.
+__device__ __forceinline__ float exp2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ bool elect_one() {
     uint32_t pred;
     asm volatile(

@@ -1,20 +1,265 @@
-// Ridge statistics from bf16 operands (placeholder routing to the CUDA-core GEMM until the
-// tcgen05 GEMM lands).
+// Ridge statistics on the sm_100a tensor cores [ISPA §3.2; notes: Method]:
+//   G += A^T A,  C += A^T R,  H += R^T R
+// from the bf16 operands A = A_loc and R = A_full - A_loc, each [n, D] row-major (the
+// layout the split-attention epilogue writes), accumulated in float32.
+//
+// One CTA owns one 128x128 output tile and reduces over all n token rows in a fixed
+// order (no atomics: results repeat bit for bit). G and H are symmetric: only tiles on or
+// above the block diagonal are computed, and each is written to both mirrored positions,
+// so the stored G and H are exactly symmetric.
+//
+// Both MMA operands are "MN-major" slices of [n, D]: a TMA box of 64 token rows x 64
+// columns (128-byte swizzle) puts 64 columns of one token in each 128-byte row, with
+// consecutive tokens (the reduction index) 128 bytes apart. 256 threads: warp 0 TMA,
+// warp 1 MMA (lane 0), warps 4..7 epilogue (read-modify-write of the float32 tile).
+#include <cuda.h>
+
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace ispa {
+namespace {
+
+constexpr int kTile = 128;         // output tile (both dimensions)
+constexpr int kKRows = 64;         // token rows per stage
+constexpr int kStages = 3;
+constexpr int kThreads = 256;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr int kOperandBytes = kKRows * kTile * 2;          // 16 KB: two 64x64 boxes
+constexpr int kStageBytes = 2 * kOperandBytes;
+constexpr int kBarOff = kStages * kStageBytes;
+constexpr int kSmemAlloc = kBarOff + 256 + 1024;
+
+struct StatsParams {
+    float *out[3];      // G, C, H
+    int D, n;
+    int nb;             // D / 128
+    int n_sym;          // upper-triangle tiles per symmetric matrix: nb*(nb+1)/2
+    int *err_flag;
+};
+
+// Work item -> (matrix, tile row bi, tile column bj). Items 0..n_sym-1: G, then C (nb*nb),
+// then H (n_sym).
+__device__ __forceinline__ void decode_item(int item, int nb, int n_sym, int &mat, int &bi, int &bj) {
+    int t;
+    if (item < n_sym) { mat = 0; t = item; }
+    else if (item < n_sym + nb * nb) { mat = 1; bi = (item - n_sym) / nb; bj = (item - n_sym) % nb; return; }
+    else { mat = 2; t = item - n_sym - nb * nb; }
+    // t-th upper-triangle tile in row-major order
+    int r = 0;
+    while (t >= nb - r) { t -= nb - r; ++r; }
+    bi = r;
+    bj = r + t;
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+stats_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmR,
+                        const StatsParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kBarOff);
+    uint64_t *empty = full + kStages;
+    uint64_t *acc_bar = empty + kStages;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_bar + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    int mat, bi, bj;
+    decode_item(blockIdx.x, p.nb, p.n_sym, mat, bi, bj);
+    const CUtensorMap *mapA = (mat == 2) ? &tmR : &tmA;   // left operand: A for G and C, R for H
+    const CUtensorMap *mapB = (mat == 0) ? &tmA : &tmR;   // right operand: A for G, R for C and H
+    const int n_k = (p.n + kKRows - 1) / kKRows;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&empty[s], 1);
+        }
+        ptx::mbar_init(acc_bar, 1);
+        *abort_flag = 0;
+        ptx::fence_barrier_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, 128);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            ptx::tma_prefetch_desc(mapA);
+            ptx::tma_prefetch_desc(mapB);
+            const uint64_t pol = ptx::policy_evict_last();
+            int issued = -1;
+            bool ok = true;
+            for (int kt = 0; kt < n_k && ok; ++kt) {
+                const int s = kt % kStages;
+                const uint32_t ph = (kt / kStages) & 1;
+                ok = ptx::mbar_wait_bounded(&empty[s], ph ^ 1, kWaitLimitNs, p.err_flag, abort_flag);
+                if (!ok) break;
+                uint8_t *base = smem + s * kStageBytes;
+                ptx::mbar_arrive_expect_tx(&full[s], kStageBytes);
+                for (int b = 0; b < 2; ++b) {
+                    ptx::tma_load_2d(base + b * (kKRows * 128), mapA, &full[s], bi * kTile + b * 64, kt * kKRows, pol);
+                    ptx::tma_load_2d(base + kOperandBytes + b * (kKRows * 128), mapB, &full[s], bj * kTile + b * 64,
+                                     kt * kKRows, pol);
+                }
+                issued = kt;
+            }
+            if (!ok) {
+                for (int kt = (issued - kStages + 1 > 0 ? issued - kStages + 1 : 0); kt <= issued; ++kt)
+                    ptx::mbar_wait_bounded(&full[kt % kStages], (kt / kStages) & 1, kWaitLimitNs, nullptr, nullptr);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = ptx::make_idesc_bf16(kTile, kTile, true, true);
+            const uint32_t sbase = ptx::smem_u32(smem);
+            bool ok = true;
+            for (int kt = 0; kt < n_k && ok; ++kt) {
+                const int s = kt % kStages;
+                ok = ptx::mbar_wait_bounded(&full[s], (kt / kStages) & 1, kWaitLimitNs, p.err_flag, abort_flag);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const uint32_t a0 = sbase + s * kStageBytes;
+                const uint32_t b0 = a0 + kOperandBytes;
+#pragma unroll
+                for (int kk = 0; kk < kKRows / 16; ++kk) {
+                    const uint64_t da = ptx::make_sdesc_sw128(a0 + kk * 2048, kKRows * 128, 1024);
+                    const uint64_t db = ptx::make_sdesc_sw128(b0 + kk * 2048, kKRows * 128, 1024);
+                    ptx::umma_f16_ss(tmem, da, db, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+                }
+                ptx::umma_commit(&empty[s]);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                __threadfence_block();
+            }
+            ptx::umma_commit(acc_bar);
+            ptx::mbar_wait_bounded(acc_bar, 0, kWaitLimitNs, p.err_flag, nullptr);
+        }
+    } else if (warp >= 4) {
+        const int wq = warp - 4;
+        const int r = wq * 32 + lane;                   // row inside the tile
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        const bool ok = ptx::mbar_wait_bounded(acc_bar, 0, kWaitLimitNs, p.err_flag, abort_flag) && !*abort_flag;
+        if (ok) {
+            ptx::tc_fence_after();
+            float *M = p.out[mat];
+            const size_t D = p.D;
+            const int gi = bi * kTile + r;
+            const bool sym = (mat != 1);
+            const bool diag = sym && bi == bj;
+#pragma unroll 1
+            for (int c = 0; c < kTile / 32; ++c) {
+                uint32_t v[32];
+                ptx::tmem_ld32(tmem + lane_off + c * 32, v);
+                ptx::tmem_wait_ld();
+                const int gj0 = bj * kTile + c * 32;
+                float *rowp = M + (size_t)gi * D + gj0;
+                if (!diag) {
+#pragma unroll
+                    for (int q = 0; q < 32; q += 4) {
+                        float4 o = *reinterpret_cast<const float4 *>(rowp + q);
+                        o.x += __uint_as_float(v[q]);
+                        o.y += __uint_as_float(v[q + 1]);
+                        o.z += __uint_as_float(v[q + 2]);
+                        o.w += __uint_as_float(v[q + 3]);
+                        *reinterpret_cast<float4 *>(rowp + q) = o;
+                        if (sym) {
+                            M[(size_t)(gj0 + q) * D + gi] = o.x;
+                            M[(size_t)(gj0 + q + 1) * D + gi] = o.y;
+                            M[(size_t)(gj0 + q + 2) * D + gi] = o.z;
+                            M[(size_t)(gj0 + q + 3) * D + gi] = o.w;
+                        }
+                    }
+                } else {
+                    // diagonal tile: the upper triangle (j >= i) is updated and mirrored
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) {
+                        const int gj = gj0 + q;
+                        if (gj >= gi) {
+                            const float o = rowp[q] + __uint_as_float(v[q]);
+                            rowp[q] = o;
+                            if (gj > gi) M[(size_t)gj * D + gi] = o;
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, 128);
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// [n, D] bf16 row-major, box = 64 rows x 64 columns, 128-byte swizzle.
+bool make_panel_map(CUtensorMap *m, const void *ptr, int n, int D) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)n};
+    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)kKRows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
 cudaError_t launch_stats_bf16(const void *a_loc, const void *r, int n, int D, float *G, float *C, float *H,
                               int *err_flag, cudaStream_t s) {
-    (void)err_flag;
-    GemmDesc g{D, D, n, D, D, D, false, false, ElemType::BF16, ElemType::BF16, ElemType::F32, 1.f, 1.f, false, 1};
-    GemmBatch b;
-    b.A[0] = a_loc; b.B[0] = a_loc; b.C[0] = G;
-    cudaError_t e = launch_gemm_simt(g, b, s);
+    if (n <= 0) return cudaSuccess;
+    if (D % kTile != 0) {
+        // D not a multiple of 128 (e.g. 64-wide single head): CUDA-core GEMM
+        GemmDesc g{D, D, n, D, D, D, false, false, ElemType::BF16, ElemType::BF16, ElemType::F32, 1.f, 1.f, false, 1};
+        GemmBatch b;
+        b.A[0] = a_loc; b.B[0] = a_loc; b.C[0] = G;
+        cudaError_t e = launch_gemm_simt(g, b, s);
+        if (e != cudaSuccess) return e;
+        b.A[0] = a_loc; b.B[0] = r; b.C[0] = C;
+        e = launch_gemm_simt(g, b, s);
+        if (e != cudaSuccess) return e;
+        b.A[0] = r; b.B[0] = r; b.C[0] = H;
+        return launch_gemm_simt(g, b, s);
+    }
+    CUtensorMap ma, mr;
+    if (!make_panel_map(&ma, a_loc, n, D) || !make_panel_map(&mr, r, n, D)) return cudaErrorInvalidValue;
+    StatsParams p;
+    p.out[0] = G; p.out[1] = C; p.out[2] = H;
+    p.D = D; p.n = n;
+    p.nb = D / kTile;
+    p.n_sym = p.nb * (p.nb + 1) / 2;
+    p.err_flag = err_flag;
+    cudaError_t e = cudaFuncSetAttribute(stats_gemm_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
     if (e != cudaSuccess) return e;
-    b.A[0] = a_loc; b.B[0] = r; b.C[0] = C;
-    e = launch_gemm_simt(g, b, s);
-    if (e != cudaSuccess) return e;
-    b.A[0] = r; b.B[0] = r; b.C[0] = H;
-    return launch_gemm_simt(g, b, s);
+    const int items = 2 * p.n_sym + p.nb * p.nb;
+    stats_gemm_sm100_kernel<<<items, kThreads, kSmemAlloc, s>>>(ma, mr, p);
+    return cudaGetLastError();
 }
+
 }  // namespace ispa
