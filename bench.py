@@ -1,0 +1,491 @@
+#!/usr/bin/env python
+"""Benchmark of the ISPA warmup hot path on B200.
+
+One step = one streaming episode of the 1.3B-shaped workload on every GPU (replicas):
+  * 3 warmup chunks x 30 layers of split attention with fused ridge statistics
+    (history 15, 18, 21 frames: n_kv = 28,080 / 32,760 / 37,440 rows, n_q = 4,680),
+  * the transition: absorb solve + reconstruction error for 30 layers (D = 1536),
+    selection of K = 15 L-layers on the host, W_new = W + dW,
+  * one post-transition chunk: 15 L-layers of local attention (sink + chunk, 6,240 rows)
+    with the W_new projection, 15 F-layers of full attention (sink + 20 frames + chunk).
+value = query tokens through the model per second = (4 chunks x 4,680 queries x N GPUs) /
+step time (max over ranks). Inputs are seeded synthetic tensors (same recipe as the
+oracle tests), resident in HBM before the timed region; ~20 GB are touched per step, far
+more than L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ispa|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures as cf
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "query tokens/s through split attention+absorb stats; % of BF16 tensor peak"
+UNIT = "query tokens/s"
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ispa", "reference"], default="ispa")
+    ap.add_argument("--config", default="1p3b_bf16")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=512)
+    return ap.parse_args(argv)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("bf16_tflops"), d.get("bf16_tflops_sustained"), d.get("hbm_gbs"), "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+# --------------------------------------------------------------------------- workload
+class Workload:
+    """Host (pinned) and device copies of one episode's inputs."""
+
+    def __init__(self, cfg: synth.IspaConfig, threads: int):
+        self.cfg = cfg
+        W = cfg.warmup_chunks
+        self.post_t = W
+        self.n_frames = cfg.chunk_start_frame(W) + cfg.chunk_frames       # frames 0 .. last post-chunk frame
+        tpf, h, d = cfg.tpf, cfg.heads, cfg.head_dim
+        L = cfg.layers
+        self.kv_host = [[torch.empty((self.n_frames * tpf, h, d), dtype=torch.bfloat16, pin_memory=True)
+                         for _ in range(2)] for _ in range(L)]
+        self.q_host = [torch.empty((W + 1, cfg.n_q, h, d), dtype=torch.bfloat16, pin_memory=True) for _ in range(L)]
+        self.w_host = [torch.empty((cfg.D, cfg.D), dtype=torch.bfloat16, pin_memory=True) for _ in range(L)]
+
+        def bits(t):
+            return t.view(torch.int16).numpy().view(np.uint16)
+
+        def fill_frame(l, f, which):
+            x = synth.frame_kv(cfg, l, f, which)
+            bits(self.kv_host[l][0 if which == "k" else 1])[f * tpf:(f + 1) * tpf] = synth.bf16_bits_from_f32(x)
+
+        def fill_q(l, t):
+            bits(self.q_host[l])[t] = synth.bf16_bits_from_f32(synth.chunk_q(cfg, l, t))
+
+        def fill_w(l):
+            bits(self.w_host[l])[:] = synth.bf16_bits_from_f32(synth.w_out(cfg, l))
+
+        jobs = [(fill_frame, (l, f, wh)) for l in range(L) for f in range(self.n_frames) for wh in ("k", "v")]
+        jobs += [(fill_q, (l, t)) for l in range(L) for t in range(W + 1)]
+        jobs += [(fill_w, (l,)) for l in range(L)]
+        with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(lambda j: j[0](*j[1]), jobs))
+
+        # per-chunk KV geometry
+        self.warm = []
+        for t in range(W):
+            fr = synth.cache_frames(cfg, t)
+            lay = synth.chunk_layout(cfg, fr, t)
+            assert fr == list(range(len(fr))), "warmup caches are contiguous frame prefixes"
+            self.warm.append(lay)
+        self.post_frames = synth.cache_frames(cfg, self.post_t)
+        self.post_layout = synth.chunk_layout(cfg, self.post_frames, self.post_t)
+        s0 = cfg.chunk_start_frame(self.post_t)
+        self.local_frames = list(range(cfg.sink_frames)) + list(range(s0, s0 + cfg.chunk_frames))
+
+    def h2d_bytes(self) -> int:
+        b = 0
+        for l in range(self.cfg.layers):
+            b += sum(t.numel() * 2 for t in self.kv_host[l]) + self.q_host[l].numel() * 2 + self.w_host[l].numel() * 2
+        return b
+
+
+class DeviceInputs:
+    def __init__(self, wl: Workload, device):
+        cfg = wl.cfg
+        tpf = cfg.tpf
+        L = cfg.layers
+        self.wl = wl
+        self.kv = [[torch.empty_like(wl.kv_host[l][i], device=device) for i in range(2)] for l in range(L)]
+        self.q = [torch.empty_like(wl.q_host[l], device=device) for l in range(L)]
+        self.w = [torch.empty_like(wl.w_host[l], device=device) for l in range(L)]
+        n_post, n_loc = len(wl.post_frames) * tpf, len(wl.local_frames) * tpf
+        h, d = cfg.heads, cfg.head_dim
+        self.kv_post = [[torch.empty((n_post, h, d), dtype=torch.bfloat16, device=device) for _ in range(2)]
+                        for _ in range(L)]
+        self.kv_loc = [[torch.empty((n_loc, h, d), dtype=torch.bfloat16, device=device) for _ in range(2)]
+                       for _ in range(L)]
+
+    def upload(self, stream=None):
+        """Host -> device copies of the step's inputs, then the derived post-transition caches."""
+        wl = self.wl
+        for l in range(wl.cfg.layers):
+            for i in range(2):
+                self.kv[l][i].copy_(wl.kv_host[l][i], non_blocking=True)
+            self.q[l].copy_(wl.q_host[l], non_blocking=True)
+            self.w[l].copy_(wl.w_host[l], non_blocking=True)
+        self.derive()
+
+    def derive(self):
+        wl = self.wl
+        tpf = wl.cfg.tpf
+        for l in range(wl.cfg.layers):
+            for i in range(2):
+                src = self.kv[l][i]
+                for dst, frames in ((self.kv_post[l][i], wl.post_frames), (self.kv_loc[l][i], wl.local_frames)):
+                    # frames are runs of consecutive indices: copy run by run
+                    pos = 0
+                    start = frames[0]
+                    prev = frames[0]
+                    for f in frames[1:] + [None]:
+                        if f is not None and f == prev + 1:
+                            prev = f
+                            continue
+                        n = prev - start + 1
+                        dst[pos * tpf:(pos + n) * tpf].copy_(src[start * tpf:(prev + 1) * tpf], non_blocking=True)
+                        pos += n
+                        if f is not None:
+                            start = prev = f
+
+
+class Outputs:
+    def __init__(self, cfg, device):
+        L = cfg.layers
+        self.o = [torch.empty((cfg.n_q, cfg.heads, cfg.head_dim), dtype=torch.bfloat16, device=device)
+                  for _ in range(L)]
+        self.lse = [torch.empty((cfg.heads, cfg.n_q), dtype=torch.float32, device=device) for _ in range(L)]
+        self.y = [torch.empty((cfg.n_q, cfg.D), dtype=torch.bfloat16, device=device) for _ in range(L)]
+
+
+def run_episode(sess, dev: DeviceInputs, out: Outputs, timers=None):
+    """One streaming episode: warmup chunks -> transition -> one post-transition chunk."""
+    cfg = dev.wl.cfg
+    sess.rewarm()
+    for t, lay in enumerate(dev.wl.warm):
+        n_kv = lay["n_kv"]
+        sink, chunk = (lay["sink_begin"], lay["sink_end"]), (lay["chunk_begin"], lay["chunk_end"])
+        for l in range(cfg.layers):
+            if timers is not None:
+                ev0 = torch.cuda.Event(enable_timing=True)
+                ev1 = torch.cuda.Event(enable_timing=True)
+                ev0.record()
+            sess.full_attention(l, dev.q[l][t], dev.kv[l][0][:n_kv], dev.kv[l][1][:n_kv], sink, chunk, out.o[l],
+                                out.lse[l], collect=True)
+            if timers is not None:
+                ev1.record()
+                timers.append((ev0, ev1, n_kv))
+    sess.transition()
+    t = dev.wl.post_t
+    lay = dev.wl.post_layout
+    sink, chunk = (lay["sink_begin"], lay["sink_end"]), (lay["chunk_begin"], lay["chunk_end"])
+    for l in range(cfg.layers):
+        if sess.is_local[l]:
+            sess.local_attention(l, dev.q[l][t], dev.kv_loc[l][0], dev.kv_loc[l][1], out.o[l], out.lse[l], out.y[l])
+        else:
+            sess.full_attention(l, dev.q[l][t], dev.kv_post[l][0], dev.kv_post[l][1], sink, chunk, out.o[l],
+                                out.lse[l], collect=False)
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.path = os.path.join("/tmp", f"ispa_clocks_{os.getpid()}_{gpu_index}.csv")
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(gpu_index)], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def physical_gpu_index(local_rank: int) -> int:
+    vis = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    if local_rank < len(vis) and vis[local_rank].isdigit():
+        return int(vis[local_rank])
+    return local_rank
+
+
+# --------------------------------------------------------------------------- CPU oracle sample
+def oracle_sample(cfg, rows: int):
+    """Time the oracle on a bounded sample: `rows` query rows of one layer's last warmup call
+    (split attention over explicit masks + statistics). Returns (seconds, threads, note)."""
+    import oracle
+    t = cfg.warmup_chunks - 1
+    frames = synth.cache_frames(cfg, t)
+    lay = synth.chunk_layout(cfg, frames, t)
+    q = synth.chunk_q(cfg, 0, t)[:rows]
+    k = synth.kv_tensor(cfg, 0, frames, "k")
+    v = synth.kv_tensor(cfg, 0, frames, "v")
+    t0 = time.perf_counter()
+    res = oracle.split_attention(q, k, v, (lay["sink_begin"], lay["sink_end"]), (lay["chunk_begin"], lay["chunk_end"]),
+                                 cfg.scale)
+    st = oracle.stats_init(cfg.D)
+    oracle.stats_update(st, res["A_loc"], res["A_full"], cfg.dtype)
+    dt = time.perf_counter() - t0
+    return dt, lay["n_kv"]
+
+
+def oracle_value(cfg, dt: float, rows: int, n_kv_sample: int, wl_calls) -> float:
+    """Extrapolate the sample to one episode (linear in query rows and KV rows per call) and
+    express it in the step's unit."""
+    est = 0.0
+    for n_kv in wl_calls:
+        est += dt * (cfg.n_q / rows) * (n_kv / n_kv_sample)
+    tokens = (cfg.warmup_chunks + 1) * cfg.n_q
+    return tokens / est
+
+
+def episode_calls(cfg):
+    calls = []
+    for t in range(cfg.warmup_chunks):
+        lay = synth.chunk_layout(cfg, synth.cache_frames(cfg, t), t)
+        calls += [lay["n_kv"]] * cfg.layers
+    post = synth.chunk_layout(cfg, synth.cache_frames(cfg, cfg.warmup_chunks), cfg.warmup_chunks)["n_kv"]
+    n_loc = (cfg.sink_frames + cfg.chunk_frames) * cfg.tpf
+    calls += [post] * (cfg.layers - cfg.K) + [n_loc] * cfg.K
+    return calls
+
+
+def cpu_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max((i.get("num_threads", 1) for i in info), default=os.cpu_count())
+    except Exception:
+        return os.cpu_count()
+
+
+# --------------------------------------------------------------------------- arms
+def reference_arm(args, cfg, rank):
+    if rank != 0:
+        return 0
+    calls = episode_calls(cfg)
+    rows = args.cpu_rows
+    for _ in range(args.warmup):
+        oracle_sample(cfg, max(8, rows // 8))
+    times = []
+    for _ in range(args.steps):
+        dt, nkv = oracle_sample(cfg, rows)
+        times.append(dt)
+    dt = sum(times) / len(times)
+    value = oracle_value(cfg, dt, rows, nkv, calls)
+    step_est_ms = (cfg.warmup_chunks + 1) * cfg.n_q / value * 1e3
+    cores = cpu_threads()
+    sample = (f"{rows} query rows of one layer's last warmup call (n_kv {nkv}), split attention over explicit "
+              f"masks + statistics in float64, extrapolated linearly in rows and KV rows to the episode")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_est_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(cfg, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_block(cfg, n):
+    return {
+        "workload": (f"{cfg.name}: ISPA episode, {cfg.layers} layers x {cfg.heads} heads x {cfg.head_dim}, "
+                     f"{cfg.tpf} tokens/frame, chunk {cfg.chunk_frames} frames ({cfg.n_q} queries), warmup history "
+                     f"{[len(synth.cache_frames(cfg, t)) - cfg.chunk_frames for t in range(cfg.warmup_chunks)]} "
+                     f"frames, transition (solve + error + select K={cfg.K}), 1 post-transition chunk"),
+        "layers": cfg.layers, "heads": cfg.heads, "head_dim": cfg.head_dim, "n_q": cfg.n_q,
+        "warmup_chunks": cfg.warmup_chunks, "K": cfg.K, "lambda": cfg.lam,
+        "l2": "inputs larger than L2 (about 20 GB touched per step)", "parallelism": f"replicas x{n}",
+    }
+
+
+def ispa_arm(args, cfg, rank, world, local_rank):
+    from streaming_video_attention_b200 import ispa
+    from streaming_video_attention_b200.session import IspaSession
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    ispa.lib()
+    threads = max(1, (os.cpu_count() or 8) // max(1, int(os.environ.get("LOCAL_WORLD_SIZE", world))))
+    t0 = time.time()
+    wl = Workload(cfg, threads)
+    gen_s = time.time() - t0
+    dev = DeviceInputs(wl, device)
+    dev.upload()
+    out = Outputs(cfg, device)
+    sess = IspaSession(cfg.layers, cfg.heads, cfg.head_dim, cfg.lam, cfg.K, "bf16", str(device))
+    sess.set_weights(dev.w)
+    sess.reserve(cfg.n_q)
+    torch.cuda.synchronize()
+
+    for _ in range(max(3, args.warmup)):
+        run_episode(sess, dev, out)
+    torch.cuda.synchronize()
+    assert ispa.ispa_device_status() == ispa.ISPA_OK
+
+    # ---- timed region: device-resident inputs
+    clocks = ClockSampler(physical_gpu_index(local_rank))
+    time.sleep(0.4)
+    timers = []
+    launches0 = ispa.ispa_kernel_launches()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        run_episode(sess, dev, out, timers)
+    e1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    launches = ispa.ispa_kernel_launches() - launches0
+    clk = clocks.stop()
+    elapsed = e0.elapsed_time(e1) / 1e3
+    t = torch.tensor([elapsed], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    elapsed = float(t.item())
+    tokens = world * args.steps * (cfg.warmup_chunks + 1) * cfg.n_q
+    value = tokens / elapsed
+    ms_per_step = elapsed / args.steps * 1e3
+
+    # roofline of the fused split-attention + statistics call (dominant kernel pair)
+    D = cfg.D
+    flops = 0.0
+    secs = 0.0
+    for ev0, ev1, n_kv in timers:
+        secs += ev0.elapsed_time(ev1) / 1e3
+        flops += 4.0 * cfg.n_q * n_kv * cfg.head_dim * cfg.heads + 4.0 * cfg.n_q * D * D
+    burst, sustained, hbm, peak_kind = peaks()
+    achieved = flops / secs / 1e12
+    roof = {"bound": "tensor", "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
+            "frac": achieved / sustained, "traffic": None,
+            "kernel": "ispa_attn_split with fused statistics (split attention + Gram GEMM)",
+            "peak_kind": f"{peak_kind} sustained bf16 (timed inside a long step)",
+            "frac_of_burst_peak": achieved / burst,
+            "per_call_ms": secs / max(1, len(timers)) * 1e3}
+
+    # ---- end to end through the public API, host buffers in the timed region
+    e2e = None
+    if not args.no_e2e:
+        host_o = [torch.empty_like(out.o[l], device="cpu").pin_memory() for l in range(cfg.layers)]
+        d2h = sum(o.numel() * 2 for o in host_o) + cfg.layers * 4
+        run_once = lambda: (dev.upload(), run_episode(sess, dev, out),
+                            [host_o[l].copy_(out.o[l], non_blocking=True) for l in range(cfg.layers)],
+                            sess.eps.cpu())
+        run_once()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record()
+        for _ in range(args.e2e_steps):
+            run_once()
+        f1.record()
+        torch.cuda.synchronize()
+        et = torch.tensor([f0.elapsed_time(f1) / 1e3], dtype=torch.float64, device=device)
+        if world > 1:
+            torch.distributed.all_reduce(et, op=torch.distributed.ReduceOp.MAX)
+        e2e = {"value": world * args.e2e_steps * (cfg.warmup_chunks + 1) * cfg.n_q / float(et.item()), "unit": UNIT,
+               "h2d_bytes_per_step": wl.h2d_bytes(), "d2h_bytes_per_step": d2h,
+               "ms_per_step": float(et.item()) / args.e2e_steps * 1e3}
+
+    assert ispa.ispa_device_status() == ispa.ISPA_OK
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, nkv = oracle_sample(cfg, args.cpu_rows)
+        cpu = {"value": oracle_value(cfg, dt, args.cpu_rows, nkv, episode_calls(cfg)), "unit": UNIT,
+               "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"{args.cpu_rows} query rows of one layer's last warmup call (n_kv {nkv}), float64 split "
+                         f"attention over explicit masks + statistics, {dt:.2f} s, extrapolated linearly in rows and "
+                         f"KV rows to the episode"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_block(cfg, world),
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches), "clocks": clk,
+            "selection": {"idx": sess.idx, "margin": sess.selection_margin()},
+            "input_generation_s": gen_s,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    cfg = synth.CONFIGS[args.config]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return reference_arm(args, cfg, rank)
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        return ispa_arm(args, cfg, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

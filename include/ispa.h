@@ -165,6 +165,10 @@ int ispa_device_status(ispa_stream_t stream);
  * returns. The GPU context stays usable. */
 int ispa_selftest_bounded_wait(unsigned limit_us, ispa_stream_t stream);
 
+/* ispa_kernel_launches -- number of kernels this library has launched in this process
+ * (every device, every stream), for accounting; never reset. */
+unsigned long long ispa_kernel_launches(void);
+
 /* ispa_last_error -- message of the last failing call on this host thread ("" if none). */
 const char *ispa_last_error(void);
 

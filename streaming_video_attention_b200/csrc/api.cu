@@ -1,6 +1,7 @@
 // C-ABI entry points of libispa: argument checks, workspace layout and dispatch to the
 // kernels. Every call enqueues on the caller's stream and allocates nothing.
 #include <algorithm>
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -17,6 +18,11 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
                         int nparts, int *status, float *eps, double *err_terms, const PtrBatch *w_new, int D,
                         float lambda, int batch, cudaStream_t s);
 }
+
+namespace ispa {
+static std::atomic<unsigned long long> g_launches{0};
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace ispa
 
 using namespace ispa;
 
@@ -157,7 +163,7 @@ int accumulate(const ispa_stats *st, const void *a_ops, const void *r_ops, int n
             CUDA_CHECK_RET(launch_gemm_simt(g, b, s), "stats GEMM H");
         }
     }
-    add_rows_kernel<<<1, 1, 0, s>>>(st->rows, n);
+    add_rows_kernel<<<1, 1, 0, s>>>(st->rows, n); note_launch();
     CUDA_CHECK_RET(cudaGetLastError(), "rows counter");
     return ISPA_OK;
 }
@@ -218,6 +224,8 @@ __global__ void bounded_wait_selftest_kernel(uint64_t limit_ns, int *flag) {
 extern "C" {
 
 const char *ispa_last_error(void) { return g_last_error.c_str(); }
+
+unsigned long long ispa_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char *ispa_version(void) { return "ispa-b200 0.1 (sm_100a)"; }
 
@@ -293,6 +301,7 @@ int ispa_accum_stats(const ispa_stats *stats, const void *a_loc, const void *a_f
             residual_kernel<bf16><<<blocks, 256, 0, s>>>((const bf16 *)a_loc, (const bf16 *)a_full, (bf16 *)ws, n);
         else
             residual_kernel<float><<<blocks, 256, 0, s>>>((const float *)a_loc, (const float *)a_full, (float *)ws, n);
+        note_launch();
         CUDA_CHECK_RET(cudaGetLastError(), "residual kernel");
     }
     return accumulate(stats, a_loc, ws, n_rows, dtype, flag, s);
@@ -444,7 +453,7 @@ int ispa_selftest_bounded_wait(unsigned limit_us, ispa_stream_t stream) {
     int rc = device_error_flag(&flag);
     if (rc != ISPA_OK) return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    bounded_wait_selftest_kernel<<<1, 32, 0, s>>>((uint64_t)limit_us * 1000ull, flag);
+    bounded_wait_selftest_kernel<<<1, 32, 0, s>>>((uint64_t)limit_us * 1000ull, flag); note_launch();
     CUDA_CHECK_RET(cudaGetLastError(), "selftest launch");
     return ISPA_OK;
 }

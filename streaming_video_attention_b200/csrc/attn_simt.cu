@@ -143,10 +143,10 @@ cudaError_t launch_simt(const AttnArgs &a, cudaStream_t s) {
     if (a.n_q == 0) return cudaSuccess;
     if (a.head_dim == 64) {
         dim3 grid((a.n_q + kThreads - 1) / kThreads, a.heads);
-        attn_split_simt_kernel<T, 64><<<grid, kThreads, 0, s>>>(a);
+        attn_split_simt_kernel<T, 64><<<grid, kThreads, 0, s>>>(a); note_launch();
     } else if (a.head_dim == 128) {
         dim3 grid((a.n_q + kThreads / 2 - 1) / (kThreads / 2), a.heads);
-        attn_split_simt_kernel<T, 128><<<grid, kThreads, 0, s>>>(a);
+        attn_split_simt_kernel<T, 128><<<grid, kThreads, 0, s>>>(a); note_launch();
     } else {
         return cudaErrorInvalidValue;
     }

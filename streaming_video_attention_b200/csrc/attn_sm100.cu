@@ -492,7 +492,7 @@ cudaError_t launch_hd(const AttnArgs &a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(attn_split_sm100_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid((a.n_q + kBlockM - 1) / kBlockM, a.heads);
-    attn_split_sm100_kernel<HD><<<grid, kThreads, smem, s>>>(mq, mk, mv, p);
+    attn_split_sm100_kernel<HD><<<grid, kThreads, smem, s>>>(mq, mk, mv, p); note_launch();
     return cudaGetLastError();
 }
 

@@ -34,6 +34,9 @@ template <typename T> __device__ __forceinline__ T from_f32(float x);
 template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ bf16 from_f32<bf16>(float x) { return __float2bfloat16_rn(x); }
 
+// Process-wide count of kernel launches made by the library (read by ispa_kernel_launches).
+void note_launch();
+
 // Latch a device-side error code (first writer wins) into the per-device flag.
 __device__ __forceinline__ void raise_device_error(int *flag, int code) {
     if (flag) atomicCAS(flag, 0, code);

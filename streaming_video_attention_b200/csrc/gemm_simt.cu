@@ -125,10 +125,10 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmDesc d, GemmBatch b)
 template <typename TA, typename TB, typename TC>
 cudaError_t dispatch_layout(const GemmDesc &d, const GemmBatch &b, cudaStream_t s) {
     dim3 grid((d.N + BN - 1) / BN, (d.M + BM - 1) / BM, d.batch);
-    if (d.a_kcontig && d.b_kcontig) gemm_simt_kernel<TA, TB, TC, true, true><<<grid, 256, 0, s>>>(d, b);
-    else if (d.a_kcontig)           gemm_simt_kernel<TA, TB, TC, true, false><<<grid, 256, 0, s>>>(d, b);
-    else if (d.b_kcontig)           gemm_simt_kernel<TA, TB, TC, false, true><<<grid, 256, 0, s>>>(d, b);
-    else                            gemm_simt_kernel<TA, TB, TC, false, false><<<grid, 256, 0, s>>>(d, b);
+    if (d.a_kcontig && d.b_kcontig) { gemm_simt_kernel<TA, TB, TC, true, true><<<grid, 256, 0, s>>>(d, b); note_launch(); }
+    else if (d.a_kcontig)           { gemm_simt_kernel<TA, TB, TC, true, false><<<grid, 256, 0, s>>>(d, b); note_launch(); }
+    else if (d.b_kcontig)           { gemm_simt_kernel<TA, TB, TC, false, true><<<grid, 256, 0, s>>>(d, b); note_launch(); }
+    else                            { gemm_simt_kernel<TA, TB, TC, false, false><<<grid, 256, 0, s>>>(d, b); note_launch(); }
     return cudaGetLastError();
 }
 

@@ -227,14 +227,14 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
     const int fill_blocks = (int)std::min<size_t>((n + 255) / 256, 1024);
 
     // M = G + lambda I
-    fill_shifted_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(G, M, D, lambda);
+    fill_shifted_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(G, M, D, lambda); note_launch();
     ISPA_TRY(cudaGetLastError());
 
     // Y = C W, and dW <- Y (solved in place below)
     {
         GemmDesc d{D, D, D, D, D, D, true, false, ElemType::F32, wt, ElemType::F32, 1.f, 0.f, false, batch};
         ISPA_TRY(launch_gemm_simt(d, make_gemm_batch(C, 0, W, 0, Y, 0, batch, 4, ew), s));
-        copy_f32_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(Y, dW, n);
+        copy_f32_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(Y, dW, n); note_launch();
         ISPA_TRY(cudaGetLastError());
     }
 
@@ -242,11 +242,11 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
     const int nblk = D / NB;
     for (int kb = 0; kb < nblk; ++kb) {
         const int k0 = kb * NB;
-        potrf_diag_kernel<<<batch, 256, 0, s>>>(M, D, k0, status);
+        potrf_diag_kernel<<<batch, 256, 0, s>>>(M, D, k0, status); note_launch();
         ISPA_TRY(cudaGetLastError());
         const int rest = D - k0 - NB;
         if (rest <= 0) break;
-        trsm_panel_kernel<<<dim3((rest + NB - 1) / NB, batch), 256, 0, s>>>(M, D, k0);
+        trsm_panel_kernel<<<dim3((rest + NB - 1) / NB, batch), 256, 0, s>>>(M, D, k0); note_launch();
         ISPA_TRY(cudaGetLastError());
         GemmDesc d{rest, rest, NB, D, D, D, true, true, ElemType::F32, ElemType::F32, ElemType::F32, -1.f, 1.f,
                    true, batch};
@@ -259,7 +259,7 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
     const dim3 tgrid((D + 127) / 128, batch);
     for (int kb = 0; kb < nblk; ++kb) {
         const int k0 = kb * NB;
-        trsv_block_kernel<false><<<tgrid, 128, 0, s>>>(M, dW, D, k0);
+        trsv_block_kernel<false><<<tgrid, 128, 0, s>>>(M, dW, D, k0); note_launch();
         ISPA_TRY(cudaGetLastError());
         const int rest = D - k0 - NB;
         if (rest <= 0) break;
@@ -272,7 +272,7 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
     // Backward substitution L^T X = Z
     for (int kb = nblk - 1; kb >= 0; --kb) {
         const int k0 = kb * NB;
-        trsv_block_kernel<true><<<tgrid, 128, 0, s>>>(M, dW, D, k0);
+        trsv_block_kernel<true><<<tgrid, 128, 0, s>>>(M, dW, D, k0); note_launch();
         ISPA_TRY(cudaGetLastError());
         if (k0 == 0) break;
         // X[0:k0, :] -= (L[k0:k0+NB, 0:k0])^T X_k
@@ -286,30 +286,30 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
     GemmDesc full{D, D, D, D, D, D, true, false, ElemType::F32, ElemType::F32, ElemType::F32, 1.f, 0.f, false, batch};
     // t0 = tr(dW^T G dW)
     ISPA_TRY(launch_gemm_simt(full, make_gemm_batch(G, 0, dW, 0, P, 0, batch, 4, 4), s));
-    dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, P, n, terms + 0 * (size_t)batch * nparts);
+    dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, P, n, terms + 0 * (size_t)batch * nparts); note_launch();
     // t1 = tr(dW^T C W)
-    dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, Y, n, terms + 1 * (size_t)batch * nparts);
+    dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, Y, n, terms + 1 * (size_t)batch * nparts); note_launch();
     // t2 = tr(W^T H W), t3 = tr(W^T G W), t4 = tr(W^T C W)
     GemmDesc fw = full;
     fw.b_type = wt;
     ISPA_TRY(launch_gemm_simt(fw, make_gemm_batch(H, 0, W, 0, P, 0, batch, 4, ew), s));
-    if (wt == ElemType::BF16) dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, P, n, terms + 2 * (size_t)batch * nparts);
-    else dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, P, n, terms + 2 * (size_t)batch * nparts);
+    if (wt == ElemType::BF16) { dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, P, n, terms + 2 * (size_t)batch * nparts); note_launch(); }
+    else { dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, P, n, terms + 2 * (size_t)batch * nparts); note_launch(); }
     ISPA_TRY(launch_gemm_simt(fw, make_gemm_batch(G, 0, W, 0, P, 0, batch, 4, ew), s));
     if (wt == ElemType::BF16) {
-        dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, P, n, terms + 3 * (size_t)batch * nparts);
-        dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, Y, n, terms + 4 * (size_t)batch * nparts);
+        dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, P, n, terms + 3 * (size_t)batch * nparts); note_launch();
+        dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, Y, n, terms + 4 * (size_t)batch * nparts); note_launch();
     } else {
-        dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, P, n, terms + 3 * (size_t)batch * nparts);
-        dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, Y, n, terms + 4 * (size_t)batch * nparts);
+        dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, P, n, terms + 3 * (size_t)batch * nparts); note_launch();
+        dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, Y, n, terms + 4 * (size_t)batch * nparts); note_launch();
     }
     ISPA_TRY(cudaGetLastError());
-    finalize_eps_kernel<<<(batch + 63) / 64, 64, 0, s>>>(terms, nparts, batch, status, eps, err_terms);
+    finalize_eps_kernel<<<(batch + 63) / 64, 64, 0, s>>>(terms, nparts, batch, status, eps, err_terms); note_launch();
     ISPA_TRY(cudaGetLastError());
 
     if (w_new) {
-        if (wt == ElemType::BF16) add_delta_kernel<bf16><<<dim3(fill_blocks, batch), 256, 0, s>>>(W, dW, *w_new, n);
-        else add_delta_kernel<float><<<dim3(fill_blocks, batch), 256, 0, s>>>(W, dW, *w_new, n);
+        if (wt == ElemType::BF16) { add_delta_kernel<bf16><<<dim3(fill_blocks, batch), 256, 0, s>>>(W, dW, *w_new, n); note_launch(); }
+        else { add_delta_kernel<float><<<dim3(fill_blocks, batch), 256, 0, s>>>(W, dW, *w_new, n); note_launch(); }
         ISPA_TRY(cudaGetLastError());
     }
     return cudaSuccess;

@@ -258,7 +258,7 @@ cudaError_t launch_stats_bf16(const void *a_loc, const void *r, int n, int D, fl
     cudaError_t e = cudaFuncSetAttribute(stats_gemm_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
     if (e != cudaSuccess) return e;
     const int items = 2 * p.n_sym + p.nb * p.nb;
-    stats_gemm_sm100_kernel<<<items, kThreads, kSmemAlloc, s>>>(ma, mr, p);
+    stats_gemm_sm100_kernel<<<items, kThreads, kSmemAlloc, s>>>(ma, mr, p); note_launch();
     return cudaGetLastError();
 }
 

@@ -42,9 +42,12 @@ def make_rng(seed: int, *key: int) -> np.random.Generator:
 def bf16_bits_from_f32(x: np.ndarray) -> np.ndarray:
     """Round float32 values to bf16 (round to nearest, ties to even); return the uint16 bit patterns."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    b = x.view(np.uint32).astype(np.uint64)
-    b = (b + 0x7FFF + ((b >> 16) & 1)) >> 16
-    return b.astype(np.uint16)
+    b = x.view(np.uint32)
+    r = (b >> 16) & np.uint32(1)
+    r += np.uint32(0x7FFF)
+    r += b                      # finite values never wrap past 2^32
+    r >>= 16
+    return r.astype(np.uint16)
 
 
 def f32_from_bf16_bits(bits: np.ndarray) -> np.ndarray:
