@@ -50,6 +50,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=512)
+    ap.add_argument("--mode", choices=["episode", "call", "local", "solve"], default="episode",
+                    help="episode: the full step (default). call / local / solve: one layer's fused split "
+                         "attention at the last warmup chunk, one L-layer local attention with projection, or "
+                         "the batched solve alone (kernel-level timing, also the target of ncu captures)")
     return ap.parse_args(argv)
 
 
@@ -467,9 +471,93 @@ def ispa_arm(args, cfg, rank, world, local_rank):
     return 0
 
 
+def unit_arm(args, cfg):
+    """Kernel-level timing of one unit of the path, inputs resident, L2 flushed between
+    iterations (a 256 MB write)."""
+    from streaming_video_attention_b200 import ispa
+    from streaming_video_attention_b200.session import IspaSession
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+
+    def up(x):
+        return torch.from_numpy(synth.bf16_bits_from_f32(x).view(np.int16)).view(torch.bfloat16).to(device)
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    t = cfg.warmup_chunks - 1
+    D = cfg.D
+    sess = IspaSession(1 if args.mode != "solve" else cfg.layers, cfg.heads, cfg.head_dim, cfg.lam, 1, "bf16",
+                       str(device))
+    if args.mode in ("call", "local"):
+        if args.mode == "call":
+            frames = synth.cache_frames(cfg, t)
+        else:
+            t = cfg.warmup_chunks
+            s0 = cfg.chunk_start_frame(t)
+            frames = list(range(cfg.sink_frames)) + list(range(s0, s0 + cfg.chunk_frames))
+        lay = synth.chunk_layout(cfg, frames, t)
+        q = up(synth.chunk_q(cfg, 0, t))
+        k = up(synth.kv_tensor(cfg, 0, frames, "k"))
+        v = up(synth.kv_tensor(cfg, 0, frames, "v"))
+        W = up(synth.w_out(cfg, 0))
+        sess.set_weights([W])
+        sess.W_new[0].copy_(W)
+        sess.reserve(cfg.n_q)
+        o = torch.empty((cfg.n_q, cfg.heads, cfg.head_dim), dtype=torch.bfloat16, device=device)
+        lse = torch.empty((cfg.heads, cfg.n_q), dtype=torch.float32, device=device)
+        y = torch.empty((cfg.n_q, D), dtype=torch.bfloat16, device=device)
+        n_kv = lay["n_kv"]
+        if args.mode == "call":
+            sink, chunk = (lay["sink_begin"], lay["sink_end"]), (lay["chunk_begin"], lay["chunk_end"])
+            fn = lambda: sess.full_attention(0, q, k, v, sink, chunk, o, lse, collect=True)
+            flops = 4.0 * cfg.n_q * n_kv * cfg.head_dim * cfg.heads + 4.0 * cfg.n_q * D * D
+            what = f"fused split attention + statistics, one layer, n_q {cfg.n_q}, n_kv {n_kv}"
+        else:
+            sess.is_local = [1]
+            fn = lambda: sess.local_attention(0, q, k, v, o, lse, y)
+            flops = 4.0 * cfg.n_q * n_kv * cfg.head_dim * cfg.heads + 2.0 * cfg.n_q * D * D
+            what = f"L-layer local attention + W_new projection, n_q {cfg.n_q}, n_kv {n_kv}"
+    else:
+        Ws = [up(synth.w_out(cfg, l)) for l in range(cfg.layers)]
+        sess.set_weights(Ws)
+        # statistics of a representative warmup: random SPD-ish Grams from seeded operands
+        g = torch.Generator(device="cpu").manual_seed(0)
+        for st in sess.stats:
+            a = (torch.randn(3 * cfg.n_q, D, generator=g) * 0.05).to(device)
+            r = (torch.randn(3 * cfg.n_q, D, generator=g) * 0.05).to(device)
+            st.G.copy_(a.T @ a)
+            st.C.copy_(a.T @ r)
+            st.H.copy_(r.T @ r)
+        fn = lambda: sess.transition()
+        flops = cfg.layers * (D ** 3 / 3 + 2 * D ** 3 + 2 * D ** 3 + 6 * D ** 3)
+        what = f"absorb solve + error for {cfg.layers} layers, D {D}"
+    for _ in range(max(3, args.warmup)):
+        fn()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) / 1e3)
+    assert ispa.ispa_device_status() == ispa.ISPA_OK
+    burst, sustained, hbm, kind = peaks()
+    dt = statistics.median(times)
+    tf = flops / dt / 1e12
+    print(json.dumps({"mode": args.mode, "what": what, "ms": dt * 1e3, "ms_all": [x * 1e3 for x in times],
+                      "tflops": tf, "frac_of_burst_peak": tf / burst, "peak_kind": kind,
+                      "query_tokens_per_s": cfg.n_q / dt if args.mode != "solve" else None}), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     cfg = synth.CONFIGS[args.config]
+    if args.mode != "episode":
+        return unit_arm(args, cfg)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

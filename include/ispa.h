@@ -165,6 +165,12 @@ int ispa_device_status(ispa_stream_t stream);
  * returns. The GPU context stays usable. */
 int ispa_selftest_bounded_wait(unsigned limit_us, ispa_stream_t stream);
 
+/* ispa_selftest_exp2_poly -- test hook: y[i] = 2^x[i] computed by the FMA-pipe
+ * exponential the split-attention softmax uses for part of its weights (range reduction
+ * + degree-3 polynomial). x, y: device float32 [n]. Valid for x <= 64; x < -125 gives a
+ * value below 3e-38. */
+int ispa_selftest_exp2_poly(const float *x, float *y, int n, ispa_stream_t stream);
+
 /* ispa_kernel_launches -- number of kernels this library has launched in this process
  * (every device, every stream), for accounting; never reset. */
 unsigned long long ispa_kernel_launches(void);

@@ -219,9 +219,24 @@ __global__ void bounded_wait_selftest_kernel(uint64_t limit_ns, int *flag) {
     __syncthreads();
 }
 
+__global__ void exp2_poly_selftest_kernel(const float *x, float *y, int n) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) y[i] = ptx::exp2_poly(x[i]);
+}
+
 }  // namespace
 
 extern "C" {
+
+int ispa_selftest_exp2_poly(const float *x, float *y, int n, ispa_stream_t stream) {
+    g_last_error.clear();
+    if (n < 0 || (n > 0 && (!x || !y))) return fail(ISPA_ERR_INVALID_ARG, "bad arguments");
+    if (n == 0) return ISPA_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    exp2_poly_selftest_kernel<<<std::min((n + 255) / 256, 1024), 256, 0, s>>>(x, y, n);
+    note_launch();
+    CUDA_CHECK_RET(cudaGetLastError(), "selftest launch");
+    return ISPA_OK;
+}
 
 const char *ispa_last_error(void) { return g_last_error.c_str(); }
 

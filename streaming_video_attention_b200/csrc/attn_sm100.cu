@@ -280,25 +280,30 @@ attn_split_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             ok = ptx::mbar_wait_bounded(&s_full[st], (j >> 1) & 1, kWaitLimitNs, p.err_flag, abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
-            float s[kBlockN];
+            // all four 32-column loads in flight before one wait
+            uint32_t sr[kBlockN];
 #pragma unroll
-            for (int c = 0; c < kBlockN / 32; ++c) {
-                uint32_t r[32];
-                ptx::tmem_ld32(tS(st) + lane_off + c * 32, r);
-                ptx::tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
-            }
+            for (int c = 0; c < kBlockN / 32; ++c)
+                ptx::tmem_ld32(tS(st) + lane_off + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+            ptx::tmem_wait_ld();
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&s_free[st]);
+            float *s = reinterpret_cast<float *>(sr);
 
-            float mx = -INFINITY;
+            if (ti.valid < kBlockN) {
 #pragma unroll
-            for (int c = 0; c < kBlockN; ++c) {
-                if (c >= ti.valid) s[c] = -INFINITY;
-                mx = fmaxf(mx, s[c]);
+                for (int c = 0; c < kBlockN; ++c)
+                    if (c >= ti.valid) s[c] = -INFINITY;
             }
+            // row maximum: four independent chains of 3-input max
+            float mx4[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+            for (int c = 4; c < kBlockN; c += 8) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) mx4[u] = ptx::max3(mx4[u], s[c + u], s[c + 4 + u < kBlockN ? c + 4 + u : c + u]);
+            }
+            float mx = ptx::max3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
             mx *= p.scale_log2;
             const int part = ti.part;
             float m_cur = part ? m_hist : m_loc;
@@ -313,17 +318,20 @@ attn_split_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                 m_cur = mx;
             }
             const float mref = m_cur;
-            float rowsum = 0.f;
+            // exponentials, eight independent partial sums, bf16 pairs for P
+            float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             uint32_t pk[kBlockN / 2];
+            const float neg_m = -mref;
 #pragma unroll
             for (int c = 0; c < kBlockN; c += 2) {
-                const float e0 = ptx::exp2_approx(fmaf(s[c], p.scale_log2, -mref));
-                const float e1 = ptx::exp2_approx(fmaf(s[c + 1], p.scale_log2, -mref));
-                const __nv_bfloat162 b = __floats2bfloat162_rn(e0, e1);
-                const float2 f = __bfloat1622float2(b);
-                rowsum += f.x + f.y;
-                pk[c / 2] = *reinterpret_cast<const uint32_t *>(&b);
+                // one column in four goes to the FMA-pipe exponential, the rest to MUFU
+                const float e0 = ptx::exp2_approx(fmaf(s[c], p.scale_log2, neg_m));
+                const float x1 = fmaf(s[c + 1], p.scale_log2, neg_m);
+                const float e1 = ((c / 2) % 2 == 1) ? ptx::exp2_poly(x1) : ptx::exp2_approx(x1);
+                sum8[(c / 2) % 8] += e0 + e1;
+                pk[c / 2] = pack_bf16x2(e0, e1);
             }
+            const float rowsum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
             l_cur = fmaf(l_cur, alpha, rowsum);
             if (part) { m_hist = m_cur; l_hist = l_cur; } else { m_loc = m_cur; l_loc = l_cur; }
             // P (row `row`, 128 bf16 = 16 chunks of 16 bytes) into the swizzled K-major tile

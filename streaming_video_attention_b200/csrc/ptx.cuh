@@ -70,6 +70,13 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
 }
 
 // ---- misc ---------------------------------------------------------------------------
+// max(a, b, c) in one instruction (sm_100).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float y;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+    return y;
+}
+
 // 2^x with the hardware approximation (MUFU.EX2), flush-to-zero; used for softmax weights
 // that are rounded to bf16 right after.
 __device__ __forceinline__ float exp2_approx(float x) {
@@ -90,6 +97,23 @@ __device__ __forceinline__ bool elect_one() {
 
 __device__ __forceinline__ void fence_proxy_async_shared() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 2^x on the FMA pipe, for softmax weights that are rounded to bf16 right after (so
+// that part of the exponentials leaves the MUFU unit). Method: Cody-Waite style range
+// reduction x = n + f with n = round(x) taken from the low mantissa bits of x + 1.5*2^23,
+// f in [-0.5, 0.5]; 2^f from a degree-3 polynomial fitted here for minimum relative error
+// on that interval (max relative error 7.6e-5, far below bf16's 2^-9 rounding); 2^n is
+// added to the exponent field. Inputs are clamped to >= -125 (results there are below
+// 3e-38, i.e. zero after the bf16 products they feed); x <= 64 is assumed.
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -125.0f);
+    const float t = x + 12582912.0f;
+    const float f = x - (t - 12582912.0f);
+    float p = fmaf(0.055174145847558975f, f, 0.24261757731437683f);
+    p = fmaf(p, f, 0.6932610869407654f);
+    p = fmaf(p, f, 0.9999275803565979f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 // ---- TMA (no multicast anywhere in this library) ------------------------------------

@@ -30,7 +30,7 @@ ISPA_FP32 = 1
 EXPORTS = (
     "ispa_attn_split", "ispa_accum_stats", "ispa_stats_reset", "ispa_solve_absorb", "ispa_select_layers",
     "ispa_local_attn", "ispa_workspace_bytes", "ispa_device_status", "ispa_selftest_bounded_wait",
-    "ispa_kernel_launches", "ispa_last_error", "ispa_version",
+    "ispa_selftest_exp2_poly", "ispa_kernel_launches", "ispa_last_error", "ispa_version",
 )
 
 
@@ -78,6 +78,7 @@ def lib() -> ctypes.CDLL:
         L.ispa_workspace_bytes.restype = ctypes.c_size_t
         L.ispa_device_status.argtypes = [vp]
         L.ispa_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp]
+        L.ispa_selftest_exp2_poly.argtypes = [vp, vp, i, vp]
         L.ispa_kernel_launches.argtypes = []
         L.ispa_kernel_launches.restype = ctypes.c_ulonglong
         L.ispa_last_error.restype = ctypes.c_char_p
@@ -189,6 +190,10 @@ def ispa_local_attn(desc, q, k_loc, v_loc, o, lse=None, w_new=None, y=None, ws=N
 
 def ispa_device_status(stream=None) -> int:
     return int(lib().ispa_device_status(_stream(stream)))
+
+
+def ispa_selftest_exp2_poly(x: torch.Tensor, y: torch.Tensor, stream=None) -> None:
+    _check(lib().ispa_selftest_exp2_poly(_p(x), _p(y), x.numel(), _stream(stream)), "ispa_selftest_exp2_poly")
 
 
 def ispa_kernel_launches() -> int:

@@ -50,3 +50,17 @@ def test_workspace_errors_are_reported():
         ispa.ispa_attn_split(desc, x[:128], x, x, o, lse, stats=bad,
                              ws=ispa.alloc_workspace(ispa.workspace_bytes(desc, 0, 0)))
     assert ei.value.code == ispa.ISPA_ERR_INVALID_ARG
+
+
+def test_fma_pipe_exponential_error_bound():
+    """The softmax's FMA-pipe 2^x stays within 1e-4 relative of the exact value (bf16 rounding
+    of the weights it feeds is 2^-9 = 2e-3), and agrees with CUDA's exp2f on the same inputs."""
+    x = torch.cat([torch.linspace(-125.0, 8.0, 1 << 20), torch.tensor([0.0, -0.5, 0.5, 1.0, -1.0, 7.99])]).cuda()
+    y = torch.empty_like(x)
+    ispa.ispa_selftest_exp2_poly(x, y)
+    torch.cuda.synchronize()
+    exact = np.exp2(x.double().cpu().numpy())
+    rel = np.abs(y.double().cpu().numpy() - exact) / exact
+    assert rel.max() < 1e-4, rel.max()
+    rel_cuda = (y - torch.exp2(x)).abs() / torch.exp2(x)
+    assert float(rel_cuda.max()) < 1e-4
