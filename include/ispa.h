@@ -100,6 +100,22 @@ int ispa_attn_split(const ispa_attn_desc *desc, const void *q, const void *k, co
                     float *lse_hist, const ispa_stats *stats, void *ws, size_t ws_bytes,
                     ispa_stream_t stream);
 
+/* ispa_attn_split_noalloc -- ispa_attn_split with fused statistics for callers that cannot
+ * allocate device memory (for example code running inside a host framework that owns all
+ * device memory and passes only its inputs and outputs, or a plugin interface without a
+ * workspace argument). The paper has no counterpart; this is a deployment variant. The
+ * bf16 (or float32) operands handed from the attention kernel to the statistics GEMM live
+ * in a static device array of 2 x 16 MiB instead of a caller workspace: each operand,
+ * n_q * heads * head_dim elements, may take at most 16 MiB (8,388,608 bf16 or 4,194,304
+ * float32 elements); larger calls return ISPA_ERR_UNSUPPORTED before any launch. stats is
+ * required. The array is held by every GPU that loads the library until the process
+ * exits. The first call on a device looks up the array's device address (make that first
+ * call before any stream capture). All calls share the array: calls that overlap on the
+ * GPU race and must be serialised by the caller. Arguments otherwise as ispa_attn_split. */
+int ispa_attn_split_noalloc(const ispa_attn_desc *desc, const void *q, const void *k, const void *v,
+                            void *o_full, float *lse_full, void *o_loc, float *lse_loc, void *o_hist,
+                            float *lse_hist, const ispa_stats *stats, ispa_stream_t stream);
+
 /* ispa_accum_stats -- the statistics of [ISPA §3.2] from attention outputs that were
  * computed elsewhere (unfused path): R = a_full - a_loc (then rounded to bf16 in bf16
  * mode), G += A_loc^T A_loc, C += A_loc^T R, H += R^T R, rows += n_rows.

@@ -22,6 +22,7 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
 namespace ispa {
 static std::atomic<unsigned long long> g_launches{0};
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+int record_error(int code, const char *msg);
 }  // namespace ispa
 
 using namespace ispa;
@@ -43,6 +44,13 @@ int fail(int code, const char *fmt, ...) {
 int cuda_fail(cudaError_t e, const char *where) {
     return fail(ISPA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
 }
+
+}  // namespace
+
+// Lets entry points defined in other files report through ispa_last_error().
+int ispa::record_error(int code, const char *msg) { return fail(code, "%s", msg); }
+
+namespace {
 
 #define CUDA_CHECK_RET(x, where)                     \
     do {                                             \

@@ -28,7 +28,7 @@ ISPA_BF16 = 0
 ISPA_FP32 = 1
 
 EXPORTS = (
-    "ispa_attn_split", "ispa_accum_stats", "ispa_stats_reset", "ispa_solve_absorb", "ispa_select_layers",
+    "ispa_attn_split", "ispa_attn_split_noalloc", "ispa_accum_stats", "ispa_stats_reset", "ispa_solve_absorb", "ispa_select_layers",
     "ispa_local_attn", "ispa_workspace_bytes", "ispa_device_status", "ispa_selftest_bounded_wait",
     "ispa_selftest_exp2_poly", "ispa_kernel_launches", "ispa_last_error", "ispa_version",
 )
@@ -67,6 +67,8 @@ def lib() -> ctypes.CDLL:
         vp, i, sz, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
         L.ispa_attn_split.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                       ctypes.POINTER(CStats), vp, sz, vp]
+        L.ispa_attn_split_noalloc.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                              ctypes.POINTER(CStats), vp]
         L.ispa_accum_stats.argtypes = [ctypes.POINTER(CStats), vp, vp, i, i, vp, sz, vp]
         L.ispa_stats_reset.argtypes = [ctypes.POINTER(CStats), vp]
         L.ispa_solve_absorb.argtypes = [ctypes.POINTER(CStats), i, ctypes.POINTER(vp), i, f, vp, vp, vp,
@@ -145,6 +147,15 @@ def ispa_attn_split(desc, q, k, v, o_full, lse_full, o_loc=None, lse_loc=None, o
                                _p(lse_loc), _p(o_hist), _p(lse_hist), cs, _p(ws),
                                0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "ispa_attn_split")
+
+
+def ispa_attn_split_noalloc(desc, q, k, v, o_full, lse_full, o_loc=None, lse_loc=None, o_hist=None,
+                            lse_hist=None, stats: Stats = None, stream=None) -> None:
+    """ispa_attn_split with fused statistics, using the library's static scratch (no workspace)."""
+    cs = ctypes.byref(stats.c()) if stats is not None else None
+    rc = lib().ispa_attn_split_noalloc(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(o_full), _p(lse_full), _p(o_loc),
+                                       _p(lse_loc), _p(o_hist), _p(lse_hist), cs, _stream(stream))
+    _check(rc, "ispa_attn_split_noalloc")
 
 
 def ispa_accum_stats(stats: Stats, a_loc, a_full, n_rows: int, dtype: int, ws=None, stream=None) -> None:
