@@ -211,7 +211,9 @@ def run_episode(cfg, n_chunks: Optional[int] = None, K: Optional[int] = None,
     it becomes an F-layer again; a former L-layer's history restarts at the cut. The new
     dW replaces the old one.
 
-    Returns per-transition eps/dW/selection and, if asked, per-chunk outputs y = O W_cur.
+    Returns per-transition eps/dW/selection and, if asked, per-chunk per-layer outputs: the
+    attention output O (A_full for an F-layer, A_loc for an L-layer), y = O W_cur and
+    whether the layer ran local.
     """
     import synth  # seeded inputs only
 
@@ -256,7 +258,7 @@ def run_episode(cfg, n_chunks: Optional[int] = None, K: Optional[int] = None,
                 if in_warmup:
                     stats_update(stats[l], res["A_loc"], res["A_full"], cfg.dtype)
             if keep_outputs:
-                chunk_out.append(project(O, W_cur[l]))
+                chunk_out.append(dict(O=O, y=project(O, W_cur[l]), local=bool(is_local[l])))
         if keep_outputs:
             outputs.append(chunk_out)
         if in_warmup and t == warm_start + cfg.warmup_chunks - 1:
@@ -270,8 +272,8 @@ def run_episode(cfg, n_chunks: Optional[int] = None, K: Optional[int] = None,
             idx, flags = select_layers(eps, K)
             for l in idx:
                 W_cur[l] = W0[l] + dWs[l]
-            is_local = flags
-            transitions.append(dict(chunk=t, eps=eps, errs=errs, dW=dWs, idx=idx, is_local=flags,
+            is_local = list(flags)
+            transitions.append(dict(chunk=t, eps=eps, errs=errs, dW=dWs, idx=idx, is_local=list(flags),
                                     stats=[dict(G=s["G"].copy(), C=s["C"].copy(), H=s["H"].copy(),
                                                 rows=s["rows"]) for s in stats]))
     return dict(transitions=transitions, outputs=outputs)

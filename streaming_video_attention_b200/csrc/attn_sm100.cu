@@ -11,16 +11,20 @@
 // (bf16) for the statistics GEMM that follows on the same stream.
 //
 // CTA = one 128-row query tile of one head; 256 threads:
-//   warp 0      TMA producer: Q once, then K/V tiles of 128 rows into a 2-stage ring
+//   warp 0      TMA producer: Q once, then K and V tiles of 128 rows into a ring of stages
 //   warp 1      TMEM allocation; lane 0 issues every tcgen05.mma and commit
 //   warps 4..7  softmax (thread i owns query row i = TMEM lane i), lazy rescale, epilogue
-// TMEM (512 columns): S double buffer (2 x 128), O_loc (HD), O_hist (HD).
-// Shared memory: Q, K[2], V[2] (TMA, 128-byte swizzle) and P[2] (bf16, written by the
-// softmax threads in the same swizzled K-major layout).
+// TMEM (512 columns): S double buffer (2 x 128), O_loc (HD), O_hist (HD). P (bf16) is
+// written over the first 64 columns of the S buffer it came from and feeds the PV MMA
+// straight from tensor memory; shared memory holds only Q and the K/V ring (TMA, 128-byte
+// swizzle).
 //
 // MMA order S_0, S_1, PV_0, S_2, PV_1, ...: S_{j+1} runs on the tensor cores while the
-// softmax works on S_j. Completion of S_j implies completion of PV_{j-2}, so P buffer
-// j%2 is free when the softmax starts on S_j.
+// softmax works on S_j. tcgen05.mma operations execute in issue order, so S_{j+2} (which
+// overwrites S buffer j%2, holding P_j) starts only after PV_j has consumed P_j, and the
+// completion of S_j implies that of PV_{j-2}. The MMA thread keeps its non-issuing work per
+// tile to two barrier waits and a few integer updates: the tensor-core queue is shallow,
+// and every cycle it spends elsewhere is idle tensor time.
 //
 // The running maximum is updated lazily: a row's reference maximum moves (and its O
 // accumulator is rescaled through TMEM) only when a new tile's maximum exceeds it by more
@@ -47,17 +51,17 @@ constexpr float kRescaleThreshold = 8.0f;          // log2 units: rescale when t
 
 template <int HD>
 struct Smem {
+    static constexpr int kStages = HD == 128 ? 3 : 4;   // K/V ring depth
     static constexpr int kQBytes = kBlockM * HD * 2;
-    static constexpr int kKVBytes = kBlockN * HD * 2;
-    static constexpr int kPBytes = kBlockM * kBlockN * 2;
+    static constexpr int kKVBytes = kBlockN * HD * 2;    // one of K or V for one tile
     static constexpr int kQ = 0;
     static constexpr int kK = kQ + kQBytes;
-    static constexpr int kV = kK + 2 * kKVBytes;
-    static constexpr int kP = kV + 2 * kKVBytes;
-    static constexpr int kBar = kP + 2 * kPBytes;
-    static constexpr int kNumBars = 16;
-    static constexpr int kMisc = kBar + kNumBars * 8;
-    static constexpr int kTotal = kMisc + 64 + kMaxSegments * 8;
+    static constexpr int kV = kK + kStages * kKVBytes;
+    static constexpr int kBar = kV + kStages * kKVBytes;
+    static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2;   // q, kv full/empty, s_full, p_full, o, done
+    static constexpr int kSeg = kBar + kNumBars * 8;              // segment table: 4 x kMaxSegments ints
+    static constexpr int kMisc = kSeg + 4 * kMaxSegments * 4;
+    static constexpr int kTotal = kMisc + 16;
     static constexpr int kAlloc = kTotal + 1024;   // slack for 1024-byte alignment
 };
 
@@ -76,28 +80,28 @@ struct SplitParams {
     int *err_flag;
 };
 
-// Tile j of the concatenated segment list: first KV row, valid rows, partition.
-struct TileInfo {
-    int row0, valid, part, first_of_part;
+// Walks the KV tiles in order: the local segments, then the history segments, 128 rows at
+// a time (the last tile of a segment may be partial). Segment data sit in shared memory;
+// the current segment's bounds stay in registers, so advancing costs an add and a compare.
+struct TileCursor {
+    const int *sb, *se, *sp, *sf;
+    int nseg, si, row0, end, part, seg_first, tile_in_seg;
+    __device__ __forceinline__ void init(const int *b, const int *e, const int *pt, const int *f, int n) {
+        sb = b; se = e; sp = pt; sf = f; nseg = n; si = 0;
+        if (n > 0) load();
+    }
+    __device__ __forceinline__ void load() {
+        row0 = sb[si]; end = se[si]; part = sp[si]; seg_first = sf[si]; tile_in_seg = 0;
+    }
+    __device__ __forceinline__ void advance() {
+        row0 += kBlockN;
+        ++tile_in_seg;
+        if (row0 >= end && ++si < nseg) load();
+    }
+    __device__ __forceinline__ int valid() const { return min(kBlockN, end - row0); }
+    // first tile of its partition: the accumulator starts from zero
+    __device__ __forceinline__ bool first_of_part() const { return seg_first && tile_in_seg == 0; }
 };
-
-__device__ __forceinline__ TileInfo tile_info(const SegmentList &sl, const int *seg_first_tile, int j) {
-    int s = 0;
-#pragma unroll 1
-    while (s + 1 < sl.count && j >= seg_first_tile[s + 1]) ++s;
-    const Segment sg = sl.seg[s];
-    const int t = j - seg_first_tile[s];
-    TileInfo ti;
-    ti.row0 = sg.begin + t * kBlockN;
-    ti.valid = min(kBlockN, sg.end - ti.row0);
-    ti.part = sg.part;
-    // first tile of its partition: first tile of the first segment with that partition
-    bool first = (t == 0);
-    for (int u = 0; u < s && first; ++u)
-        if (sl.seg[u].part == sg.part && sl.seg[u].end > sl.seg[u].begin) first = false;
-    ti.first_of_part = first ? 1 : 0;
-    return ti;
-}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -109,48 +113,54 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_split_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const SplitParams p) {
     using L = Smem<HD>;
+    constexpr int NS = L::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = smem + L::kQ;
     uint8_t *sK = smem + L::kK;
     uint8_t *sV = smem + L::kV;
-    uint8_t *sP = smem + L::kP;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
     uint64_t *q_full = bars + 0;
-    uint64_t *k_full = bars + 1;    // [2]
-    uint64_t *k_empty = bars + 3;   // [2]
-    uint64_t *v_full = bars + 5;    // [2]
-    uint64_t *v_empty = bars + 7;   // [2]
-    uint64_t *s_full = bars + 9;    // [2]
-    uint64_t *s_free = bars + 11;   // [2]
-    uint64_t *p_full = bars + 13;   // [2]
-    uint64_t *o_bar = bars + 15;
+    uint64_t *kv_full = bars + 1;             // [NS] K and V of one tile landed
+    uint64_t *kv_empty = kv_full + NS;        // [NS] S and PV of that tile done
+    uint64_t *s_full = kv_empty + NS;         // [2]  S buffer written by the MMA
+    uint64_t *p_full = s_full + 2;            // [2]  P written (and O rescaled) by the softmax
+    uint64_t *o_bar = p_full + 2;             //      one phase per PV
+    uint64_t *done_bar = o_bar + 1;           //      every MMA of this CTA finished
+    int *seg_begin = reinterpret_cast<int *>(smem + L::kSeg);
+    int *seg_end = seg_begin + kMaxSegments;
+    int *seg_part = seg_end + kMaxSegments;
+    int *seg_first = seg_part + kMaxSegments;
     uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
-    uint64_t *done_bar = reinterpret_cast<uint64_t *>(smem + L::kMisc + 8);
-    int *seg_first_tile = reinterpret_cast<int *>(smem + L::kMisc + 64);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int q0 = blockIdx.x * kBlockM;
     const int head = blockIdx.y;
+    const int nseg = p.segs.count;
 
-    // total tiles and per-segment first-tile table
     int n_tiles = 0;
-    for (int s = 0; s < p.segs.count; ++s) {
-        if (threadIdx.x == 0) seg_first_tile[s] = n_tiles;
-        n_tiles += (p.segs.seg[s].end - p.segs.seg[s].begin + kBlockN - 1) / kBlockN;
-    }
+    for (int s = 0; s < nseg; ++s) n_tiles += (p.segs.seg[s].end - p.segs.seg[s].begin + kBlockN - 1) / kBlockN;
 
     if (threadIdx.x == 0) {
+        for (int s = 0; s < nseg; ++s) {
+            const Segment sg = p.segs.seg[s];
+            seg_begin[s] = sg.begin;
+            seg_end[s] = sg.end;
+            seg_part[s] = sg.part;
+            int first = 1;
+            for (int u = 0; u < s; ++u)
+                if (p.segs.seg[u].part == sg.part) first = 0;
+            seg_first[s] = first;
+        }
         ptx::mbar_init(q_full, 1);
+        for (int i = 0; i < NS; ++i) {
+            ptx::mbar_init(&kv_full[i], 1);
+            ptx::mbar_init(&kv_empty[i], 1);
+        }
         for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(&k_full[i], 1);
-            ptx::mbar_init(&k_empty[i], 1);
-            ptx::mbar_init(&v_full[i], 1);
-            ptx::mbar_init(&v_empty[i], 1);
             ptx::mbar_init(&s_full[i], 1);
-            ptx::mbar_init(&s_free[i], 4);
-            ptx::mbar_init(&p_full[i], 128);
+            ptx::mbar_init(&p_full[i], 4);      // one arrival per softmax warp
         }
         ptx::mbar_init(o_bar, 1);
         ptx::mbar_init(done_bar, 1);
@@ -180,35 +190,27 @@ attn_split_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             ptx::mbar_arrive_expect_tx(q_full, L::kQBytes);
             for (int b = 0; b < HD / 64; ++b)
                 ptx::tma_load_3d(sQ + b * (kBlockM * 128), &tmQ, q_full, b * 64, head, q0, pol_q);
-            int outstanding_k[2] = {-1, -1}, outstanding_v[2] = {-1, -1};
+            TileCursor cur;
+            cur.init(seg_begin, seg_end, seg_part, seg_first, nseg);
+            int issued = -1;
             bool ok = true;
-            for (int j = 0; j < n_tiles && ok; ++j) {
-                const TileInfo ti = tile_info(p.segs, seg_first_tile, j);
-                const int st = j & 1;
-                const uint32_t ph = (j >> 1) & 1;
-                ok = ptx::mbar_wait_bounded(&k_empty[st], ph ^ 1, kWaitLimitNs, p.err_flag, abort_flag);
+            for (int j = 0; j < n_tiles; ++j, cur.advance()) {
+                const int st = j % NS;
+                ok = ptx::mbar_wait_bounded(&kv_empty[st], ((j / NS) & 1) ^ 1, kWaitLimitNs, p.err_flag, abort_flag);
                 if (!ok) break;
-                ptx::mbar_arrive_expect_tx(&k_full[st], L::kKVBytes);
-                for (int b = 0; b < HD / 64; ++b)
-                    ptx::tma_load_3d(sK + st * L::kKVBytes + b * (kBlockN * 128), &tmK, &k_full[st], b * 64, head,
-                                     ti.row0, pol_kv);
-                outstanding_k[st] = j;
-                ok = ptx::mbar_wait_bounded(&v_empty[st], ph ^ 1, kWaitLimitNs, p.err_flag, abort_flag);
-                if (!ok) break;
-                ptx::mbar_arrive_expect_tx(&v_full[st], L::kKVBytes);
-                for (int b = 0; b < HD / 64; ++b)
-                    ptx::tma_load_3d(sV + st * L::kKVBytes + b * (kBlockN * 128), &tmV, &v_full[st], b * 64, head,
-                                     ti.row0, pol_kv);
-                outstanding_v[st] = j;
+                ptx::mbar_arrive_expect_tx(&kv_full[st], 2 * L::kKVBytes);
+                for (int b = 0; b < HD / 64; ++b) {
+                    ptx::tma_load_3d(sK + st * L::kKVBytes + b * (kBlockN * 128), &tmK, &kv_full[st], b * 64, head,
+                                     cur.row0, pol_kv);
+                    ptx::tma_load_3d(sV + st * L::kKVBytes + b * (kBlockN * 128), &tmV, &kv_full[st], b * 64, head,
+                                     cur.row0, pol_kv);
+                }
+                issued = j;
             }
             if (!ok) {
                 // drain copies that may still be writing shared memory
-                for (int st = 0; st < 2; ++st) {
-                    if (outstanding_k[st] >= 0)
-                        ptx::mbar_wait_bounded(&k_full[st], (outstanding_k[st] >> 1) & 1, kWaitLimitNs, nullptr, nullptr);
-                    if (outstanding_v[st] >= 0)
-                        ptx::mbar_wait_bounded(&v_full[st], (outstanding_v[st] >> 1) & 1, kWaitLimitNs, nullptr, nullptr);
-                }
+                for (int j = issued - NS + 1 > 0 ? issued - NS + 1 : 0; j <= issued; ++j)
+                    ptx::mbar_wait_bounded(&kv_full[j % NS], (j / NS) & 1, kWaitLimitNs, nullptr, nullptr);
                 ptx::mbar_wait_bounded(q_full, 0, kWaitLimitNs, nullptr, nullptr);
             }
         }
@@ -217,50 +219,46 @@ attn_split_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         if (lane == 0) {
             constexpr uint32_t idesc_qk = ptx::make_idesc_bf16(kBlockM, kBlockN, false, false);
             constexpr uint32_t idesc_pv = ptx::make_idesc_bf16(kBlockM, HD, false, true);
-            const uint32_t aQ = ptx::smem_u32(sQ), aK = ptx::smem_u32(sK), aV = ptx::smem_u32(sV),
-                           aP = ptx::smem_u32(sP);
+            const uint32_t aQ = ptx::smem_u32(sQ), aK = ptx::smem_u32(sK), aV = ptx::smem_u32(sV);
             bool ok = ptx::mbar_wait_bounded(q_full, 0, kWaitLimitNs, p.err_flag, abort_flag);
+            // S_j = Q K_j^T into S buffer j%2 (waits for K_j and V_j: they land together)
             auto issue_s = [&](int j) -> bool {
-                const int st = j & 1;
-                if (!ptx::mbar_wait_bounded(&k_full[st], (j >> 1) & 1, kWaitLimitNs, p.err_flag, abort_flag))
-                    return false;
-                if (j >= 2 && !ptx::mbar_wait_bounded(&s_free[st], ((j - 2) >> 1) & 1, kWaitLimitNs, p.err_flag,
-                                                       abort_flag))
+                const int sb = j & 1, ks = j % NS;
+                if (!ptx::mbar_wait_bounded(&kv_full[ks], (j / NS) & 1, kWaitLimitNs, p.err_flag, abort_flag))
                     return false;
                 ptx::tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
                     const uint32_t koff = (kk / 4) * (kBlockM * 128) + (kk % 4) * 32;
                     const uint64_t da = ptx::make_sdesc_sw128(aQ + koff, 16, 1024);
-                    const uint64_t db = ptx::make_sdesc_sw128(aK + st * L::kKVBytes + koff, 16, 1024);
-                    ptx::umma_f16_ss(tS(st), da, db, idesc_qk, kk > 0 ? 1u : 0u);
+                    const uint64_t db = ptx::make_sdesc_sw128(aK + ks * L::kKVBytes + koff, 16, 1024);
+                    ptx::umma_f16_ss(tS(sb), da, db, idesc_qk, kk > 0 ? 1u : 0u);
                 }
-                ptx::umma_commit(&s_full[st]);
-                ptx::umma_commit(&k_empty[st]);
+                ptx::umma_commit(&s_full[sb]);
                 return true;
             };
             if (ok && n_tiles > 0) ok = issue_s(0);
-            for (int j = 0; j < n_tiles && ok; ++j) {
+            TileCursor cur;
+            cur.init(seg_begin, seg_end, seg_part, seg_first, nseg);
+            for (int j = 0; j < n_tiles && ok; ++j, cur.advance()) {
                 if (j + 1 < n_tiles) {
                     ok = issue_s(j + 1);
                     if (!ok) break;
                 }
-                const TileInfo ti = tile_info(p.segs, seg_first_tile, j);
-                const int st = j & 1;
-                ok = ptx::mbar_wait_bounded(&p_full[st], (j >> 1) & 1, kWaitLimitNs, p.err_flag, abort_flag);
-                if (!ok) break;
-                ok = ptx::mbar_wait_bounded(&v_full[st], (j >> 1) & 1, kWaitLimitNs, p.err_flag, abort_flag);
+                const int sb = j & 1, vs = j % NS;
+                const uint32_t acc0 = cur.first_of_part() ? 0u : 1u;
+                const uint32_t dO = tO(cur.part);
+                ok = ptx::mbar_wait_bounded(&p_full[sb], (j >> 1) & 1, kWaitLimitNs, p.err_flag, abort_flag);
                 if (!ok) break;
                 ptx::tc_fence_after();
+                // O += P V with P (bf16) in the first 64 columns of S buffer sb: 16 keys = 8 columns per step
 #pragma unroll
                 for (int kk = 0; kk < kBlockN / 16; ++kk) {
-                    const uint32_t poff = (kk / 4) * (kBlockM * 128) + (kk % 4) * 32;
-                    const uint64_t da = ptx::make_sdesc_sw128(aP + st * L::kPBytes + poff, 16, 1024);
-                    const uint64_t db = ptx::make_sdesc_sw128(aV + st * L::kKVBytes + kk * 2048, kBlockN * 128, 1024);
-                    ptx::umma_f16_ss(tO(ti.part), da, db, idesc_pv, (kk > 0 || !ti.first_of_part) ? 1u : 0u);
+                    const uint64_t db = ptx::make_sdesc_sw128(aV + vs * L::kKVBytes + kk * 2048, kBlockN * 128, 1024);
+                    ptx::umma_f16_ts(dO, tS(sb) + kk * 8, db, idesc_pv, kk > 0 ? 1u : acc0);
                 }
                 ptx::umma_commit(o_bar);
-                ptx::umma_commit(&v_empty[st]);
+                ptx::umma_commit(&kv_empty[vs]);
             }
             // all MMAs issued by this thread must finish before TMEM is released
             ptx::umma_commit(done_bar);
@@ -273,10 +271,13 @@ attn_split_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
         float m_loc = -INFINITY, m_hist = -INFINITY;   // reference maxima (log2 units)
         float l_loc = 0.f, l_hist = 0.f;               // softmax denominators
+        TileCursor cur;
+        cur.init(seg_begin, seg_end, seg_part, seg_first, nseg);
         bool ok = true;
-        for (int j = 0; j < n_tiles && ok; ++j) {
-            const TileInfo ti = tile_info(p.segs, seg_first_tile, j);
+        for (int j = 0; j < n_tiles && ok; ++j, cur.advance()) {
             const int st = j & 1;
+            const int valid = cur.valid();
+            const int part = cur.part;
             ok = ptx::mbar_wait_bounded(&s_full[st], (j >> 1) & 1, kWaitLimitNs, p.err_flag, abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
@@ -286,15 +287,12 @@ attn_split_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             for (int c = 0; c < kBlockN / 32; ++c)
                 ptx::tmem_ld32(tS(st) + lane_off + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
             ptx::tmem_wait_ld();
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&s_free[st]);
             float *s = reinterpret_cast<float *>(sr);
 
-            if (ti.valid < kBlockN) {
+            if (valid < kBlockN) {
 #pragma unroll
                 for (int c = 0; c < kBlockN; ++c)
-                    if (c >= ti.valid) s[c] = -INFINITY;
+                    if (c >= valid) s[c] = -INFINITY;
             }
             // row maximum: four independent chains of 3-input max
             float mx4[4] = {s[0], s[1], s[2], s[3]};
@@ -305,7 +303,6 @@ attn_split_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             }
             float mx = ptx::max3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
             mx *= p.scale_log2;
-            const int part = ti.part;
             float m_cur = part ? m_hist : m_loc;
             float l_cur = part ? l_hist : l_loc;
             float alpha = 1.f;
@@ -334,15 +331,11 @@ attn_split_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             const float rowsum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
             l_cur = fmaf(l_cur, alpha, rowsum);
             if (part) { m_hist = m_cur; l_hist = l_cur; } else { m_loc = m_cur; l_loc = l_cur; }
-            // P (row `row`, 128 bf16 = 16 chunks of 16 bytes) into the swizzled K-major tile
-            uint8_t *prow = sP + st * L::kPBytes + row * 128;
-#pragma unroll
-            for (int cc = 0; cc < kBlockN / 8; ++cc) {
-                const int blk = cc / 8, ch = cc % 8;
-                uint4 v = make_uint4(pk[cc * 4 + 0], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
-                *reinterpret_cast<uint4 *>(prow + blk * (kBlockM * 128) + ((ch ^ (row & 7)) << 4)) = v;
-            }
-            ptx::fence_proxy_async_shared();
+            // P (row `row`: 128 bf16 packed in 64 columns) over the first half of this S buffer,
+            // the A operand of the PV MMA
+            ptx::tmem_st32(tS(st) + lane_off, &pk[0]);
+            ptx::tmem_st32(tS(st) + lane_off + 32, &pk[32]);
+            ptx::tmem_wait_st();
             // PV_{j-1} must be complete before O may be rescaled (and before P_{j} is handed over
             // when it goes into the accumulator PV_{j-1} wrote).
             if (j >= 1) {
@@ -363,7 +356,8 @@ attn_split_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                 ptx::tmem_wait_st();
             }
             ptx::tc_fence_before();
-            ptx::mbar_arrive(&p_full[st]);
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&p_full[st]);
         }
         // ---------------------------------------------------------------- epilogue
         if (ok && n_tiles > 0) ok = ptx::mbar_wait_bounded(o_bar, (n_tiles - 1) & 1, kWaitLimitNs, p.err_flag, abort_flag);
