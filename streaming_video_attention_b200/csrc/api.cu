@@ -14,9 +14,10 @@
 
 namespace ispa {
 cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H, const PtrBatch &W, ElemType wt,
-                        const PtrBatch &dW, const PtrBatch &M, const PtrBatch &Y, const PtrBatch &P, double *terms,
-                        int nparts, int *status, float *eps, double *err_terms, const PtrBatch *w_new, int D,
-                        float lambda, int batch, cudaStream_t s);
+                        const PtrBatch &dW, const PtrBatch &M, const PtrBatch &Y, const PtrBatch &P, float *Yc,
+                        float *Pc, float *split, double *terms, int nparts, int *status, float *eps,
+                        double *err_terms, const PtrBatch *w_new, int D, float lambda, int batch, int *err_flag,
+                        cudaStream_t s);
 }
 
 namespace ispa {
@@ -100,8 +101,8 @@ constexpr int kEpsParts = 64;
 
 size_t solve_ws_bytes(int n_layers, int D) {
     const size_t b = (size_t)std::min(n_layers, kMaxBatch);
-    const size_t mat = align_up((size_t)D * D * sizeof(float), 256);
-    return b * 3 * mat + align_up(5 * b * kEpsParts * sizeof(double), 256);
+    const size_t mat = (size_t)D * D * sizeof(float);   // D is a multiple of 64: 256-byte multiple
+    return b * 9 * mat + align_up(5 * b * kEpsParts * sizeof(double), 256);
 }
 
 int check_desc(const ispa_attn_desc *d, bool need_ranges) {
@@ -367,10 +368,17 @@ int ispa_solve_absorb(const ispa_stats *per_layer, int n_layers, const void *con
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     CUDA_CHECK_RET(cudaMemsetAsync(layer_status, 0, sizeof(int) * n_layers, s), "memset layer_status");
 
-    const size_t mat = align_up((size_t)D * D * sizeof(float), 256);
+    // workspace: M, Y, P blocks of bmax D x D float32 matrices each (contiguous per block), the
+    // 3xTF32 split operands (6 blocks), then the trace partial sums
+    const size_t mat = (size_t)D * D * sizeof(float);
     const int bmax = std::min(n_layers, kMaxBatch);
     char *wsb = static_cast<char *>(ws);
-    double *terms = reinterpret_cast<double *>(wsb + (size_t)bmax * 3 * mat);
+    char *Mb = wsb, *Yb = wsb + (size_t)bmax * mat, *Pb = wsb + 2 * (size_t)bmax * mat;
+    float *split = reinterpret_cast<float *>(wsb + 3 * (size_t)bmax * mat);
+    double *terms = reinterpret_cast<double *>(wsb + 9 * (size_t)bmax * mat);
+    int *flag = nullptr;
+    rc = device_error_flag(&flag);
+    if (rc != ISPA_OK) return rc;
     for (int l0 = 0; l0 < n_layers; l0 += kMaxBatch) {
         const int b = std::min(kMaxBatch, n_layers - l0);
         PtrBatch G, C, H, W, DW, M, Y, P, WN;
@@ -379,15 +387,16 @@ int ispa_solve_absorb(const ispa_stats *per_layer, int n_layers, const void *con
             G.p[z] = st.G; C.p[z] = st.C; H.p[z] = st.H;
             W.p[z] = const_cast<void *>(w_o[l0 + z]);
             DW.p[z] = dW + (size_t)(l0 + z) * D * D;
-            M.p[z] = wsb + (size_t)z * 3 * mat;
-            Y.p[z] = wsb + (size_t)z * 3 * mat + mat;
-            P.p[z] = wsb + (size_t)z * 3 * mat + 2 * mat;
+            M.p[z] = Mb + (size_t)z * mat;
+            Y.p[z] = Yb + (size_t)z * mat;
+            P.p[z] = Pb + (size_t)z * mat;
             if (w_new) WN.p[z] = w_new[l0 + z];
         }
         cudaError_t e = solve_batch(G, C, H, W, w_dtype == ISPA_BF16 ? ElemType::BF16 : ElemType::F32, DW, M, Y, P,
-                                    terms, kEpsParts, layer_status + l0, eps + l0,
+                                    reinterpret_cast<float *>(Yb), reinterpret_cast<float *>(Pb), split, terms,
+                                    kEpsParts, layer_status + l0, eps + l0,
                                     err_terms ? err_terms + 2 * (size_t)l0 : nullptr, w_new ? &WN : nullptr, D, lambda,
-                                    b, s);
+                                    b, flag, s);
         if (e != cudaSuccess) return cuda_fail(e, "absorb solve");
     }
     return ISPA_OK;

@@ -92,6 +92,12 @@ cudaError_t launch_stats_bf16(const void *a_loc, const void *r, int n, int D, fl
 struct PtrBatch {
     void *p[kMaxBatch];
 };
+
+// 3xTF32 tensor-core GEMM for D x D products (gemm_tf32_sm100.cu).
+cudaError_t launch_split_tf32(const PtrBatch &src, ElemType t, float *hi, float *lo, int rows, int cols,
+                              bool transpose, int batch, cudaStream_t s);
+cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh, const float *Bl, float *C, int M,
+                               int N, int K, int batch, int *err_flag, cudaStream_t s);
 cudaError_t launch_fill_shifted(const PtrBatch &src, const PtrBatch &dst, int D, float lambda, int batch,
                                 cudaStream_t s);
 cudaError_t launch_potrf_diag(const PtrBatch &M, int D, int k0, int nb, int *status, int batch, cudaStream_t s);

@@ -1,0 +1,301 @@
+// Float32-accurate batched GEMM on the sm_100a tensor cores (3xTF32), for the absorb solve's
+// D x D products [ISPA §3.2, §3.3]: Y = C W, and G dW, H W, G W for the error traces.
+//
+// Each float32 operand X is split once into X_hi = X rounded to TF32 (11 significant bits)
+// and X_lo = X - X_hi (exact in float32; the tensor core keeps its leading 11 bits). The
+// product is accumulated in float32 TMEM as A_hi B_hi + A_hi B_lo + A_lo B_hi; the dropped
+// A_lo B_lo term and the truncation of the lo parts are ~2^-22 relative, i.e. float32-level
+// accuracy. A bf16 operand is exact in TF32 (lo = 0) and costs two terms instead of three.
+//
+// Layouts: both MMA operands are K-major (32-bit K-major tiles with the 128-byte swizzle):
+// A split as [batch][M][K], B split *and transposed* as [batch][N][K] (the split kernel for B
+// writes B^T), so C = A B = A (B^T)^T. C [batch][M][N] row-major float32, overwritten. The
+// split operands are contiguous batches in the workspace, so one 3-D tensor map covers all
+// layers. CTA = one 128 x 128 tile of one batch entry; K in steps of 32 through a 3-stage
+// ring; warp 0 TMA, warp 1 lane 0 MMA (kind::tf32, K = 8 per instruction), warps 4..7
+// epilogue.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace ispa {
+namespace {
+
+constexpr int kTile = 128;
+constexpr int kKStep = 32;                      // fp32 elements per stage = one 128-byte row
+constexpr int kStages = 3;
+constexpr int kThreads = 256;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr int kOpBytes = kTile * kKStep * 4;    // 16 KB per operand part per stage
+constexpr int kStageBytes = 4 * kOpBytes;       // A_hi, A_lo, B_hi, B_lo
+constexpr int kBarOff = kStages * kStageBytes;
+constexpr int kSmem = kBarOff + 128;
+
+__host__ __device__ constexpr uint32_t make_idesc_tf32(int M, int N, bool b_mn) {
+    return (1u << 4)                    // D: f32
+           | (2u << 7)                  // A: tf32
+           | (2u << 10)                 // B: tf32
+           | ((b_mn ? 1u : 0u) << 16)   // B major
+           | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+struct Tf32Params {
+    float *C;
+    int M, N, K;
+    int three_terms;    // B_lo present
+    int *err_flag;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constant__ CUtensorMap tAl,
+                   const __grid_constant__ CUtensorMap tBh, const __grid_constant__ CUtensorMap tBl,
+                   const Tf32Params p) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (ptx::smem_u32(smem) & 1023u) {
+        if (threadIdx.x == 0) atomicCAS(p.err_flag, 0, ISPA_ERR_UNSUPPORTED);
+        return;
+    }
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kBarOff);
+    uint64_t *empty = full + kStages;
+    uint64_t *acc_bar = empty + kStages;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_bar + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int n0 = blockIdx.x * kTile, m0 = blockIdx.y * kTile, z = blockIdx.z;
+    const int n_k = (p.K + kKStep - 1) / kKStep;
+    const uint32_t stage_tx = (p.three_terms ? 4 : 3) * kOpBytes;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&empty[s], 1);
+        }
+        ptx::mbar_init(acc_bar, 1);
+        *abort_flag = 0;
+        ptx::fence_barrier_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, 128);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t pol = ptx::policy_evict_normal();
+            int issued = -1;
+            bool ok = true;
+            for (int kt = 0; kt < n_k; ++kt) {
+                const int s = kt % kStages;
+                ok = ptx::mbar_wait_bounded(&empty[s], ((kt / kStages) & 1) ^ 1, kWaitLimitNs, p.err_flag, abort_flag);
+                if (!ok) break;
+                uint8_t *base = smem + s * kStageBytes;
+                ptx::mbar_arrive_expect_tx(&full[s], stage_tx);
+                const int k0 = kt * kKStep;
+                ptx::tma_load_3d(base, &tAh, &full[s], k0, m0, z, pol);
+                ptx::tma_load_3d(base + kOpBytes, &tAl, &full[s], k0, m0, z, pol);
+                ptx::tma_load_3d(base + 2 * kOpBytes, &tBh, &full[s], k0, n0, z, pol);
+                if (p.three_terms) ptx::tma_load_3d(base + 3 * kOpBytes, &tBl, &full[s], k0, n0, z, pol);
+                issued = kt;
+            }
+            if (!ok)
+                for (int kt = issued - kStages + 1 > 0 ? issued - kStages + 1 : 0; kt <= issued; ++kt)
+                    ptx::mbar_wait_bounded(&full[kt % kStages], (kt / kStages) & 1, kWaitLimitNs, nullptr, nullptr);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = make_idesc_tf32(kTile, kTile, false);
+            const uint32_t sbase = ptx::smem_u32(smem);
+            bool ok = true;
+            for (int kt = 0; kt < n_k && ok; ++kt) {
+                const int s = kt % kStages;
+                ok = ptx::mbar_wait_bounded(&full[s], (kt / kStages) & 1, kWaitLimitNs, p.err_flag, abort_flag);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const uint32_t ah = sbase + s * kStageBytes, al = ah + kOpBytes, bh = al + kOpBytes, bl = bh + kOpBytes;
+#pragma unroll
+                for (int kk = 0; kk < kKStep / 8; ++kk) {
+                    const uint64_t dah = ptx::make_sdesc_sw128(ah + kk * 32, 16, 1024);
+                    const uint64_t dal = ptx::make_sdesc_sw128(al + kk * 32, 16, 1024);
+                    const uint64_t dbh = ptx::make_sdesc_sw128(bh + kk * 32, 16, 1024);
+                    const uint32_t first = (kt == 0 && kk == 0) ? 0u : 1u;
+                    umma_tf32_ss(tmem, dal, dbh, idesc, first);
+                    if (p.three_terms) {
+                        const uint64_t dbl = ptx::make_sdesc_sw128(bl + kk * 32, 16, 1024);
+                        umma_tf32_ss(tmem, dah, dbl, idesc, 1u);
+                    }
+                    umma_tf32_ss(tmem, dah, dbh, idesc, 1u);
+                }
+                ptx::umma_commit(&empty[s]);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                __threadfence_block();
+            }
+            ptx::umma_commit(acc_bar);
+            ptx::mbar_wait_bounded(acc_bar, 0, kWaitLimitNs, p.err_flag, nullptr);
+        }
+    } else if (warp >= 4) {
+        const int wq = warp - 4;
+        const int r = wq * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        const bool ok = ptx::mbar_wait_bounded(acc_bar, 0, kWaitLimitNs, p.err_flag, abort_flag) && !*abort_flag;
+        if (ok) {
+            ptx::tc_fence_after();
+            const int gm = m0 + r;
+            float *crow = p.C + ((size_t)z * p.M + gm) * p.N + n0;
+#pragma unroll 1
+            for (int c = 0; c < kTile / 32; ++c) {
+                uint32_t v[32];
+                ptx::tmem_ld32(tmem + lane_off + c * 32, v);
+                ptx::tmem_wait_ld();
+                if (gm < p.M) {
+#pragma unroll
+                    for (int q = 0; q < 32; q += 4) {
+                        if (n0 + c * 32 + q + 3 < p.N) {
+                            *reinterpret_cast<float4 *>(crow + c * 32 + q) =
+                                make_float4(__uint_as_float(v[q]), __uint_as_float(v[q + 1]), __uint_as_float(v[q + 2]),
+                                            __uint_as_float(v[q + 3]));
+                        } else {
+                            for (int u = 0; u < 4; ++u)
+                                if (n0 + c * 32 + q + u < p.N) crow[c * 32 + q + u] = __uint_as_float(v[q + u]);
+                        }
+                    }
+                }
+            }
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, 128);
+    }
+}
+
+// X_hi = X rounded to TF32 (round to nearest, ties away from zero on the 13 dropped bits),
+// X_lo = X - X_hi, for a batch of float32 or bf16 matrices of n elements, written to
+// contiguous [batch][n] arrays. bf16 inputs are exact in TF32: lo is not written.
+template <typename T>
+__global__ void split_tf32_kernel(PtrBatch src, float *hi, float *lo, size_t n) {
+    const int z = blockIdx.y;
+    const T *s = static_cast<const T *>(src.p[z]);
+    float *h = hi + (size_t)z * n;
+    float *l = lo ? lo + (size_t)z * n : nullptr;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        const float x = to_f32(s[i]);
+        const float xh = __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
+        h[i] = xh;
+        if (l) l[i] = x - xh;
+    }
+}
+
+// The same split of a batch of row-major [rows][cols] matrices, written transposed
+// ([cols][rows]) through a 32 x 32 shared-memory tile so that reads and writes stay coalesced.
+template <typename T>
+__global__ void split_tf32_transposed_kernel(PtrBatch src, float *hi, float *lo, int rows, int cols) {
+    __shared__ float tile[32][33];
+    const int z = blockIdx.z;
+    const T *s = static_cast<const T *>(src.p[z]);
+    const size_t n = (size_t)rows * cols;
+    const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int r = r0 + i, c = c0 + threadIdx.x;
+        tile[i][threadIdx.x] = (r < rows && c < cols) ? to_f32(s[(size_t)r * cols + c]) : 0.f;
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+        const int c = c0 + i, r = r0 + threadIdx.x;
+        if (r < rows && c < cols) {
+            const float x = tile[threadIdx.x][i];
+            const float xh = __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
+            const size_t o = (size_t)z * n + (size_t)c * rows + r;
+            hi[o] = xh;
+            if (lo) lo[o] = x - xh;
+        }
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// [batch][rows][cols] float32, box = (32 cols, box_rows rows, 1), 128-byte swizzle.
+bool make_map(CUtensorMap *m, const float *ptr, int batch, int rows, int cols, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)batch};
+    cuuint64_t strides[2] = {(cuuint64_t)cols * 4, (cuuint64_t)rows * cols * 4};
+    cuuint32_t box[3] = {32, (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_split_tf32(const PtrBatch &src, ElemType t, float *hi, float *lo, int rows, int cols,
+                              bool transpose, int batch, cudaStream_t s) {
+    if (transpose) {
+        const dim3 grid((cols + 31) / 32, (rows + 31) / 32, batch), block(32, 8);
+        if (t == ElemType::BF16) split_tf32_transposed_kernel<bf16><<<grid, block, 0, s>>>(src, hi, nullptr, rows, cols);
+        else split_tf32_transposed_kernel<float><<<grid, block, 0, s>>>(src, hi, lo, rows, cols);
+    } else {
+        const size_t n = (size_t)rows * cols;
+        const int blocks = (int)std::min<size_t>((n + 255) / 256, 1024);
+        if (t == ElemType::BF16) split_tf32_kernel<bf16><<<dim3(blocks, batch), 256, 0, s>>>(src, hi, nullptr, n);
+        else split_tf32_kernel<float><<<dim3(blocks, batch), 256, 0, s>>>(src, hi, lo, n);
+    }
+    note_launch();
+    return cudaGetLastError();
+}
+
+// C[z] = A[z] B[z] for z < batch; A given as (A_hi, A_lo) [batch][M][K], B as (B_hi, B_lo or
+// null) transposed, [batch][N][K], all contiguous float32. M, N multiples of 128; K of 32.
+cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh, const float *Bl, float *C, int M,
+                               int N, int K, int batch, int *err_flag, cudaStream_t s) {
+    if (M % kTile || N % kTile || K % kKStep || batch <= 0) return cudaErrorInvalidValue;
+    CUtensorMap ah, al, bh, bl;
+    if (!make_map(&ah, Ah, batch, M, K, kTile) || !make_map(&al, Al, batch, M, K, kTile) ||
+        !make_map(&bh, Bh, batch, N, K, kTile) || !make_map(&bl, Bl ? Bl : Bh, batch, N, K, kTile))
+        return cudaErrorInvalidValue;
+    Tf32Params p;
+    p.C = C; p.M = M; p.N = N; p.K = K;
+    p.three_terms = Bl != nullptr;
+    p.err_flag = err_flag;
+    cudaError_t e = cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess) return e;
+    gemm_tf32x3_kernel<<<dim3(N / kTile, M / kTile, batch), kThreads, kSmem, s>>>(ah, al, bh, bl, p);
+    note_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace ispa

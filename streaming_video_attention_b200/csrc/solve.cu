@@ -219,24 +219,35 @@ static GemmBatch make_gemm_batch(const PtrBatch &A, size_t offA, const PtrBatch 
 //   G, C, H: statistics; W: weights of type wt; dW: output; M, Y: D*D float scratch each;
 //   P: D*D float scratch; terms: 5 * batch * nparts doubles; status: batch ints (zeroed).
 cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H, const PtrBatch &W, ElemType wt,
-                        const PtrBatch &dW, const PtrBatch &M, const PtrBatch &Y, const PtrBatch &P, double *terms,
-                        int nparts, int *status, float *eps, double *err_terms, const PtrBatch *w_new, int D,
-                        float lambda, int batch, cudaStream_t s) {
+                        const PtrBatch &dW, const PtrBatch &M, const PtrBatch &Y, const PtrBatch &P, float *Yc,
+                        float *Pc, float *split, double *terms, int nparts, int *status, float *eps,
+                        double *err_terms, const PtrBatch *w_new, int D, float lambda, int batch, int *err_flag,
+                        cudaStream_t s) {
     const size_t n = (size_t)D * D;
     const size_t ew = wt == ElemType::BF16 ? 2 : 4;
     const int fill_blocks = (int)std::min<size_t>((n + 255) / 256, 1024);
+    // D x D products on the tensor cores (3xTF32) when D is a multiple of 128; the split
+    // operands live in `split`: A_hi, A_lo, B_hi, B_lo, W_hi, W_lo, each [batch][D][D].
+    const bool tc = (D % 128 == 0) && split != nullptr;
+    const size_t bn = (size_t)batch * n;
+    float *Ahi = split, *Alo = split + bn, *Bhi = split + 2 * bn, *Blo = split + 3 * bn;
+    float *Whi = split + 4 * bn, *Wlo = wt == ElemType::BF16 ? nullptr : split + 5 * bn;
+    if (tc) ISPA_TRY(launch_split_tf32(W, wt, Whi, Wlo, D, D, true, batch, s));
 
     // M = G + lambda I
     fill_shifted_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(G, M, D, lambda); note_launch();
     ISPA_TRY(cudaGetLastError());
 
     // Y = C W, and dW <- Y (solved in place below)
-    {
+    if (tc) {
+        ISPA_TRY(launch_split_tf32(C, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Yc, D, D, D, batch, err_flag, s));
+    } else {
         GemmDesc d{D, D, D, D, D, D, true, false, ElemType::F32, wt, ElemType::F32, 1.f, 0.f, false, batch};
         ISPA_TRY(launch_gemm_simt(d, make_gemm_batch(C, 0, W, 0, Y, 0, batch, 4, ew), s));
-        copy_f32_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(Y, dW, n); note_launch();
-        ISPA_TRY(cudaGetLastError());
     }
+    copy_f32_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(Y, dW, n); note_launch();
+    ISPA_TRY(cudaGetLastError());
 
     // Cholesky factorisation, blocked
     const int nblk = D / NB;
@@ -285,22 +296,37 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
     const dim3 rgrid(nparts, batch);
     GemmDesc full{D, D, D, D, D, D, true, false, ElemType::F32, ElemType::F32, ElemType::F32, 1.f, 0.f, false, batch};
     // t0 = tr(dW^T G dW)
-    ISPA_TRY(launch_gemm_simt(full, make_gemm_batch(G, 0, dW, 0, P, 0, batch, 4, 4), s));
+    if (tc) {
+        ISPA_TRY(launch_split_tf32(G, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
+        ISPA_TRY(launch_split_tf32(dW, ElemType::F32, Bhi, Blo, D, D, true, batch, s));
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Bhi, Blo, Pc, D, D, D, batch, err_flag, s));
+    } else {
+        ISPA_TRY(launch_gemm_simt(full, make_gemm_batch(G, 0, dW, 0, P, 0, batch, 4, 4), s));
+    }
     dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, P, n, terms + 0 * (size_t)batch * nparts); note_launch();
     // t1 = tr(dW^T C W)
     dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, Y, n, terms + 1 * (size_t)batch * nparts); note_launch();
-    // t2 = tr(W^T H W), t3 = tr(W^T G W), t4 = tr(W^T C W)
+    // t3 = tr(W^T G W) first while G's split is in place, then t2 = tr(W^T H W); t4 = tr(W^T C W)
     GemmDesc fw = full;
     fw.b_type = wt;
-    ISPA_TRY(launch_gemm_simt(fw, make_gemm_batch(H, 0, W, 0, P, 0, batch, 4, ew), s));
+    if (tc) {
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Pc, D, D, D, batch, err_flag, s));
+    } else {
+        ISPA_TRY(launch_gemm_simt(fw, make_gemm_batch(G, 0, W, 0, P, 0, batch, 4, ew), s));
+    }
+    if (wt == ElemType::BF16) { dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, P, n, terms + 3 * (size_t)batch * nparts); note_launch(); }
+    else { dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, P, n, terms + 3 * (size_t)batch * nparts); note_launch(); }
+    if (tc) {
+        ISPA_TRY(launch_split_tf32(H, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Pc, D, D, D, batch, err_flag, s));
+    } else {
+        ISPA_TRY(launch_gemm_simt(fw, make_gemm_batch(H, 0, W, 0, P, 0, batch, 4, ew), s));
+    }
     if (wt == ElemType::BF16) { dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, P, n, terms + 2 * (size_t)batch * nparts); note_launch(); }
     else { dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, P, n, terms + 2 * (size_t)batch * nparts); note_launch(); }
-    ISPA_TRY(launch_gemm_simt(fw, make_gemm_batch(G, 0, W, 0, P, 0, batch, 4, ew), s));
     if (wt == ElemType::BF16) {
-        dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, P, n, terms + 3 * (size_t)batch * nparts); note_launch();
         dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, Y, n, terms + 4 * (size_t)batch * nparts); note_launch();
     } else {
-        dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, P, n, terms + 3 * (size_t)batch * nparts); note_launch();
         dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, Y, n, terms + 4 * (size_t)batch * nparts); note_launch();
     }
     ISPA_TRY(cudaGetLastError());

@@ -180,7 +180,9 @@ def test_solve_absorb_matches_oracle(dtype, D, L):
         assert rel_fro(to_numpy(dW[l]), dW_ref) < 1e-3, l
         e = oracle.reconstruction_error(G, C, H, W_np[l], dW_ref)
         eps_ref.append(e["eps"])
-        assert abs(float(eps[l]) - e["eps"]) <= 1e-3 * abs(e["eps"]) + 1e-6, (l, float(eps[l]), e["eps"])
+        # eps = E^2/T^2 with E^2 a difference of traces of order T^2: float32-accurate products
+        # (3xTF32 on the tensor cores, float32 accumulation) leave an absolute floor of a few 1e-6
+        assert abs(float(eps[l]) - e["eps"]) <= 1e-3 * abs(e["eps"]) + 4e-6, (l, float(eps[l]), e["eps"])
         assert abs(float(terms[l, 1]) - e["T2"]) <= 1e-4 * abs(e["T2"])
         wn_ref = W_np[l].astype(np.float64) + dW_ref
         assert rel_fro(to_numpy(W_new[l]), wn_ref) < (1e-5 if dtype == "fp32" else 1e-2)
