@@ -452,11 +452,18 @@ int ispa_local_attn(const ispa_attn_desc *desc, const void *q, const void *k_loc
     rc = run_attention(desc, q, k_loc, v_loc, o, lse_out, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, true, s);
     if (rc != ISPA_OK) return rc;
     if (w_new) {
-        const ElemType t = desc->dtype == ISPA_BF16 ? ElemType::BF16 : ElemType::F32;
-        GemmDesc g{desc->n_q, D, D, D, D, D, true, false, t, t, t, 1.f, 0.f, false, 1};
-        GemmBatch b;
-        b.A[0] = o; b.B[0] = w_new; b.C[0] = y;
-        CUDA_CHECK_RET(launch_gemm_simt(g, b, s), "projection GEMM");
+        if (desc->dtype == ISPA_BF16 && D % 128 == 0) {
+            int *flag = nullptr;
+            rc = device_error_flag(&flag);
+            if (rc != ISPA_OK) return rc;
+            CUDA_CHECK_RET(launch_gemm_bf16(o, w_new, y, desc->n_q, D, D, flag, s), "projection GEMM (tcgen05)");
+        } else {
+            const ElemType t = desc->dtype == ISPA_BF16 ? ElemType::BF16 : ElemType::F32;
+            GemmDesc g{desc->n_q, D, D, D, D, D, true, false, t, t, t, 1.f, 0.f, false, 1};
+            GemmBatch b;
+            b.A[0] = o; b.B[0] = w_new; b.C[0] = y;
+            CUDA_CHECK_RET(launch_gemm_simt(g, b, s), "projection GEMM");
+        }
     }
     return ISPA_OK;
 }

@@ -88,6 +88,10 @@ cudaError_t launch_gemm_simt(const GemmDesc &d, const GemmBatch &b, cudaStream_t
 cudaError_t launch_stats_bf16(const void *a_loc, const void *r, int n, int D, float *G, float *C,
                                float *H, int *err_flag, cudaStream_t s);
 
+// y[M][N] = A[M][K] W[K][N], bf16 in and out, tensor cores (gemm_bf16_sm100.cu).
+cudaError_t launch_gemm_bf16(const void *A, const void *W, void *y, int M, int N, int K, int *err_flag,
+                             cudaStream_t s);
+
 // Solve-phase kernels (float32, batched over layers).
 struct PtrBatch {
     void *p[kMaxBatch];
