@@ -54,6 +54,9 @@ def parse_args(argv=None):
                     help="episode: the full step (default). call / local / solve: one layer's fused split "
                          "attention at the last warmup chunk, one L-layer local attention with projection, or "
                          "the batched solve alone (kernel-level timing, also the target of ncu captures)")
+    ap.add_argument("--attn-kernel", choices=["auto", "single", "pair"], default="auto",
+                    help="bf16 head_dim-128 attention kernel: one CTA per query tile, or CTA pairs "
+                         "(cta_group::2); auto = the library's default")
     return ap.parse_args(argv)
 
 
@@ -556,6 +559,10 @@ def unit_arm(args, cfg):
 def main(argv=None):
     args = parse_args(argv)
     cfg = synth.CONFIGS[args.config]
+    if args.impl != "reference":
+        from streaming_video_attention_b200 import ispa
+        ispa.ispa_set_attn_kernel({"auto": ispa.ISPA_ATTN_AUTO, "single": ispa.ISPA_ATTN_SINGLE,
+                                   "pair": ispa.ISPA_ATTN_PAIR}[args.attn_kernel])
     if args.mode != "episode":
         return unit_arm(args, cfg)
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -193,6 +193,9 @@ int check_ws(void *ws, size_t have, size_t need) {
     return ISPA_OK;
 }
 
+// Kernel used by bf16 head_dim-128 attention (ispa_set_attn_kernel).
+std::atomic<int> g_attn_kernel{ISPA_ATTN_AUTO};
+
 int run_attention(const ispa_attn_desc *d, const void *q, const void *k, const void *v, void *o_full, float *lse_full,
                   void *o_loc, float *lse_loc, void *o_hist, float *lse_hist, void *a_ops, void *r_ops,
                   bool local_only, cudaStream_t s) {
@@ -209,7 +212,13 @@ int run_attention(const ispa_attn_desc *d, const void *q, const void *k, const v
     a.scale = d->scale;
     a.segs = make_segments(d, local_only);
     a.err_flag = flag;
-    cudaError_t e = d->dtype == ISPA_FP32 ? launch_attn_simt_f32(a, s) : launch_attn_bf16(a, s);
+    cudaError_t e;
+    if (d->dtype == ISPA_FP32)
+        e = launch_attn_simt_f32(a, s);
+    else if (d->head_dim == 128 && g_attn_kernel.load(std::memory_order_relaxed) == ISPA_ATTN_PAIR)
+        e = launch_attn_bf16_2sm(a, s);
+    else
+        e = launch_attn_bf16(a, s);
     if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
     return ISPA_OK;
 }
@@ -466,6 +475,12 @@ int ispa_local_attn(const ispa_attn_desc *desc, const void *q, const void *k_loc
         }
     }
     return ISPA_OK;
+}
+
+int ispa_set_attn_kernel(int choice) {
+    if (choice != ISPA_ATTN_AUTO && choice != ISPA_ATTN_SINGLE && choice != ISPA_ATTN_PAIR)
+        return fail(ISPA_ERR_INVALID_ARG, "ispa_set_attn_kernel: unknown choice %d", choice);
+    return g_attn_kernel.exchange(choice);
 }
 
 int ispa_device_status(ispa_stream_t stream) {

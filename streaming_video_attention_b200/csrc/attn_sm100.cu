@@ -336,13 +336,17 @@ attn_split_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             ptx::tmem_st32(tS(st) + lane_off, &pk[0]);
             ptx::tmem_st32(tS(st) + lane_off + 32, &pk[32]);
             ptx::tmem_wait_st();
-            // PV_{j-1} must be complete before O may be rescaled (and before P_{j} is handed over
-            // when it goes into the accumulator PV_{j-1} wrote).
-            if (j >= 1) {
+            // O may be rescaled only once PV_{j-1} is complete. Without a rescale there is nothing
+            // to wait for: PV_j queues behind PV_{j-1} on the tensor pipe, and P_j's buffer was
+            // last read by PV_{j-2}, which completed before S_j (s_full tracks every earlier MMA).
+            // The same fact keeps the o_bar phase here at j-1 or j, so the parity wait is exact.
+            // The last tile always waits, so that the epilogue's wait (phase n-1) is exact too.
+            const bool rescale_warp = __any_sync(0xffffffffu, rescale);
+            if ((rescale_warp || j == n_tiles - 1) && j >= 1) {
                 ok = ptx::mbar_wait_bounded(o_bar, (j - 1) & 1, kWaitLimitNs, p.err_flag, abort_flag);
                 if (!ok) break;
             }
-            if (__any_sync(0xffffffffu, rescale)) {
+            if (rescale_warp) {
                 ptx::tc_fence_after();
 #pragma unroll
                 for (int c = 0; c < HD / 16; ++c) {

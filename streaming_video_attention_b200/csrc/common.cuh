@@ -63,6 +63,7 @@ struct AttnArgs {
 cudaError_t launch_attn_simt_f32(const AttnArgs &a, cudaStream_t s);
 cudaError_t launch_attn_simt_bf16(const AttnArgs &a, cudaStream_t s);
 cudaError_t launch_attn_bf16(const AttnArgs &a, cudaStream_t s);   // tcgen05 path
+cudaError_t launch_attn_bf16_2sm(const AttnArgs &a, cudaStream_t s);   // tcgen05 CTA-pair path, head_dim 128
 
 // Batched SIMT GEMM: C_z[m][n] = alpha * sum_k A_z(m,k) B_z(k,n) + beta * C_z[m][n].
 // A_z(m,k) = A[m*lda + k] if a_kcontig else A[k*lda + m]; B_z(k,n) = B[n*ldb + k] if
@@ -102,16 +103,5 @@ cudaError_t launch_split_tf32(const PtrBatch &src, ElemType t, float *hi, float 
                               bool transpose, int batch, cudaStream_t s);
 cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh, const float *Bl, float *C, int M,
                                int N, int K, int batch, int *err_flag, cudaStream_t s);
-cudaError_t launch_fill_shifted(const PtrBatch &src, const PtrBatch &dst, int D, float lambda, int batch,
-                                cudaStream_t s);
-cudaError_t launch_potrf_diag(const PtrBatch &M, int D, int k0, int nb, int *status, int batch, cudaStream_t s);
-cudaError_t launch_trsm_panel(const PtrBatch &M, int D, int k0, int nb, int batch, cudaStream_t s);
-cudaError_t launch_trsv_block(const PtrBatch &L, const PtrBatch &X, int D, int k0, int nb, bool transpose,
-                              int batch, cudaStream_t s);
-cudaError_t launch_trace_terms(const PtrBatch &X, const PtrBatch &P, int D, int which, int ncols_x_is_w_bf16,
-                               double *partials, int nparts, int batch, cudaStream_t s);
-cudaError_t launch_copy_f32(const PtrBatch &src, const PtrBatch &dst, size_t n, int batch, cudaStream_t s);
-cudaError_t launch_convert_w(const PtrBatch &w, ElemType t, const PtrBatch &out, size_t n, int batch,
-                             cudaStream_t s);
 
 }  // namespace ispa

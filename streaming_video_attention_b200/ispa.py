@@ -30,7 +30,7 @@ ISPA_FP32 = 1
 EXPORTS = (
     "ispa_attn_split", "ispa_attn_split_noalloc", "ispa_accum_stats", "ispa_stats_reset", "ispa_solve_absorb", "ispa_select_layers",
     "ispa_local_attn", "ispa_workspace_bytes", "ispa_device_status", "ispa_selftest_bounded_wait",
-    "ispa_selftest_exp2_poly", "ispa_kernel_launches", "ispa_last_error", "ispa_version",
+    "ispa_selftest_exp2_poly", "ispa_set_attn_kernel", "ispa_kernel_launches", "ispa_last_error", "ispa_version",
 )
 
 
@@ -205,6 +205,17 @@ def ispa_device_status(stream=None) -> int:
 
 def ispa_selftest_exp2_poly(x: torch.Tensor, y: torch.Tensor, stream=None) -> None:
     _check(lib().ispa_selftest_exp2_poly(_p(x), _p(y), x.numel(), _stream(stream)), "ispa_selftest_exp2_poly")
+
+
+ISPA_ATTN_AUTO, ISPA_ATTN_SINGLE, ISPA_ATTN_PAIR = 0, 1, 2
+
+
+def ispa_set_attn_kernel(choice: int) -> int:
+    """Choose the bf16 head_dim-128 attention kernel; returns the previous choice."""
+    rc = lib().ispa_set_attn_kernel(int(choice))
+    if rc < 0:
+        _check(rc, "ispa_set_attn_kernel")
+    return rc
 
 
 def ispa_kernel_launches() -> int:

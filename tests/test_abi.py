@@ -80,3 +80,14 @@ def test_select_layers_matches_oracle_on_random_errors():
         eps = eps.astype(np.float32).tolist()
         K = int(rng.integers(0, L + 2))
         assert ispa.ispa_select_layers(eps, K) == oracle.select_layers(eps, K)
+
+
+def test_set_attn_kernel_choice_round_trips():
+    prev = ispa.ispa_set_attn_kernel(ispa.ISPA_ATTN_PAIR)
+    try:
+        assert ispa.ispa_set_attn_kernel(ispa.ISPA_ATTN_SINGLE) == ispa.ISPA_ATTN_PAIR
+        with pytest.raises(ispa.IspaError):
+            ispa.ispa_set_attn_kernel(7)
+        assert ispa.ispa_set_attn_kernel(ispa.ISPA_ATTN_AUTO) == ispa.ISPA_ATTN_SINGLE
+    finally:
+        ispa.ispa_set_attn_kernel(prev)
