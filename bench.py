@@ -358,12 +358,13 @@ def config_block(cfg, n):
 
 
 def ispa_arm(args, cfg, rank, world, local_rank):
-    from streaming_video_attention_b200 import ispa
+    from streaming_video_attention_b200 import ispa, replicas
     from streaming_video_attention_b200.session import IspaSession
 
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     ispa.lib()
+    cfg = replicas.replica_config(cfg, rank)
     threads = max(1, (os.cpu_count() or 8) // max(1, int(os.environ.get("LOCAL_WORLD_SIZE", world))))
     t0 = time.time()
     wl = Workload(cfg, threads)
@@ -386,8 +387,7 @@ def ispa_arm(args, cfg, rank, world, local_rank):
     time.sleep(0.4)
     timers = []
     launches0 = ispa.ispa_kernel_launches()
-    if world > 1:
-        torch.distributed.barrier()
+    replicas.barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
@@ -395,17 +395,11 @@ def ispa_arm(args, cfg, rank, world, local_rank):
         run_episode(sess, dev, out, timers)
     e1.record()
     torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+    replicas.barrier()
     launches = ispa.ispa_kernel_launches() - launches0
     clk = clocks.stop()
-    elapsed = e0.elapsed_time(e1) / 1e3
-    t = torch.tensor([elapsed], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    elapsed = float(t.item())
-    tokens = world * args.steps * (cfg.warmup_chunks + 1) * cfg.n_q
-    value = tokens / elapsed
+    value, elapsed = replicas.job_throughput(args.steps * (cfg.warmup_chunks + 1) * cfg.n_q,
+                                             e0.elapsed_time(e1) / 1e3, device)
     ms_per_step = elapsed / args.steps * 1e3
 
     # roofline of the fused split-attention + statistics call (dominant kernel pair)
@@ -434,8 +428,7 @@ def ispa_arm(args, cfg, rank, world, local_rank):
                             sess.eps.cpu())
         run_once()
         torch.cuda.synchronize()
-        if world > 1:
-            torch.distributed.barrier()
+        replicas.barrier()
         torch.cuda.synchronize()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record()
@@ -443,12 +436,11 @@ def ispa_arm(args, cfg, rank, world, local_rank):
             run_once()
         f1.record()
         torch.cuda.synchronize()
-        et = torch.tensor([f0.elapsed_time(f1) / 1e3], dtype=torch.float64, device=device)
-        if world > 1:
-            torch.distributed.all_reduce(et, op=torch.distributed.ReduceOp.MAX)
-        e2e = {"value": world * args.e2e_steps * (cfg.warmup_chunks + 1) * cfg.n_q / float(et.item()), "unit": UNIT,
+        e2e_value, et = replicas.job_throughput(args.e2e_steps * (cfg.warmup_chunks + 1) * cfg.n_q,
+                                                f0.elapsed_time(f1) / 1e3, device)
+        e2e = {"value": e2e_value, "unit": UNIT,
                "h2d_bytes_per_step": wl.h2d_bytes(), "d2h_bytes_per_step": d2h,
-               "ms_per_step": float(et.item()) / args.e2e_steps * 1e3}
+               "ms_per_step": et / args.e2e_steps * 1e3}
 
     assert ispa.ispa_device_status() == ispa.ISPA_OK
 
