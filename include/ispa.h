@@ -183,8 +183,9 @@ int ispa_selftest_bounded_wait(unsigned limit_us, ispa_stream_t stream);
 
 /* ispa_selftest_exp2_poly -- test hook: y[i] = 2^x[i] computed by the FMA-pipe
  * exponential the split-attention softmax uses for part of its weights (range reduction
- * + degree-3 polynomial). x, y: device float32 [n]. Valid for x <= 64; x < -125 gives a
- * value below 3e-38. */
+ * + degree-3 polynomial): elements 2q, 2q+1 by its packed two-lane form, an odd last
+ * element by its scalar form. x, y: device float32 [n]. Valid for x <= 64; x < -125 gives
+ * a value below 3e-38. */
 int ispa_selftest_exp2_poly(const float *x, float *y, int n, ispa_stream_t stream);
 
 /* ispa_set_attn_kernel -- choose the tensor-core kernel that bf16 attention calls with

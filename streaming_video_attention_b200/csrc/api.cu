@@ -237,8 +237,18 @@ __global__ void bounded_wait_selftest_kernel(uint64_t limit_ns, int *flag) {
     __syncthreads();
 }
 
+// Pairs (2q, 2q+1) through the packed form the softmax uses; an odd last element through the
+// scalar form.
 __global__ void exp2_poly_selftest_kernel(const float *x, float *y, int n) {
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) y[i] = ptx::exp2_poly(x[i]);
+    for (int q = blockIdx.x * blockDim.x + threadIdx.x; 2 * q < n; q += gridDim.x * blockDim.x) {
+        if (2 * q + 1 < n) {
+            const uint64_t r = ptx::exp2_poly2(ptx::f2_pack(x[2 * q], x[2 * q + 1]));
+            y[2 * q] = ptx::f2_lo(r);
+            y[2 * q + 1] = ptx::f2_hi(r);
+        } else {
+            y[2 * q] = ptx::exp2_poly(x[2 * q]);
+        }
+    }
 }
 
 }  // namespace

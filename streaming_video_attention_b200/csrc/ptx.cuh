@@ -116,6 +116,54 @@ __device__ __forceinline__ float exp2_poly(float x) {
     return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// ---- packed float32 pairs (sm_100 f32x2: two lanes of work per instruction) ----------
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+    return d;
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return lo;
+}
+__device__ __forceinline__ float f2_hi(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return hi;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// exp2_poly on both halves of a pair (the same reduction and polynomial, packed arithmetic).
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x) {
+    const float x0 = fmaxf(f2_lo(x), -125.0f), x1 = fmaxf(f2_hi(x), -125.0f);
+    const uint64_t xc = f2_pack(x0, x1);
+    const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
+    const uint64_t t = f2_add(xc, magic);
+    const uint64_t f = f2_sub(xc, f2_sub(t, magic));
+    uint64_t p = f2_fma(f2_pack(0.055174145847558975f, 0.055174145847558975f), f,
+                        f2_pack(0.24261757731437683f, 0.24261757731437683f));
+    p = f2_fma(p, f, f2_pack(0.6932610869407654f, 0.6932610869407654f));
+    p = f2_fma(p, f, f2_pack(0.9999275803565979f, 0.9999275803565979f));
+    const float r0 = __int_as_float(__float_as_int(f2_lo(p)) + (__float_as_int(f2_lo(t)) << 23));
+    const float r1 = __int_as_float(__float_as_int(f2_hi(p)) + (__float_as_int(f2_hi(t)) << 23));
+    return f2_pack(r0, r1);
+}
+
 // ---- TMA (no multicast anywhere in this library) ------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const void *desc) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(desc)) : "memory");
@@ -263,6 +311,57 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// ---- warp-uniform issue --------------------------------------------------------------
+// Called by all 32 lanes of a converged warp; one lane (elect.sync) issues. Keeping the whole
+// warp on the path lets the compiler hold descriptors and addresses in uniform registers,
+// which the tcgen05 and TMA instructions read directly: a single-lane branch around these
+// instructions costs several times their issue time.
+__device__ __forceinline__ void umma_f16_ss_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_f16_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit_warp(uint64_t *bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx_warp(uint64_t *bar, uint32_t bytes) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t.reg .b64 st;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
+        "@e mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(smem_u32(bar)),
+        "r"(bytes)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_warp(void *smem_dst, const void *desc, uint64_t *bar, int c0, int c1,
+                                                 int c2, uint64_t cache_hint) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
+        "@e cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5}], [%2], %6;\n\t}" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(desc)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "l"(cache_hint)
+        : "memory");
+}
 
 // ---- CTA pairs (cluster of 2, tcgen05 cta_group::2) ----------------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank() {

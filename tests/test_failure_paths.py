@@ -55,7 +55,8 @@ def test_workspace_errors_are_reported():
 def test_fma_pipe_exponential_error_bound():
     """The softmax's FMA-pipe 2^x stays within 1e-4 relative of the exact value (bf16 rounding
     of the weights it feeds is 2^-9 = 2e-3), and agrees with CUDA's exp2f on the same inputs."""
-    x = torch.cat([torch.linspace(-125.0, 8.0, 1 << 20), torch.tensor([0.0, -0.5, 0.5, 1.0, -1.0, 7.99])]).cuda()
+    # odd length: pairs go through the packed form, the last element through the scalar one
+    x = torch.cat([torch.linspace(-125.0, 8.0, 1 << 20), torch.tensor([0.0, -0.5, 0.5, 1.0, -1.0, 7.99, 3.3])]).cuda()
     y = torch.empty_like(x)
     ispa.ispa_selftest_exp2_poly(x, y)
     torch.cuda.synchronize()
