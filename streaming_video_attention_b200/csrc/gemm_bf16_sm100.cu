@@ -67,54 +67,54 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constant__
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    // producer and MMA warps stay converged; one elected lane issues (uniform registers)
     if (warp == 0) {
-        if (lane == 0) {
-            const uint64_t pol_a = ptx::policy_evict_normal();
-            const uint64_t pol_b = ptx::policy_evict_last();
-            int issued = -1;
-            bool ok = true;
-            for (int kt = 0; kt < n_k; ++kt) {
-                const int s = kt % kStages;
-                ok = ptx::mbar_wait_bounded(&empty[s], ((kt / kStages) & 1) ^ 1, kWaitLimitNs, p.err_flag, abort_flag);
-                if (!ok) break;
-                uint8_t *base = smem + s * kStageBytes;
-                ptx::mbar_arrive_expect_tx(&full[s], kStageBytes);
-                const int k0 = kt * kKStep;
-                ptx::tma_load_2d(base, &tA, &full[s], k0, m0, pol_a);
-                for (int b = 0; b < 2; ++b)
-                    ptx::tma_load_2d(base + kABytes + b * (kKStep * 128), &tB, &full[s], n0 + b * 64, k0, pol_b);
-                issued = kt;
-            }
-            if (!ok)
-                for (int kt = issued - kStages + 1 > 0 ? issued - kStages + 1 : 0; kt <= issued; ++kt)
-                    ptx::mbar_wait_bounded(&full[kt % kStages], (kt / kStages) & 1, kWaitLimitNs, nullptr, nullptr);
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc = ptx::make_idesc_bf16(kTile, kTile, false, true);
-            const uint32_t sbase = ptx::smem_u32(smem);
-            bool ok = true;
-            for (int kt = 0; kt < n_k && ok; ++kt) {
-                const int s = kt % kStages;
-                ok = ptx::mbar_wait_bounded(&full[s], (kt / kStages) & 1, kWaitLimitNs, p.err_flag, abort_flag);
-                if (!ok) break;
-                ptx::tc_fence_after();
-                const uint32_t a = sbase + s * kStageBytes, b = a + kABytes;
+        const uint64_t pol_a = ptx::policy_evict_normal();
+        const uint64_t pol_b = ptx::policy_evict_last();
+        int issued = -1;
+        bool ok = true;
+        for (int kt = 0; kt < n_k; ++kt) {
+            const int s = kt % kStages;
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&empty[s], ((kt / kStages) & 1) ^ 1, kWaitLimitNs,
+                                                                 p.err_flag, abort_flag));
+            if (!ok) break;
+            uint8_t *base = smem + s * kStageBytes;
+            ptx::mbar_arrive_expect_tx_warp(&full[s], kStageBytes);
+            const int k0 = kt * kKStep;
+            ptx::tma_load_2d_warp(base, &tA, &full[s], k0, m0, pol_a);
 #pragma unroll
-                for (int kk = 0; kk < kKStep / 16; ++kk) {
-                    const uint64_t da = ptx::make_sdesc_sw128(a + kk * 32, 16, 1024);
-                    const uint64_t db = ptx::make_sdesc_sw128(b + kk * 2048, kKStep * 128, 1024);
-                    ptx::umma_f16_ss(tmem, da, db, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
-                }
-                ptx::umma_commit(&empty[s]);
-            }
-            if (!ok) {
-                *abort_flag = 1;
-                __threadfence_block();
-            }
-            ptx::umma_commit(acc_bar);
-            ptx::mbar_wait_bounded(acc_bar, 0, kWaitLimitNs, p.err_flag, nullptr);
+            for (int b = 0; b < 2; ++b)
+                ptx::tma_load_2d_warp(base + kABytes + b * (kKStep * 128), &tB, &full[s], n0 + b * 64, k0, pol_b);
+            issued = kt;
         }
+        if (!ok)
+            for (int kt = issued - kStages + 1 > 0 ? issued - kStages + 1 : 0; kt <= issued; ++kt)
+                ptx::mbar_wait_bounded(&full[kt % kStages], (kt / kStages) & 1, kWaitLimitNs, nullptr, nullptr);
+    } else if (warp == 1) {
+        constexpr uint32_t idesc = ptx::make_idesc_bf16(kTile, kTile, false, true);
+        const uint32_t sbase = ptx::smem_u32(smem);
+        bool ok = true;
+        for (int kt = 0; kt < n_k && ok; ++kt) {
+            const int s = kt % kStages;
+            ok = __all_sync(0xffffffffu,
+                            ptx::mbar_wait_bounded(&full[s], (kt / kStages) & 1, kWaitLimitNs, p.err_flag, abort_flag));
+            if (!ok) break;
+            ptx::tc_fence_after();
+            const uint32_t a = sbase + s * kStageBytes, b = a + kABytes;
+#pragma unroll
+            for (int kk = 0; kk < kKStep / 16; ++kk) {
+                const uint64_t da = ptx::make_sdesc_sw128(a + kk * 32, 16, 1024);
+                const uint64_t db = ptx::make_sdesc_sw128(b + kk * 2048, kKStep * 128, 1024);
+                ptx::umma_f16_ss_warp(tmem, da, db, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+            }
+            ptx::umma_commit_warp(&empty[s]);
+        }
+        if (!ok) {
+            if (lane == 0) *abort_flag = 1;
+            __threadfence_block();
+        }
+        ptx::umma_commit_warp(acc_bar);
+        ptx::mbar_wait_bounded(acc_bar, 0, kWaitLimitNs, p.err_flag, nullptr);
     } else if (warp >= 4) {
         const int wq = warp - 4;
         const int r = wq * 32 + lane;

@@ -40,16 +40,6 @@ __host__ __device__ constexpr uint32_t make_idesc_tf32(int M, int N, bool b_mn) 
            | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-__device__ __forceinline__ void umma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 struct Tf32Params {
     float *C;
     int M, N, K;
@@ -95,61 +85,60 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    // producer and MMA warps stay converged; one elected lane issues (uniform registers)
     if (warp == 0) {
-        if (lane == 0) {
-            const uint64_t pol = ptx::policy_evict_normal();
-            int issued = -1;
-            bool ok = true;
-            for (int kt = 0; kt < n_k; ++kt) {
-                const int s = kt % kStages;
-                ok = ptx::mbar_wait_bounded(&empty[s], ((kt / kStages) & 1) ^ 1, kWaitLimitNs, p.err_flag, abort_flag);
-                if (!ok) break;
-                uint8_t *base = smem + s * kStageBytes;
-                ptx::mbar_arrive_expect_tx(&full[s], stage_tx);
-                const int k0 = kt * kKStep;
-                ptx::tma_load_3d(base, &tAh, &full[s], k0, m0, z, pol);
-                ptx::tma_load_3d(base + kOpBytes, &tAl, &full[s], k0, m0, z, pol);
-                ptx::tma_load_3d(base + 2 * kOpBytes, &tBh, &full[s], k0, n0, z, pol);
-                if (p.three_terms) ptx::tma_load_3d(base + 3 * kOpBytes, &tBl, &full[s], k0, n0, z, pol);
-                issued = kt;
-            }
-            if (!ok)
-                for (int kt = issued - kStages + 1 > 0 ? issued - kStages + 1 : 0; kt <= issued; ++kt)
-                    ptx::mbar_wait_bounded(&full[kt % kStages], (kt / kStages) & 1, kWaitLimitNs, nullptr, nullptr);
+        const uint64_t pol = ptx::policy_evict_normal();
+        int issued = -1;
+        bool ok = true;
+        for (int kt = 0; kt < n_k; ++kt) {
+            const int s = kt % kStages;
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&empty[s], ((kt / kStages) & 1) ^ 1, kWaitLimitNs,
+                                                                 p.err_flag, abort_flag));
+            if (!ok) break;
+            uint8_t *base = smem + s * kStageBytes;
+            ptx::mbar_arrive_expect_tx_warp(&full[s], stage_tx);
+            const int k0 = kt * kKStep;
+            ptx::tma_load_3d_warp(base, &tAh, &full[s], k0, m0, z, pol);
+            ptx::tma_load_3d_warp(base + kOpBytes, &tAl, &full[s], k0, m0, z, pol);
+            ptx::tma_load_3d_warp(base + 2 * kOpBytes, &tBh, &full[s], k0, n0, z, pol);
+            if (p.three_terms) ptx::tma_load_3d_warp(base + 3 * kOpBytes, &tBl, &full[s], k0, n0, z, pol);
+            issued = kt;
         }
+        if (!ok)
+            for (int kt = issued - kStages + 1 > 0 ? issued - kStages + 1 : 0; kt <= issued; ++kt)
+                ptx::mbar_wait_bounded(&full[kt % kStages], (kt / kStages) & 1, kWaitLimitNs, nullptr, nullptr);
     } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc = make_idesc_tf32(kTile, kTile, false);
-            const uint32_t sbase = ptx::smem_u32(smem);
-            bool ok = true;
-            for (int kt = 0; kt < n_k && ok; ++kt) {
-                const int s = kt % kStages;
-                ok = ptx::mbar_wait_bounded(&full[s], (kt / kStages) & 1, kWaitLimitNs, p.err_flag, abort_flag);
-                if (!ok) break;
-                ptx::tc_fence_after();
-                const uint32_t ah = sbase + s * kStageBytes, al = ah + kOpBytes, bh = al + kOpBytes, bl = bh + kOpBytes;
+        constexpr uint32_t idesc = make_idesc_tf32(kTile, kTile, false);
+        const uint32_t sbase = ptx::smem_u32(smem);
+        bool ok = true;
+        for (int kt = 0; kt < n_k && ok; ++kt) {
+            const int s = kt % kStages;
+            ok = __all_sync(0xffffffffu,
+                            ptx::mbar_wait_bounded(&full[s], (kt / kStages) & 1, kWaitLimitNs, p.err_flag, abort_flag));
+            if (!ok) break;
+            ptx::tc_fence_after();
+            const uint32_t ah = sbase + s * kStageBytes, al = ah + kOpBytes, bh = al + kOpBytes, bl = bh + kOpBytes;
 #pragma unroll
-                for (int kk = 0; kk < kKStep / 8; ++kk) {
-                    const uint64_t dah = ptx::make_sdesc_sw128(ah + kk * 32, 16, 1024);
-                    const uint64_t dal = ptx::make_sdesc_sw128(al + kk * 32, 16, 1024);
-                    const uint64_t dbh = ptx::make_sdesc_sw128(bh + kk * 32, 16, 1024);
-                    const uint32_t first = (kt == 0 && kk == 0) ? 0u : 1u;
-                    umma_tf32_ss(tmem, dal, dbh, idesc, first);
-                    if (p.three_terms) {
-                        const uint64_t dbl = ptx::make_sdesc_sw128(bl + kk * 32, 16, 1024);
-                        umma_tf32_ss(tmem, dah, dbl, idesc, 1u);
-                    }
-                    umma_tf32_ss(tmem, dah, dbh, idesc, 1u);
+            for (int kk = 0; kk < kKStep / 8; ++kk) {
+                const uint64_t dah = ptx::make_sdesc_sw128(ah + kk * 32, 16, 1024);
+                const uint64_t dal = ptx::make_sdesc_sw128(al + kk * 32, 16, 1024);
+                const uint64_t dbh = ptx::make_sdesc_sw128(bh + kk * 32, 16, 1024);
+                const uint32_t first = (kt == 0 && kk == 0) ? 0u : 1u;
+                ptx::umma_tf32_ss_warp(tmem, dal, dbh, idesc, first);
+                if (p.three_terms) {
+                    const uint64_t dbl = ptx::make_sdesc_sw128(bl + kk * 32, 16, 1024);
+                    ptx::umma_tf32_ss_warp(tmem, dah, dbl, idesc, 1u);
                 }
-                ptx::umma_commit(&empty[s]);
+                ptx::umma_tf32_ss_warp(tmem, dah, dbh, idesc, 1u);
             }
-            if (!ok) {
-                *abort_flag = 1;
-                __threadfence_block();
-            }
-            ptx::umma_commit(acc_bar);
-            ptx::mbar_wait_bounded(acc_bar, 0, kWaitLimitNs, p.err_flag, nullptr);
+            ptx::umma_commit_warp(&empty[s]);
         }
+        if (!ok) {
+            if (lane == 0) *abort_flag = 1;
+            __threadfence_block();
+        }
+        ptx::umma_commit_warp(acc_bar);
+        ptx::mbar_wait_bounded(acc_bar, 0, kWaitLimitNs, p.err_flag, nullptr);
     } else if (warp >= 4) {
         const int wq = warp - 4;
         const int r = wq * 32 + lane;

@@ -88,59 +88,60 @@ stats_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    // producer and MMA warps stay converged; one elected lane issues (uniform registers)
     if (warp == 0) {
         if (lane == 0) {
             ptx::tma_prefetch_desc(mapA);
             ptx::tma_prefetch_desc(mapB);
-            const uint64_t pol = ptx::policy_evict_last();
-            int issued = -1;
-            bool ok = true;
-            for (int kt = 0; kt < n_k && ok; ++kt) {
-                const int s = kt % kStages;
-                const uint32_t ph = (kt / kStages) & 1;
-                ok = ptx::mbar_wait_bounded(&empty[s], ph ^ 1, kWaitLimitNs, p.err_flag, abort_flag);
-                if (!ok) break;
-                uint8_t *base = smem + s * kStageBytes;
-                ptx::mbar_arrive_expect_tx(&full[s], kStageBytes);
-                for (int b = 0; b < 2; ++b) {
-                    ptx::tma_load_2d(base + b * (kKRows * 128), mapA, &full[s], bi * kTile + b * 64, kt * kKRows, pol);
-                    ptx::tma_load_2d(base + kOperandBytes + b * (kKRows * 128), mapB, &full[s], bj * kTile + b * 64,
-                                     kt * kKRows, pol);
-                }
-                issued = kt;
+        }
+        const uint64_t pol = ptx::policy_evict_last();
+        int issued = -1;
+        bool ok = true;
+        for (int kt = 0; kt < n_k && ok; ++kt) {
+            const int s = kt % kStages;
+            const uint32_t ph = (kt / kStages) & 1;
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&empty[s], ph ^ 1, kWaitLimitNs, p.err_flag, abort_flag));
+            if (!ok) break;
+            uint8_t *base = smem + s * kStageBytes;
+            ptx::mbar_arrive_expect_tx_warp(&full[s], kStageBytes);
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                ptx::tma_load_2d_warp(base + b * (kKRows * 128), mapA, &full[s], bi * kTile + b * 64, kt * kKRows, pol);
+                ptx::tma_load_2d_warp(base + kOperandBytes + b * (kKRows * 128), mapB, &full[s], bj * kTile + b * 64,
+                                      kt * kKRows, pol);
             }
-            if (!ok) {
-                for (int kt = (issued - kStages + 1 > 0 ? issued - kStages + 1 : 0); kt <= issued; ++kt)
-                    ptx::mbar_wait_bounded(&full[kt % kStages], (kt / kStages) & 1, kWaitLimitNs, nullptr, nullptr);
-            }
+            issued = kt;
+        }
+        if (!ok) {
+            for (int kt = (issued - kStages + 1 > 0 ? issued - kStages + 1 : 0); kt <= issued; ++kt)
+                ptx::mbar_wait_bounded(&full[kt % kStages], (kt / kStages) & 1, kWaitLimitNs, nullptr, nullptr);
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc = ptx::make_idesc_bf16(kTile, kTile, true, true);
-            const uint32_t sbase = ptx::smem_u32(smem);
-            bool ok = true;
-            for (int kt = 0; kt < n_k && ok; ++kt) {
-                const int s = kt % kStages;
-                ok = ptx::mbar_wait_bounded(&full[s], (kt / kStages) & 1, kWaitLimitNs, p.err_flag, abort_flag);
-                if (!ok) break;
-                ptx::tc_fence_after();
-                const uint32_t a0 = sbase + s * kStageBytes;
-                const uint32_t b0 = a0 + kOperandBytes;
+        constexpr uint32_t idesc = ptx::make_idesc_bf16(kTile, kTile, true, true);
+        const uint32_t sbase = ptx::smem_u32(smem);
+        bool ok = true;
+        for (int kt = 0; kt < n_k && ok; ++kt) {
+            const int s = kt % kStages;
+            ok = __all_sync(0xffffffffu,
+                            ptx::mbar_wait_bounded(&full[s], (kt / kStages) & 1, kWaitLimitNs, p.err_flag, abort_flag));
+            if (!ok) break;
+            ptx::tc_fence_after();
+            const uint32_t a0 = sbase + s * kStageBytes;
+            const uint32_t b0 = a0 + kOperandBytes;
 #pragma unroll
-                for (int kk = 0; kk < kKRows / 16; ++kk) {
-                    const uint64_t da = ptx::make_sdesc_sw128(a0 + kk * 2048, kKRows * 128, 1024);
-                    const uint64_t db = ptx::make_sdesc_sw128(b0 + kk * 2048, kKRows * 128, 1024);
-                    ptx::umma_f16_ss(tmem, da, db, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
-                }
-                ptx::umma_commit(&empty[s]);
+            for (int kk = 0; kk < kKRows / 16; ++kk) {
+                const uint64_t da = ptx::make_sdesc_sw128(a0 + kk * 2048, kKRows * 128, 1024);
+                const uint64_t db = ptx::make_sdesc_sw128(b0 + kk * 2048, kKRows * 128, 1024);
+                ptx::umma_f16_ss_warp(tmem, da, db, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
             }
-            if (!ok) {
-                *abort_flag = 1;
-                __threadfence_block();
-            }
-            ptx::umma_commit(acc_bar);
-            ptx::mbar_wait_bounded(acc_bar, 0, kWaitLimitNs, p.err_flag, nullptr);
+            ptx::umma_commit_warp(&empty[s]);
         }
+        if (!ok) {
+            if (lane == 0) *abort_flag = 1;
+            __threadfence_block();
+        }
+        ptx::umma_commit_warp(acc_bar);
+        ptx::mbar_wait_bounded(acc_bar, 0, kWaitLimitNs, p.err_flag, nullptr);
     } else if (warp >= 4) {
         const int wq = warp - 4;
         const int r = wq * 32 + lane;                   // row inside the tile
