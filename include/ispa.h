@@ -147,6 +147,24 @@ int ispa_solve_absorb(const ispa_stats *per_layer, int n_layers, const void *con
                       void *const *w_new, int *layer_status, void *ws, size_t ws_bytes,
                       ispa_stream_t stream);
 
+/* ispa_absorb_error -- the reconstruction error eps[l] of a GIVEN dW[l] on GIVEN statistics:
+ * eps = E^2 / T^2 with E^2 = tr(dW^T G dW) - 2 tr(dW^T C W) + tr(W^T H W) and
+ * T^2 = tr(W^T (G + C + C^T + H) W) [ISPA §3.3, the error the selection ranks; the same
+ * formula ispa_solve_absorb evaluates after solving]. Without a solve it serves the
+ * re-warmup trigger [ISPA §3.1 last paragraph, §3.3 last paragraph, which leave the
+ * trigger open]: on the statistics of one chunk after the transition, eps of the dW solved
+ * at the transition measures how well the absorbed projection still reconstructs the full
+ * output of an F-layer.
+ *   per_layer: n_layers statistics (device, as for ispa_solve_absorb); w_o, w_dtype: the
+ *   original projections [D_in, D_out]; dW: n_layers device pointers to float32 [D][D]
+ *   (16-byte aligned); eps: device float [n_layers]; err_terms: device double
+ *   [n_layers][2] = (E^2, T^2), optional. eps = 0 when T^2 = 0.
+ *   ws: ispa_workspace_bytes(NULL, n_layers, D) bytes (the solve's workspace suffices).
+ * D must be a multiple of 64; the statistics are read only. */
+int ispa_absorb_error(const ispa_stats *per_layer, int n_layers, const void *const *w_o,
+                      ispa_dtype w_dtype, const float *const *dW, float *eps, double *err_terms,
+                      void *ws, size_t ws_bytes, ispa_stream_t stream);
+
 /* ispa_select_layers -- Dynamic Layer Selection [ISPA §3.3], host only: rank layers by
  * eps ascending (ties: lower layer index first; NaN last) and take the first K.
  *   eps_host [n_layers] (host), idx_out [min(K, n_layers)] (host, rank order),

@@ -18,4 +18,6 @@ from .ispa_oracle import (  # noqa: F401
     select_layers,
     project,
     run_episode,
+    live_error,
+    rewarm_trigger,
 )

@@ -35,6 +35,16 @@ What is computed (per layer, per warmup chunk, then once at the transition):
    NaN ranks last); the first K become L-layers with W_new = W + dW [ISPA §3.1 step 3].
 6. After the switch an L-layer attends to the sink + chunk rows only and projects with
    W_new [ISPA §3.1 step 3, §3.3].
+7. Re-warmup trigger [ISPA §3.1 last paragraph, §3.3 last paragraph: the warmup is entered
+   again when the scene changes; no trigger is given]. Reading: after a transition each
+   F-layer still sees its history, so the statistics of one live chunk (step 2 on that chunk
+   alone) and the dW solved at the transition give a live error eps_live (step 4 on those
+   statistics). The warmup is re-entered when a monitored layer's eps_live exceeds both 4 x
+   and 0.02 + the lowest eps_live that layer showed since the transition. The reference is
+   that live minimum, not the eps of the selection: eps at the selection is an in-sample
+   figure, and where the residual is not predictable from A_loc (i.i.d. layers) dW overfits
+   the warmup, so a fresh chunk's error is far above it without any change of scene. L-layers
+   cannot be monitored: their history is gone.
 """
 from __future__ import annotations
 
@@ -203,8 +213,27 @@ def project(A: np.ndarray, W: np.ndarray) -> np.ndarray:
 # --------------------------------------------------------------------------------------
 # A whole streaming run, chunk by chunk [ISPA §3.1, §3.3 re-triggered warmup].
 # --------------------------------------------------------------------------------------
+def live_error(A_loc, A_full, dtype: str, W, dW) -> float:
+    """Step 7: eps of a given dW on the statistics of one chunk."""
+    st = stats_init(np.asarray(W).shape[0])
+    stats_update(st, A_loc, A_full, dtype)
+    return reconstruction_error(st["G"], st["C"], st["H"], W, dW)["eps"]
+
+
+def rewarm_trigger(previous: Sequence[Dict[int, float]], eps_live: Dict[int, float], ratio: float = 4.0,
+                   min_rise: float = 0.02) -> List[int]:
+    """Step 7's rule: the monitored layers whose live error rose above the lowest live error
+    they showed on the earlier chunks since the transition (`previous`, oldest first)."""
+    fired = []
+    for l, e in eps_live.items():
+        seen = [p[l] for p in previous if l in p]
+        if seen and e > ratio * min(seen) and e > min(seen) + min_rise:
+            fired.append(l)
+    return sorted(fired)
+
+
 def run_episode(cfg, n_chunks: Optional[int] = None, K: Optional[int] = None,
-                keep_outputs: bool = False) -> Dict[str, object]:
+                keep_outputs: bool = False, rewarm_at="cut", monitor: bool = False) -> Dict[str, object]:
     """Warmup -> transition -> L/F inference (-> re-warmup at a scene cut) for a workload
     from `synth`. Reading of the schedule: the warmup covers cfg.warmup_chunks chunks; at
     a scene cut every layer restores its original W, its statistics restart from zero and
@@ -214,6 +243,11 @@ def run_episode(cfg, n_chunks: Optional[int] = None, K: Optional[int] = None,
     Returns per-transition eps/dW/selection and, if asked, per-chunk per-layer outputs: the
     attention output O (A_full for an F-layer, A_loc for an L-layer), y = O W_cur and
     whether the layer ran local.
+
+    rewarm_at: the chunk where the warmup is re-entered -- "cut" (the workload's scene cut,
+    the default), None (never), or a chunk index. The scene itself always changes at the
+    workload's cut. monitor=True adds step 7: for every chunk after a transition, the live
+    error of each F-layer (key "live": list of (chunk, {layer: eps_live})).
     """
     import synth  # seeded inputs only
 
@@ -228,8 +262,10 @@ def run_episode(cfg, n_chunks: Optional[int] = None, K: Optional[int] = None,
     warm_start = 0
     transitions = []
     outputs = []
+    live = []
+    rewarm_chunk = cfg.cut_chunk if rewarm_at == "cut" else rewarm_at
     for t in range(n_chunks):
-        if cfg.cut_chunk is not None and t == cfg.cut_chunk:
+        if rewarm_chunk is not None and t == rewarm_chunk:
             for l in range(L):
                 if is_local[l]:
                     hist_from[l] = cfg.chunk_start_frame(t)
@@ -238,6 +274,8 @@ def run_episode(cfg, n_chunks: Optional[int] = None, K: Optional[int] = None,
                 stats[l] = stats_init(cfg.D)
             warm_start = t
         in_warmup = warm_start <= t < warm_start + cfg.warmup_chunks
+        watch = monitor and transitions and not in_warmup
+        chunk_live = {}
         chunk_out = []
         for l in range(L):
             q = synth.chunk_q(cfg, l, t)
@@ -257,10 +295,15 @@ def run_episode(cfg, n_chunks: Optional[int] = None, K: Optional[int] = None,
                 O = res["A_full"]
                 if in_warmup:
                     stats_update(stats[l], res["A_loc"], res["A_full"], cfg.dtype)
+                elif watch:
+                    chunk_live[l] = live_error(res["A_loc"], res["A_full"], cfg.dtype, W0[l],
+                                               transitions[-1]["dW"][l])
             if keep_outputs:
                 chunk_out.append(dict(O=O, y=project(O, W_cur[l]), local=bool(is_local[l])))
         if keep_outputs:
             outputs.append(chunk_out)
+        if watch:
+            live.append((t, chunk_live))
         if in_warmup and t == warm_start + cfg.warmup_chunks - 1:
             dWs, errs = [], []
             for l in range(L):
@@ -276,4 +319,4 @@ def run_episode(cfg, n_chunks: Optional[int] = None, K: Optional[int] = None,
             transitions.append(dict(chunk=t, eps=eps, errs=errs, dW=dWs, idx=idx, is_local=list(flags),
                                     stats=[dict(G=s["G"].copy(), C=s["C"].copy(), H=s["H"].copy(),
                                                 rows=s["rows"]) for s in stats]))
-    return dict(transitions=transitions, outputs=outputs)
+    return dict(transitions=transitions, outputs=outputs, live=live)

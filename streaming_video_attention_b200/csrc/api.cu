@@ -13,6 +13,10 @@
 #include "ptx.cuh"
 
 namespace ispa {
+cudaError_t error_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H, const PtrBatch &W, ElemType wt,
+                        const PtrBatch &dW, const PtrBatch &Y, const PtrBatch &P, float *Yc, float *Pc, float *split,
+                        double *terms, int nparts, float *eps, double *err_terms, int D, int batch, int *err_flag,
+                        cudaStream_t s);
 cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H, const PtrBatch &W, ElemType wt,
                         const PtrBatch &dW, const PtrBatch &M, const PtrBatch &Y, const PtrBatch &P, float *Yc,
                         float *Pc, float *split, double *terms, int nparts, int *status, float *eps,
@@ -417,6 +421,56 @@ int ispa_solve_absorb(const ispa_stats *per_layer, int n_layers, const void *con
                                     err_terms ? err_terms + 2 * (size_t)l0 : nullptr, w_new ? &WN : nullptr, D, lambda,
                                     b, flag, s);
         if (e != cudaSuccess) return cuda_fail(e, "absorb solve");
+    }
+    return ISPA_OK;
+}
+
+int ispa_absorb_error(const ispa_stats *per_layer, int n_layers, const void *const *w_o, ispa_dtype w_dtype,
+                      const float *const *dW, float *eps, double *err_terms, void *ws, size_t ws_bytes,
+                      ispa_stream_t stream) {
+    g_last_error.clear();
+    if (n_layers < 0) return fail(ISPA_ERR_INVALID_ARG, "n_layers < 0");
+    if (n_layers == 0) return ISPA_OK;
+    if (!per_layer || !w_o || !dW || !eps) return fail(ISPA_ERR_INVALID_ARG, "per_layer, w_o, dW and eps are required");
+    if (w_dtype != ISPA_BF16 && w_dtype != ISPA_FP32) return fail(ISPA_ERR_INVALID_ARG, "bad w_dtype");
+    const int D = per_layer[0].D;
+    if (D <= 0 || D % 64 != 0) return fail(ISPA_ERR_UNSUPPORTED, "D=%d: needs D %% 64 == 0", D);
+    for (int l = 0; l < n_layers; ++l) {
+        int rc = check_stats(&per_layer[l], D);
+        if (rc != ISPA_OK) return fail(rc, "layer %d: %s", l, g_last_error.c_str());
+        if (!w_o[l]) return fail(ISPA_ERR_INVALID_ARG, "w_o[%d] is NULL", l);
+        if (!dW[l]) return fail(ISPA_ERR_INVALID_ARG, "dW[%d] is NULL", l);
+        if (!aligned(dW[l], 16)) return fail(ISPA_ERR_INVALID_ARG, "dW[%d] must be 16-byte aligned", l);
+    }
+    int rc = check_ws(ws, ws_bytes, solve_ws_bytes(n_layers, D));
+    if (rc != ISPA_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // workspace layout as for the solve (the M block is unused here)
+    const size_t mat = (size_t)D * D * sizeof(float);
+    const int bmax = std::min(n_layers, kMaxBatch);
+    char *wsb = static_cast<char *>(ws);
+    char *Yb = wsb + (size_t)bmax * mat, *Pb = wsb + 2 * (size_t)bmax * mat;
+    float *split = reinterpret_cast<float *>(wsb + 3 * (size_t)bmax * mat);
+    double *terms = reinterpret_cast<double *>(wsb + 9 * (size_t)bmax * mat);
+    int *flag = nullptr;
+    rc = device_error_flag(&flag);
+    if (rc != ISPA_OK) return rc;
+    for (int l0 = 0; l0 < n_layers; l0 += kMaxBatch) {
+        const int b = std::min(kMaxBatch, n_layers - l0);
+        PtrBatch G, C, H, W, DW, Y, P;
+        for (int z = 0; z < b; ++z) {
+            const ispa_stats &st = per_layer[l0 + z];
+            G.p[z] = st.G; C.p[z] = st.C; H.p[z] = st.H;
+            W.p[z] = const_cast<void *>(w_o[l0 + z]);
+            DW.p[z] = const_cast<float *>(dW[l0 + z]);
+            Y.p[z] = Yb + (size_t)z * mat;
+            P.p[z] = Pb + (size_t)z * mat;
+        }
+        cudaError_t e = error_batch(G, C, H, W, w_dtype == ISPA_BF16 ? ElemType::BF16 : ElemType::F32, DW, Y, P,
+                                    reinterpret_cast<float *>(Yb), reinterpret_cast<float *>(Pb), split, terms,
+                                    kEpsParts, eps + l0, err_terms ? err_terms + 2 * (size_t)l0 : nullptr, D, b, flag,
+                                    s);
+        if (e != cudaSuccess) return cuda_fail(e, "absorb error");
     }
     return ISPA_OK;
 }

@@ -168,7 +168,7 @@ __global__ void finalize_eps_kernel(const double *terms, int nparts, int batch, 
     const double E2 = t[0] - 2.0 * t[1] + t[2];
     const double T2 = t[3] + 2.0 * t[4] + t[2];
     float e = T2 == 0.0 ? 0.f : (float)(E2 / T2);
-    if (status[z] != ISPA_OK) e = __int_as_float(0x7fc00000);
+    if (status && status[z] != ISPA_OK) e = __int_as_float(0x7fc00000);
     eps[z] = e;
     if (err_terms) {
         err_terms[2 * z] = E2;
@@ -215,6 +215,92 @@ static GemmBatch make_gemm_batch(const PtrBatch &A, size_t offA, const PtrBatch 
         if (e_ != cudaSuccess) return e_;    \
     } while (0)
 
+// The five traces of the error and eps = E^2 / T^2 for dW given, Y = C W already in Y
+// (and W already split when tc): t0 = tr(dW^T G dW), t1 = tr(dW^T Y), t2 = tr(W^T H W),
+// t3 = tr(W^T G W), t4 = tr(W^T Y).
+cudaError_t error_terms(const PtrBatch &G, const PtrBatch &H, const PtrBatch &W, ElemType wt, const PtrBatch &dW,
+                        const PtrBatch &Y, const PtrBatch &P, float *Pc, float *split, double *terms, int nparts,
+                        const int *status, float *eps, double *err_terms, int D, int batch, int *err_flag, bool tc,
+                        cudaStream_t s) {
+    const size_t n = (size_t)D * D;
+    const size_t ew = wt == ElemType::BF16 ? 2 : 4;
+    const size_t bn = (size_t)batch * n;
+    float *Ahi = split, *Alo = split + bn, *Bhi = split + 2 * bn, *Blo = split + 3 * bn;
+    float *Whi = split + 4 * bn, *Wlo = wt == ElemType::BF16 ? nullptr : split + 5 * bn;
+    const dim3 rgrid(nparts, batch);
+    GemmDesc full{D, D, D, D, D, D, true, false, ElemType::F32, ElemType::F32, ElemType::F32, 1.f, 0.f, false, batch};
+    // t0 = tr(dW^T G dW)
+    if (tc) {
+        ISPA_TRY(launch_split_tf32(G, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
+        ISPA_TRY(launch_split_tf32(dW, ElemType::F32, Bhi, Blo, D, D, true, batch, s));
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Bhi, Blo, Pc, D, D, D, batch, err_flag, s));
+    } else {
+        ISPA_TRY(launch_gemm_simt(full, make_gemm_batch(G, 0, dW, 0, P, 0, batch, 4, 4), s));
+    }
+    dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, P, n, terms + 0 * (size_t)batch * nparts); note_launch();
+    // t1 = tr(dW^T C W)
+    dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, Y, n, terms + 1 * (size_t)batch * nparts); note_launch();
+    // t3 = tr(W^T G W) first while G's split is in place, then t2 = tr(W^T H W); t4 = tr(W^T C W)
+    GemmDesc fw = full;
+    fw.b_type = wt;
+    if (tc) {
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Pc, D, D, D, batch, err_flag, s));
+    } else {
+        ISPA_TRY(launch_gemm_simt(fw, make_gemm_batch(G, 0, W, 0, P, 0, batch, 4, ew), s));
+    }
+    if (wt == ElemType::BF16) { dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, P, n, terms + 3 * (size_t)batch * nparts); note_launch(); }
+    else { dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, P, n, terms + 3 * (size_t)batch * nparts); note_launch(); }
+    if (tc) {
+        ISPA_TRY(launch_split_tf32(H, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Pc, D, D, D, batch, err_flag, s));
+    } else {
+        ISPA_TRY(launch_gemm_simt(fw, make_gemm_batch(H, 0, W, 0, P, 0, batch, 4, ew), s));
+    }
+    if (wt == ElemType::BF16) { dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, P, n, terms + 2 * (size_t)batch * nparts); note_launch(); }
+    else { dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, P, n, terms + 2 * (size_t)batch * nparts); note_launch(); }
+    if (wt == ElemType::BF16) {
+        dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, Y, n, terms + 4 * (size_t)batch * nparts); note_launch();
+    } else {
+        dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, Y, n, terms + 4 * (size_t)batch * nparts); note_launch();
+    }
+    ISPA_TRY(cudaGetLastError());
+    finalize_eps_kernel<<<(batch + 63) / 64, 64, 0, s>>>(terms, nparts, batch, status, eps, err_terms); note_launch();
+    ISPA_TRY(cudaGetLastError());
+
+    return cudaSuccess;
+}
+
+// Y = C W for one batch of layers (W split into Whi/Wlo first when tc).
+static cudaError_t c_times_w(const PtrBatch &C, const PtrBatch &W, ElemType wt, const PtrBatch &Y, float *Yc,
+                             float *split, int D, int batch, int *err_flag, bool tc, cudaStream_t s) {
+    const size_t n = (size_t)D * D;
+    const size_t ew = wt == ElemType::BF16 ? 2 : 4;
+    const size_t bn = (size_t)batch * n;
+    float *Ahi = split, *Alo = split + bn;
+    float *Whi = split + 4 * bn, *Wlo = wt == ElemType::BF16 ? nullptr : split + 5 * bn;
+    if (tc) {
+        ISPA_TRY(launch_split_tf32(W, wt, Whi, Wlo, D, D, true, batch, s));
+        ISPA_TRY(launch_split_tf32(C, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Yc, D, D, D, batch, err_flag, s));
+    } else {
+        GemmDesc d{D, D, D, D, D, D, true, false, ElemType::F32, wt, ElemType::F32, 1.f, 0.f, false, batch};
+        ISPA_TRY(launch_gemm_simt(d, make_gemm_batch(C, 0, W, 0, Y, 0, batch, 4, ew), s));
+    }
+    return cudaSuccess;
+}
+
+// The error of a given dW on given statistics (no solve): Y = C W, then the five traces.
+// Scratch as for solve_batch (Y, P, the split blocks, terms).
+cudaError_t error_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H, const PtrBatch &W, ElemType wt,
+                        const PtrBatch &dW, const PtrBatch &Y, const PtrBatch &P, float *Yc, float *Pc, float *split,
+                        double *terms, int nparts, float *eps, double *err_terms, int D, int batch, int *err_flag,
+                        cudaStream_t s) {
+    const bool tc = (D % 128 == 0) && split != nullptr;
+    ISPA_TRY(c_times_w(C, W, wt, Y, Yc, split, D, batch, err_flag, tc, s));
+    return error_terms(G, H, W, wt, dW, Y, P, Pc, split, terms, nparts, nullptr, eps, err_terms, D, batch, err_flag,
+                       tc, s);
+}
+
 // Solve for one batch of layers. All pointers are device pointers, one per layer.
 //   G, C, H: statistics; W: weights of type wt; dW: output; M, Y: D*D float scratch each;
 //   P: D*D float scratch; terms: 5 * batch * nparts doubles; status: batch ints (zeroed).
@@ -224,28 +310,17 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
                         double *err_terms, const PtrBatch *w_new, int D, float lambda, int batch, int *err_flag,
                         cudaStream_t s) {
     const size_t n = (size_t)D * D;
-    const size_t ew = wt == ElemType::BF16 ? 2 : 4;
     const int fill_blocks = (int)std::min<size_t>((n + 255) / 256, 1024);
     // D x D products on the tensor cores (3xTF32) when D is a multiple of 128; the split
     // operands live in `split`: A_hi, A_lo, B_hi, B_lo, W_hi, W_lo, each [batch][D][D].
     const bool tc = (D % 128 == 0) && split != nullptr;
-    const size_t bn = (size_t)batch * n;
-    float *Ahi = split, *Alo = split + bn, *Bhi = split + 2 * bn, *Blo = split + 3 * bn;
-    float *Whi = split + 4 * bn, *Wlo = wt == ElemType::BF16 ? nullptr : split + 5 * bn;
-    if (tc) ISPA_TRY(launch_split_tf32(W, wt, Whi, Wlo, D, D, true, batch, s));
 
     // M = G + lambda I
     fill_shifted_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(G, M, D, lambda); note_launch();
     ISPA_TRY(cudaGetLastError());
 
     // Y = C W, and dW <- Y (solved in place below)
-    if (tc) {
-        ISPA_TRY(launch_split_tf32(C, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
-        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Yc, D, D, D, batch, err_flag, s));
-    } else {
-        GemmDesc d{D, D, D, D, D, D, true, false, ElemType::F32, wt, ElemType::F32, 1.f, 0.f, false, batch};
-        ISPA_TRY(launch_gemm_simt(d, make_gemm_batch(C, 0, W, 0, Y, 0, batch, 4, ew), s));
-    }
+    ISPA_TRY(c_times_w(C, W, wt, Y, Yc, split, D, batch, err_flag, tc, s));
     copy_f32_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(Y, dW, n); note_launch();
     ISPA_TRY(cudaGetLastError());
 
@@ -293,45 +368,8 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
     }
 
     // Reconstruction error terms
-    const dim3 rgrid(nparts, batch);
-    GemmDesc full{D, D, D, D, D, D, true, false, ElemType::F32, ElemType::F32, ElemType::F32, 1.f, 0.f, false, batch};
-    // t0 = tr(dW^T G dW)
-    if (tc) {
-        ISPA_TRY(launch_split_tf32(G, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
-        ISPA_TRY(launch_split_tf32(dW, ElemType::F32, Bhi, Blo, D, D, true, batch, s));
-        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Bhi, Blo, Pc, D, D, D, batch, err_flag, s));
-    } else {
-        ISPA_TRY(launch_gemm_simt(full, make_gemm_batch(G, 0, dW, 0, P, 0, batch, 4, 4), s));
-    }
-    dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, P, n, terms + 0 * (size_t)batch * nparts); note_launch();
-    // t1 = tr(dW^T C W)
-    dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, Y, n, terms + 1 * (size_t)batch * nparts); note_launch();
-    // t3 = tr(W^T G W) first while G's split is in place, then t2 = tr(W^T H W); t4 = tr(W^T C W)
-    GemmDesc fw = full;
-    fw.b_type = wt;
-    if (tc) {
-        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Pc, D, D, D, batch, err_flag, s));
-    } else {
-        ISPA_TRY(launch_gemm_simt(fw, make_gemm_batch(G, 0, W, 0, P, 0, batch, 4, ew), s));
-    }
-    if (wt == ElemType::BF16) { dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, P, n, terms + 3 * (size_t)batch * nparts); note_launch(); }
-    else { dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, P, n, terms + 3 * (size_t)batch * nparts); note_launch(); }
-    if (tc) {
-        ISPA_TRY(launch_split_tf32(H, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
-        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Pc, D, D, D, batch, err_flag, s));
-    } else {
-        ISPA_TRY(launch_gemm_simt(fw, make_gemm_batch(H, 0, W, 0, P, 0, batch, 4, ew), s));
-    }
-    if (wt == ElemType::BF16) { dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, P, n, terms + 2 * (size_t)batch * nparts); note_launch(); }
-    else { dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, P, n, terms + 2 * (size_t)batch * nparts); note_launch(); }
-    if (wt == ElemType::BF16) {
-        dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, Y, n, terms + 4 * (size_t)batch * nparts); note_launch();
-    } else {
-        dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, Y, n, terms + 4 * (size_t)batch * nparts); note_launch();
-    }
-    ISPA_TRY(cudaGetLastError());
-    finalize_eps_kernel<<<(batch + 63) / 64, 64, 0, s>>>(terms, nparts, batch, status, eps, err_terms); note_launch();
-    ISPA_TRY(cudaGetLastError());
+    ISPA_TRY(error_terms(G, H, W, wt, dW, Y, P, Pc, split, terms, nparts, status, eps, err_terms, D, batch, err_flag,
+                         tc, s));
 
     if (w_new) {
         if (wt == ElemType::BF16) { add_delta_kernel<bf16><<<dim3(fill_blocks, batch), 256, 0, s>>>(W, dW, *w_new, n); note_launch(); }

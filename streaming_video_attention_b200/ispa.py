@@ -28,7 +28,8 @@ ISPA_BF16 = 0
 ISPA_FP32 = 1
 
 EXPORTS = (
-    "ispa_attn_split", "ispa_attn_split_noalloc", "ispa_accum_stats", "ispa_stats_reset", "ispa_solve_absorb", "ispa_select_layers",
+    "ispa_attn_split", "ispa_attn_split_noalloc", "ispa_accum_stats", "ispa_stats_reset", "ispa_solve_absorb",
+    "ispa_absorb_error", "ispa_select_layers",
     "ispa_local_attn", "ispa_workspace_bytes", "ispa_device_status", "ispa_selftest_bounded_wait",
     "ispa_selftest_exp2_poly", "ispa_set_attn_kernel", "ispa_kernel_launches", "ispa_last_error", "ispa_version",
 )
@@ -180,6 +181,18 @@ def ispa_solve_absorb(stats: Sequence[Stats], w_o: Sequence[torch.Tensor], w_dty
                                  _p(layer_status), _p(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                                  _stream(stream))
     _check(rc, "ispa_solve_absorb")
+
+
+def ispa_absorb_error(stats: Sequence[Stats], w_o: Sequence[torch.Tensor], w_dtype: int,
+                      dW: Sequence[torch.Tensor], eps: torch.Tensor, err_terms: Optional[torch.Tensor] = None,
+                      ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    L = len(stats)
+    arr = (CStats * L)(*[s.c() for s in stats])
+    wp = (ctypes.c_void_p * L)(*[w.data_ptr() for w in w_o])
+    dp = (ctypes.c_void_p * L)(*[d.data_ptr() for d in dW])
+    rc = lib().ispa_absorb_error(arr, L, wp, w_dtype, dp, _p(eps), _p(err_terms), _p(ws),
+                                 0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "ispa_absorb_error")
 
 
 def ispa_select_layers(eps: Sequence[float], K: int):

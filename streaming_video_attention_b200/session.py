@@ -10,10 +10,19 @@ weights and zeroes the statistics; the next transition replaces the old dW.
 
 The session owns the statistics buffers, dW, the error vector and the updated weights; the
 caller owns the KV cache (evicting the history of an L-layer is the caller freeing it).
+
+Re-warmup trigger (the pages leave it open; reading): after a transition the F-layers still
+see their history, so full_attention(..., monitor=True) accumulates one chunk's statistics
+and live_errors() evaluates the error of the dW solved at the transition on them
+(ispa_absorb_error). rewarm_layers() names the monitored layers whose live error rose above
+both RATIO x and MIN_RISE + the lowest live error they showed since the transition -- a
+scene change that the absorbed projection no longer reconstructs. The reference is the live
+minimum rather than the selection's eps, which is in-sample: where the residual is not
+predictable (i.i.d. layers) dW overfits the warmup and every fresh chunk sits far above it.
 """
 from __future__ import annotations
 
-from typing import List, Optional, Sequence, Tuple
+from typing import Dict, List, Optional, Sequence, Tuple
 
 import torch
 
@@ -21,6 +30,9 @@ from . import ispa
 
 
 class IspaSession:
+    RATIO = 4.0        # live error above RATIO x its minimum since the transition ...
+    MIN_RISE = 0.02    # ... and above that minimum + MIN_RISE
+
     def __init__(self, layers: int, heads: int, head_dim: int, lam: float, K: int, dtype: str = "bf16",
                  device: str = "cuda"):
         self.layers, self.heads, self.head_dim = layers, heads, head_dim
@@ -43,6 +55,9 @@ class IspaSession:
         self.idx: List[int] = []
         self.eps_host: List[float] = []
         self.transitions = 0
+        self.monitor: List[Optional[ispa.Stats]] = [None] * layers
+        self.live_history: List[Dict[int, float]] = []
+        self._eps_live = torch.empty(layers, dtype=torch.float32, device=device)
 
     # ---------------------------------------------------------------- state
     def set_weights(self, W: Sequence[torch.Tensor]) -> None:
@@ -56,6 +71,13 @@ class IspaSession:
             ispa.ispa_stats_reset(st, stream)
         self.is_local = [0] * self.layers
         self.idx = []
+        self._reset_monitor(stream)
+
+    def _reset_monitor(self, stream=None) -> None:
+        for st in self.monitor:
+            if st is not None:
+                ispa.ispa_stats_reset(st, stream)
+        self.live_history = []
 
     def weight(self, layer: int) -> torch.Tensor:
         return self.W_new[layer] if self.is_local[layer] else self.W0[layer]
@@ -73,13 +95,21 @@ class IspaSession:
 
     # ---------------------------------------------------------------- per-layer calls
     def full_attention(self, layer: int, q, k, v, sink: Tuple[int, int], chunk: Tuple[int, int], o, lse,
-                       collect: bool, o_loc=None, lse_loc=None, o_hist=None, lse_hist=None, stream=None) -> None:
-        """An F-layer call; with collect=True (warmup) the ridge statistics accumulate too."""
+                       collect: bool, o_loc=None, lse_loc=None, o_hist=None, lse_hist=None, stream=None,
+                       monitor: bool = False) -> None:
+        """An F-layer call; with collect=True (warmup) the ridge statistics accumulate too; with
+        monitor=True (after a transition) this chunk's statistics go to the layer's monitor."""
         n_q, n_kv = q.shape[0], k.shape[0]
         desc = ispa.make_desc(n_q, n_kv, self.heads, self.head_dim, sink, chunk, dtype=self.code)
-        ws = self._attn_ws(desc) if collect else None
-        ispa.ispa_attn_split(desc, q, k, v, o, lse, o_loc, lse_loc, o_hist, lse_hist,
-                             stats=self.stats[layer] if collect else None, ws=ws, stream=stream)
+        st = None
+        if collect:
+            st = self.stats[layer]
+        elif monitor:
+            if self.monitor[layer] is None:
+                self.monitor[layer] = ispa.Stats(self.D, self.device)
+            st = self.monitor[layer]
+        ws = self._attn_ws(desc) if st is not None else None
+        ispa.ispa_attn_split(desc, q, k, v, o, lse, o_loc, lse_loc, o_hist, lse_hist, stats=st, ws=ws, stream=stream)
 
     def local_attention(self, layer: int, q, k_loc, v_loc, o, lse=None, y=None, stream=None) -> None:
         """An L-layer call: sink + chunk rows only; y = O W_new when y is given."""
@@ -101,10 +131,39 @@ class IspaSession:
         self.idx, flags = ispa.ispa_select_layers(eps, K)
         self.is_local = [int(f) for f in flags]
         self.transitions += 1
+        self._reset_monitor(stream)
         if any(s != ispa.ISPA_OK for s in status):
             bad = [l for l, s in enumerate(status) if s != ispa.ISPA_OK]
             raise ispa.IspaError(ispa.ISPA_ERR_NOT_SPD, "transition", f"G + lambda I not SPD in layers {bad}")
         return list(self.idx)
+
+    # ---------------------------------------------------------------- re-warmup trigger
+    def live_errors(self, stream=None) -> Dict[int, float]:
+        """Error of the transition's dW on the statistics each monitored F-layer gathered since
+        the last call; resets those statistics and records the result. Synchronises `stream`."""
+        layers = [l for l in range(self.layers) if self.monitor[l] is not None and not self.is_local[l]]
+        if not layers or self.transitions == 0:
+            return {}
+        ispa.ispa_absorb_error([self.monitor[l] for l in layers], [self.W0[l] for l in layers], self.code,
+                               [self.dW[l] for l in layers], self._eps_live, ws=self.ws_solve, stream=stream)
+        vals = self._eps_live[:len(layers)].to("cpu").tolist()
+        for l in layers:
+            ispa.ispa_stats_reset(self.monitor[l], stream)
+        live = dict(zip(layers, vals))
+        self.live_history.append(live)
+        return live
+
+    def rewarm_layers(self) -> List[int]:
+        """Monitored layers whose latest live error left the range seen since the transition."""
+        if len(self.live_history) < 2:
+            return []
+        latest, earlier = self.live_history[-1], self.live_history[:-1]
+        out = []
+        for l, e in latest.items():
+            ref = [d[l] for d in earlier if l in d]
+            if ref and e > self.RATIO * min(ref) and e > min(ref) + self.MIN_RISE:
+                out.append(l)
+        return sorted(out)
 
     def selection_margin(self) -> Optional[float]:
         """(eps_(K+1) - eps_(K)) / eps_(K) of the last transition: how decisive the cut was."""

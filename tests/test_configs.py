@@ -26,10 +26,17 @@ from tests.helpers import rel_fro, to_device, to_numpy, torch_dtype
 pytestmark = pytest.mark.gpu
 
 
-def gpu_episode(cfg, K=None, n_chunks=None, keep_layers=None):
+def gpu_episode(cfg, K=None, n_chunks=None, keep_layers=None, rewarm="cut", monitor=False):
     """Drive IspaSession through a streaming run laid out by `synth` (the caller owns the KV
-    cache: it builds each layer's cache from the frames that layer still holds)."""
+    cache: it builds each layer's cache from the frames that layer still holds).
+
+    rewarm: "cut" re-enters the warmup at the workload's scene cut, None never, "auto" at the
+    chunk after the session's trigger fired (monitoring every F-layer after a transition).
+    monitor: record the live errors (implied by "auto")."""
     K = cfg.K if K is None else K
+    monitor = monitor or rewarm == "auto"
+    live, fired = [], []
+    pending_rewarm = False
     n_chunks = cfg.n_chunks if n_chunks is None else n_chunks
     L = cfg.layers
     td = torch_dtype(cfg.dtype)
@@ -40,13 +47,16 @@ def gpu_episode(cfg, K=None, n_chunks=None, keep_layers=None):
     warm_start = 0
     transitions, outputs = [], []
     for t in range(n_chunks):
-        if cfg.cut_chunk is not None and t == cfg.cut_chunk:
+        scheduled = rewarm == "cut" and cfg.cut_chunk is not None and t == cfg.cut_chunk
+        if scheduled or pending_rewarm:
             for l in range(L):
                 if sess.is_local[l]:
                     hist_from[l] = cfg.chunk_start_frame(t)
             sess.rewarm()
             warm_start = t
+            pending_rewarm = False
         in_warmup = warm_start <= t < warm_start + cfg.warmup_chunks
+        watch = monitor and sess.transitions > 0 and not in_warmup
         chunk_out = []
         for l in range(L):
             q = to_device(synth.chunk_q(cfg, l, t), cfg.dtype)
@@ -66,16 +76,23 @@ def gpu_episode(cfg, K=None, n_chunks=None, keep_layers=None):
                 k = to_device(synth.kv_tensor(cfg, l, frames, "k"), cfg.dtype)
                 v = to_device(synth.kv_tensor(cfg, l, frames, "v"), cfg.dtype)
                 sess.full_attention(l, q, k, v, (lay["sink_begin"], lay["sink_end"]),
-                                    (lay["chunk_begin"], lay["chunk_end"]), o, lse, collect=in_warmup)
+                                    (lay["chunk_begin"], lay["chunk_end"]), o, lse, collect=in_warmup,
+                                    monitor=watch)
                 chunk_out.append(dict(O=o, y=None, local=False))
         outputs.append(chunk_out)
+        if watch:
+            live.append((t, sess.live_errors()))
+            f = sess.rewarm_layers()
+            fired.append((t, f))
+            if f and rewarm == "auto":
+                pending_rewarm = True
         if in_warmup and t == warm_start + cfg.warmup_chunks - 1:
             idx = sess.transition()
             transitions.append(dict(chunk=t, eps=list(sess.eps_host), idx=idx, is_local=list(sess.is_local),
                                     dW=sess.dW.clone(), rows=[int(s.rows.item()) for s in sess.stats]))
     torch.cuda.synchronize()
     assert ispa.ispa_device_status() == ispa.ISPA_OK
-    return dict(transitions=transitions, outputs=outputs)
+    return dict(transitions=transitions, outputs=outputs, live=live, fired=fired)
 
 
 def _compare_runs(cfg, got, want, attn_tol, eps_tol, dW_tol=None, y_tol=None):
@@ -126,6 +143,36 @@ def test_structured_run_with_scene_cut_and_rewarmup(K):
         planted = [tr["eps"][l] for l in range(cfg.layers) if cfg.planted(l)]
         iid = [tr["eps"][l] for l in range(cfg.layers) if not cfg.planted(l)]
         assert max(planted) < 0.25 * min(iid)
+    _compare_runs(cfg, got, want, attn_tol=2e-2, eps_tol=5e-2, y_tol=5e-2)
+
+
+def test_structured_live_error_detects_the_scene_cut():
+    """Re-warmup trigger, no scheduled re-warmup: the live errors of the F-layers against the
+    oracle's (eps tolerance of the bf16 chain), and the trigger fires at the cut chunk, for the
+    planted F-layer only, as the oracle's statement of the rule does on the oracle's errors."""
+    cfg = _small_structured(K=1)
+    got = gpu_episode(cfg, K=1, rewarm=None, monitor=True)
+    want = oracle.run_episode(cfg, K=1, rewarm_at=None, monitor=True)
+    assert [t for t, _ in got["live"]] == [t for t, _ in want["live"]] == [3, 4, 5, 6, 7]
+    prev = []
+    for (t, lg), (_, lw), (_, fg) in zip(got["live"], want["live"], got["fired"]):
+        assert sorted(lg) == sorted(lw)
+        for l in lw:
+            assert abs(lg[l] - lw[l]) <= 5e-2 * abs(lw[l]) + 1e-4, (t, l, lg[l], lw[l])
+        assert fg == oracle.rewarm_trigger(prev, lw), (t, fg)
+        prev.append(lw)
+    first = next(t for t, f in got["fired"] if f)
+    assert first == cfg.cut_chunk
+    assert dict(got["fired"])[first] == [l for l in range(cfg.layers) if cfg.planted(l) and l not in got["transitions"][0]["idx"]]
+
+
+def test_structured_run_with_automatic_rewarmup():
+    """The trigger drives the re-warmup: it fires at the cut, the warmup restarts at the next
+    chunk, and the whole run matches the oracle scheduled to re-warm there."""
+    cfg = _small_structured(K=1, total_chunks=10)
+    got = gpu_episode(cfg, K=1, rewarm="auto")
+    want = oracle.run_episode(cfg, K=1, rewarm_at=cfg.cut_chunk + 1, keep_outputs=True)
+    assert [t["chunk"] for t in got["transitions"]] == [2, cfg.cut_chunk + 3]
     _compare_runs(cfg, got, want, attn_tol=2e-2, eps_tol=5e-2, y_tol=5e-2)
 
 

@@ -192,6 +192,44 @@ def test_solve_absorb_matches_oracle(dtype, D, L):
     assert ispa.ispa_select_layers(eps_gpu, 1)[0] == oracle.select_layers(eps_ref, 1)[0]
 
 
+@pytest.mark.parametrize("dtype,D,L", [("fp32", 128, 2), ("bf16", 256, 3), ("bf16", 1536, 2)])
+def test_absorb_error_of_a_given_dW_matches_oracle(dtype, D, L):
+    """ispa_absorb_error: eps of a given dW on given statistics (the live error of the
+    re-warmup trigger), against the oracle's trace formula on the same float32 inputs. D = 1536
+    runs the 3xTF32 tensor-core products, D = 128 and 256 too (multiples of 128)."""
+    n = max(2 * D, 512)
+    stats_np = [_oracle_stats_for(dtype, 60 + l, n, D, planted=(l % 2 == 0)) for l in range(L)]
+    W_np = [synth.normal_tensor(70 + l, (31,), (D, D), dtype, std=1 / math.sqrt(D)) for l in range(L)]
+    dW_np = [synth.normal_tensor(80 + l, (32,), (D, D), "fp32", std=0.3 / math.sqrt(D)) for l in range(L)]
+    stats = []
+    for s in stats_np:
+        st = ispa.Stats(D)
+        st.G.copy_(torch.from_numpy(s["G"].astype(np.float32)))
+        st.C.copy_(torch.from_numpy(s["C"].astype(np.float32)))
+        st.H.copy_(torch.from_numpy(s["H"].astype(np.float32)))
+        stats.append(st)
+    Ws = [to_device(w, dtype) for w in W_np]
+    dWs = [torch.from_numpy(d).cuda() for d in dW_np]
+    eps = torch.full((L,), float("nan"), device="cuda")
+    terms = torch.zeros((L, 2), dtype=torch.float64, device="cuda")
+    ws = ispa.alloc_workspace(ispa.workspace_bytes(None, L, D))
+    code = ispa.ISPA_BF16 if dtype == "bf16" else ispa.ISPA_FP32
+    ispa.ispa_absorb_error(stats, Ws, code, dWs, eps, terms, ws)
+    torch.cuda.synchronize()
+    assert ispa.ispa_device_status() == ispa.ISPA_OK
+    for l in range(L):
+        G = stats_np[l]["G"].astype(np.float32).astype(np.float64)
+        C = stats_np[l]["C"].astype(np.float32).astype(np.float64)
+        H = stats_np[l]["H"].astype(np.float32).astype(np.float64)
+        e = oracle.reconstruction_error(G, C, H, W_np[l], dW_np[l])
+        assert abs(float(eps[l]) - e["eps"]) <= 1e-3 * abs(e["eps"]) + 4e-6, (l, float(eps[l]), e["eps"])
+        assert abs(float(terms[l, 0]) - e["E2"]) <= 1e-3 * abs(e["E2"]) + 4e-6 * abs(e["T2"])
+        assert abs(float(terms[l, 1]) - e["T2"]) <= 1e-4 * abs(e["T2"])
+    # the statistics are read only
+    for st, s in zip(stats, stats_np):
+        assert np.array_equal(to_numpy(st.G), s["G"].astype(np.float32))
+
+
 def test_solve_reports_non_spd_layers():
     D = 128
     st_bad, st_ok = ispa.Stats(D), ispa.Stats(D)

@@ -322,3 +322,47 @@ def test_episode_warmup_schedule_rows():
     tr = out["transitions"][0]
     assert tr["chunk"] == cfg.warmup_chunks - 1 and len(tr["idx"]) == cfg.K
     assert len(out["outputs"]) == cfg.warmup_chunks
+
+
+# ------------------------------------------------------------------ re-warmup trigger (step 7)
+def test_live_error_is_the_relative_residual_of_one_chunk():
+    """eps_live from one chunk's statistics equals ||A_loc (W + dW) - A_full W||^2 /
+    ||A_full W||^2 computed directly on that chunk (fp32 mode: no operand rounding)."""
+    rng = np.random.default_rng(11)
+    n, D = 60, 16
+    a_loc = rng.standard_normal((n, 1, D))
+    a_full = a_loc + 0.3 * rng.standard_normal((n, 1, D))
+    W = rng.standard_normal((D, D)) / 4
+    dW = 0.1 * rng.standard_normal((D, D))
+    got = oracle.live_error(a_loc, a_full, "fp32", W, dW)
+    A, F = a_loc.reshape(n, D), a_full.reshape(n, D)
+    want = np.sum((A @ (W + dW) - F @ W) ** 2) / np.sum((F @ W) ** 2)
+    assert got == pytest.approx(want, rel=1e-12)
+    # no history at all: the residual is zero and dW = 0 reconstructs exactly
+    assert oracle.live_error(a_loc, a_loc, "fp32", W, np.zeros((D, D))) == 0.0
+
+
+def test_rewarm_trigger_rule_cases():
+    hist = [{1: 0.01, 2: 2.0}, {1: 0.012, 2: 2.4}]
+    assert oracle.rewarm_trigger(hist, {1: 0.3, 2: 2.2}) == [1]          # 30x its minimum, +0.29
+    assert oracle.rewarm_trigger(hist, {1: 0.011, 2: 7.0}) == []         # 3.5x its minimum: not enough
+    assert oracle.rewarm_trigger(hist, {1: 0.011, 2: 8.5}) == [2]        # 4.25x
+    assert oracle.rewarm_trigger(hist, {1: 0.029, 2: 2.0}) == []         # 2.9x, below the ratio
+    assert oracle.rewarm_trigger([{3: 1e-4}], {3: 9e-3}) == []           # 90x but a rise of 0.009 only
+    assert oracle.rewarm_trigger([], {1: 5.0}) == []                     # no reference yet
+    assert oracle.rewarm_trigger(hist, {4: 5.0}) == []                   # a layer never seen before
+
+
+def test_live_error_fires_at_the_scene_cut_only():
+    """Structured workload, no scheduled re-warmup: the planted layer that stayed an F-layer
+    keeps a small live error until the cut, where it jumps; the i.i.d. layers stay put."""
+    cfg = _small(structured=True, cut_chunk=5, total_chunks=8, K=1)
+    out = oracle.run_episode(cfg, K=1, rewarm_at=None, monitor=True)
+    assert [t for t, _ in out["live"]] == [3, 4, 5, 6, 7]
+    fired, prev = {}, []
+    for t, live in out["live"]:
+        assert set(live) == {l for l in range(cfg.layers) if l not in out["transitions"][0]["idx"]}
+        fired[t] = oracle.rewarm_trigger(prev, live)
+        prev.append(live)
+    planted_f = [l for l in range(cfg.layers) if cfg.planted(l) and l not in out["transitions"][0]["idx"]]
+    assert planted_f and fired[3] == [] and fired[4] == [] and fired[5] == planted_f

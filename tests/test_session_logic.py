@@ -1,0 +1,39 @@
+"""Host logic of the streaming session that needs no GPU: the re-warmup trigger rule, against
+the oracle's statement of the same rule on hand cases and random live-error histories."""
+import types
+
+import numpy as np
+
+import oracle
+from streaming_video_attention_b200.session import IspaSession
+
+
+def _session_rule(history):
+    fake = types.SimpleNamespace(live_history=history, RATIO=IspaSession.RATIO, MIN_RISE=IspaSession.MIN_RISE)
+    return IspaSession.rewarm_layers(fake)
+
+
+def test_rule_needs_a_reference_chunk():
+    assert _session_rule([]) == []
+    assert _session_rule([{0: 3.0}]) == []
+
+
+def test_rule_hand_cases():
+    hist = [{1: 0.01, 2: 2.0}, {1: 0.012, 2: 2.4}]
+    assert _session_rule(hist + [{1: 0.3, 2: 2.2}]) == [1]
+    assert _session_rule(hist + [{1: 0.011, 2: 8.5}]) == [2]
+    assert _session_rule(hist + [{1: 0.029, 2: 2.0}]) == []
+    assert _session_rule([{3: 1e-4}, {3: 9e-3}]) == []
+
+
+def test_rule_matches_oracle_on_random_histories():
+    rng = np.random.default_rng(3)
+    for _ in range(300):
+        n_chunks = int(rng.integers(2, 7))
+        layers = list(range(int(rng.integers(1, 6))))
+        hist = []
+        for _ in range(n_chunks):
+            present = [l for l in layers if rng.random() < 0.9]
+            hist.append({l: float(np.exp(rng.normal(-3.0, 2.0))) for l in present})
+        want = oracle.rewarm_trigger(hist[:-1], hist[-1])
+        assert _session_rule(hist) == want, hist
