@@ -54,6 +54,8 @@ def parse_args(argv=None):
                     help="episode: the full step (default). call / local / solve: one layer's fused split "
                          "attention at the last warmup chunk, one L-layer local attention with projection, or "
                          "the batched solve alone (kernel-level timing, also the target of ncu captures)")
+    ap.add_argument("--w8a8", action="store_true",
+                    help="local mode: the L-layer projection through int8 weights and activations")
     ap.add_argument("--attn-kernel", choices=["auto", "single", "pair"], default="auto",
                     help="bf16 head_dim-128 attention kernel: one CTA per query tile, or CTA pairs "
                          "(cta_group::2); auto = the library's default")
@@ -511,7 +513,7 @@ def unit_arm(args, cfg):
     t = cfg.warmup_chunks - 1
     D = cfg.D
     sess = IspaSession(1 if args.mode != "solve" else cfg.layers, cfg.heads, cfg.head_dim, cfg.lam, 1, "bf16",
-                       str(device))
+                       str(device), w8a8=args.w8a8)
     if args.mode in ("call", "local"):
         if args.mode == "call":
             frames = synth.cache_frames(cfg, t)
@@ -538,9 +540,14 @@ def unit_arm(args, cfg):
             what = f"fused split attention + statistics, one layer, n_q {cfg.n_q}, n_kv {n_kv}"
         else:
             sess.is_local = [1]
+            if args.w8a8:
+                sess.wq[0] = torch.empty(D, D, dtype=torch.int8, device=device)
+                sess.wq_scale[0] = torch.empty(D, dtype=torch.float32, device=device)
+                ispa.ispa_quantize_w8(sess.W_new[0], ispa.ISPA_BF16, sess.wq[0], sess.wq_scale[0])
             fn = lambda: sess.local_attention(0, q, k, v, o, lse, y)
             flops = 4.0 * cfg.n_q * n_kv * cfg.head_dim * cfg.heads + 2.0 * cfg.n_q * D * D
-            what = f"L-layer local attention + W_new projection, n_q {cfg.n_q}, n_kv {n_kv}"
+            what = (f"L-layer local attention + W_new projection{' (W8A8 int8)' if args.w8a8 else ''}, "
+                    f"n_q {cfg.n_q}, n_kv {n_kv}")
     else:
         Ws = [up(synth.w_out(cfg, l)) for l in range(cfg.layers)]
         sess.set_weights(Ws)

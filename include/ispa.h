@@ -183,9 +183,32 @@ int ispa_local_attn(const ispa_attn_desc *desc, const void *q, const void *k_loc
                     const void *v_loc, void *o, float *lse, const void *w_new, void *y, void *ws,
                     size_t ws_bytes, ispa_stream_t stream);
 
+/* ispa_quantize_w8 -- int8 weights for the W8A8 projection of the L-layers [ISPA §4.4: ISPA
+ * is combined with 8-bit weights and activations; the scheme is not given -- reading:
+ * symmetric int8, one scale per output column]. For each output column j of w [d_in][d_out]
+ * (row-major, bf16 or float32, device): w_scale[j] = m / 127 with m = max_i |w[i][j]|, and
+ * wq_t[j][i] = rint(w[i][j] * (127 / m)) clamped to [-127, 127] (float32 IEEE division and
+ * multiplication, round to nearest even; a zero column gives scale 0 and codes 0). wq_t is
+ * int8 [d_out][d_in] (transposed, 16-byte aligned), w_scale float32 [d_out]. d_in and d_out:
+ * positive multiples of 128. Run once per transition on W_new. */
+int ispa_quantize_w8(const void *w, ispa_dtype w_dtype, int d_in, int d_out, signed char *wq_t,
+                     float *w_scale, ispa_stream_t stream);
+
+/* ispa_project_w8a8 -- y = A W through int8 operands [ISPA §4.4, reading as for
+ * ispa_quantize_w8]: each row r of a [n][d_in] (bf16, device, 16-byte aligned) is quantised
+ * like a weight column (scale s_r = max|a_r| / 127), the int8 product accumulates exactly in
+ * int32 on the tensor cores, and y[r][j] = bf16((float(acc) * s_r) * w_scale[j]) (round to
+ * nearest even at each step) -- reproducible bit for bit. wq_t / w_scale from
+ * ispa_quantize_w8; y [n][d_out] bf16 (device, 16-byte aligned). ws: scratch for the row codes
+ * and scales, ispa_workspace_bytes(NULL, n, d_in) bytes (or the attention call's desc with
+ * n_q = n). d_in and d_out: positive multiples of 128. */
+int ispa_project_w8a8(const void *a, int n, int d_in, const signed char *wq_t, const float *w_scale,
+                      int d_out, void *y, void *ws, size_t ws_bytes, ispa_stream_t stream);
+
 /* ispa_workspace_bytes -- bytes of workspace that suffice for every call above with
  * these shapes: attention calls described by `desc` (may be NULL), ispa_accum_stats
- * with n_rows = n (when desc is NULL) and ispa_solve_absorb over n layers of size D. */
+ * and ispa_project_w8a8 with n rows of width D (when desc is NULL; with desc: n_q rows of
+ * width heads*head_dim) and ispa_solve_absorb / ispa_absorb_error over n layers of size D. */
 size_t ispa_workspace_bytes(const ispa_attn_desc *desc, int n, int D);
 
 /* ispa_device_status -- synchronise `stream`, read and clear the current device's

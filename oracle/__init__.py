@@ -20,4 +20,6 @@ from .ispa_oracle import (  # noqa: F401
     run_episode,
     live_error,
     rewarm_trigger,
+    quantize_int8,
+    project_w8a8,
 )

@@ -211,6 +211,39 @@ def project(A: np.ndarray, W: np.ndarray) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------------------
+# W8A8 projection of the L-layers [ISPA §4.4: ISPA combined with 8-bit weights and
+# activations for the linear layers; the scheme is not given]. Reading: int8, symmetric,
+# one scale per activation row (token) and one per weight output column; scales and the
+# quantisation in float32 (round to nearest, ties to even, clamp to +-127); exact integer
+# accumulation; y = bf16((float32(acc) * s_row) * s_col). Every step is a plain float32 or
+# integer operation, so the GPU result is reproducible bit for bit.
+# --------------------------------------------------------------------------------------
+def quantize_int8(x: np.ndarray, axis: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Symmetric int8 quantisation along `axis` (the reduced axis). Returns (q, scale) with
+    scale = amax / 127 (float32) and q = rint(x * (127 / amax)) clamped to [-127, 127]; an
+    all-zero slice has scale 0 and q = 0."""
+    x = np.asarray(x, dtype=np.float32)
+    amax = np.max(np.abs(x), axis=axis, keepdims=True).astype(np.float32)
+    inv = np.zeros_like(amax)
+    nz = amax > 0
+    inv[nz] = np.float32(127.0) / amax[nz]
+    q = np.clip(np.rint(x * inv), -127, 127).astype(np.int8)
+    scale = (amax / np.float32(127.0)).astype(np.float32)
+    return q, np.squeeze(scale, axis=axis)
+
+
+def project_w8a8(A: np.ndarray, W: np.ndarray) -> np.ndarray:
+    """y = A W through the int8 path above; A [n, D_in] (or [n, h, d]), W [D_in, D_out].
+    Returns the bf16-rounded values as float64."""
+    n = A.shape[0]
+    qa, sa = quantize_int8(np.asarray(A, np.float32).reshape(n, -1), axis=1)
+    qw, sw = quantize_int8(np.asarray(W, np.float32), axis=0)
+    acc = qa.astype(np.int64) @ qw.astype(np.int64)
+    y = (acc.astype(np.float32) * sa[:, None]) * sw[None, :]
+    return bf16_round(y.astype(np.float64))
+
+
+# --------------------------------------------------------------------------------------
 # A whole streaming run, chunk by chunk [ISPA §3.1, §3.3 re-triggered warmup].
 # --------------------------------------------------------------------------------------
 def live_error(A_loc, A_full, dtype: str, W, dW) -> float:

@@ -101,6 +101,11 @@ size_t accum_ws_bytes(int n_rows, int D, ispa_dtype t) {
     return align_up((size_t)n_rows * D * elem_size(t), 256);
 }
 
+// ispa_project_w8a8: int8 codes [n][D] then float scales [n]
+size_t w8a8_ws_bytes(int n_rows, int D) {
+    return align_up((size_t)n_rows * D, 256) + align_up((size_t)n_rows * sizeof(float), 256);
+}
+
 constexpr int kEpsParts = 64;
 
 size_t solve_ws_bytes(int n_layers, int D) {
@@ -282,8 +287,10 @@ size_t ispa_workspace_bytes(const ispa_attn_desc *desc, int n, int D) {
         need = std::max(need, attn_ws_bytes(desc));
         const size_t Dd = (size_t)desc->heads * desc->head_dim;
         need = std::max(need, align_up((size_t)desc->n_q * Dd * elem_size(desc->dtype), 256));
+        need = std::max(need, w8a8_ws_bytes(desc->n_q, (int)Dd));
     } else if (n > 0 && D > 0) {
         need = std::max(need, accum_ws_bytes(n, D, ISPA_FP32));
+        need = std::max(need, w8a8_ws_bytes(n, D));
     }
     if (n > 0 && D > 0) need = std::max(need, solve_ws_bytes(n, D));
     return need;
@@ -472,6 +479,44 @@ int ispa_absorb_error(const ispa_stats *per_layer, int n_layers, const void *con
                                     s);
         if (e != cudaSuccess) return cuda_fail(e, "absorb error");
     }
+    return ISPA_OK;
+}
+
+int ispa_quantize_w8(const void *w, ispa_dtype w_dtype, int d_in, int d_out, signed char *wq_t, float *w_scale,
+                     ispa_stream_t stream) {
+    g_last_error.clear();
+    if (!w || !wq_t || !w_scale) return fail(ISPA_ERR_INVALID_ARG, "w, wq_t and w_scale are required");
+    if (w_dtype != ISPA_BF16 && w_dtype != ISPA_FP32) return fail(ISPA_ERR_INVALID_ARG, "bad w_dtype");
+    if (d_in <= 0 || d_out <= 0 || d_in % 128 || d_out % 128)
+        return fail(ISPA_ERR_UNSUPPORTED, "d_in=%d d_out=%d: both must be positive multiples of 128", d_in, d_out);
+    if (!aligned(wq_t, 16)) return fail(ISPA_ERR_INVALID_ARG, "wq_t must be 16-byte aligned");
+    cudaError_t e = launch_quant_cols(w, w_dtype == ISPA_BF16 ? ElemType::BF16 : ElemType::F32, d_in, d_out,
+                                      reinterpret_cast<int8_t *>(wq_t), w_scale,
+                                      reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "weight quantisation");
+    return ISPA_OK;
+}
+
+int ispa_project_w8a8(const void *a, int n, int d_in, const signed char *wq_t, const float *w_scale, int d_out,
+                      void *y, void *ws, size_t ws_bytes, ispa_stream_t stream) {
+    g_last_error.clear();
+    if (n < 0) return fail(ISPA_ERR_INVALID_ARG, "n < 0");
+    if (n == 0) return ISPA_OK;
+    if (!a || !wq_t || !w_scale || !y) return fail(ISPA_ERR_INVALID_ARG, "a, wq_t, w_scale and y are required");
+    if (d_in <= 0 || d_out <= 0 || d_in % 128 || d_out % 128)
+        return fail(ISPA_ERR_UNSUPPORTED, "d_in=%d d_out=%d: both must be positive multiples of 128", d_in, d_out);
+    if (!aligned(a, 16) || !aligned(y, 16) || !aligned(wq_t, 16))
+        return fail(ISPA_ERR_INVALID_ARG, "a, y and wq_t must be 16-byte aligned");
+    int rc = check_ws(ws, ws_bytes, w8a8_ws_bytes(n, d_in));
+    if (rc != ISPA_OK) return rc;
+    int *flag = nullptr;
+    rc = device_error_flag(&flag);
+    if (rc != ISPA_OK) return rc;
+    int8_t *q_a = static_cast<int8_t *>(ws);
+    float *s_a = reinterpret_cast<float *>(static_cast<char *>(ws) + align_up((size_t)n * d_in, 256));
+    cudaError_t e = launch_project_w8a8(a, n, d_in, reinterpret_cast<const int8_t *>(wq_t), w_scale, d_out, y, q_a,
+                                        s_a, flag, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "W8A8 projection");
     return ISPA_OK;
 }
 

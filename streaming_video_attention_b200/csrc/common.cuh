@@ -93,6 +93,12 @@ cudaError_t launch_stats_bf16(const void *a_loc, const void *r, int n, int D, fl
 cudaError_t launch_gemm_bf16(const void *A, const void *W, void *y, int M, int N, int K, int *err_flag,
                              cudaStream_t s);
 
+// W8A8 projection (w8a8_sm100.cu): weights [K][N] -> int8 [N][K] + column scales; then
+// y[M][N] (bf16) from activations A [M][K] (bf16) quantised by rows into q_a / s_a.
+cudaError_t launch_quant_cols(const void *w, ElemType t, int K, int N, int8_t *qt, float *scale, cudaStream_t s);
+cudaError_t launch_project_w8a8(const void *A, int M, int K, const int8_t *qt, const float *col_scale, int N,
+                                void *y, int8_t *q_a, float *s_a, int *err_flag, cudaStream_t s);
+
 // Solve-phase kernels (float32, batched over layers).
 struct PtrBatch {
     void *p[kMaxBatch];

@@ -29,7 +29,7 @@ ISPA_FP32 = 1
 
 EXPORTS = (
     "ispa_attn_split", "ispa_attn_split_noalloc", "ispa_accum_stats", "ispa_stats_reset", "ispa_solve_absorb",
-    "ispa_absorb_error", "ispa_select_layers",
+    "ispa_absorb_error", "ispa_quantize_w8", "ispa_project_w8a8", "ispa_select_layers",
     "ispa_local_attn", "ispa_workspace_bytes", "ispa_device_status", "ispa_selftest_bounded_wait",
     "ispa_selftest_exp2_poly", "ispa_set_attn_kernel", "ispa_kernel_launches", "ispa_last_error", "ispa_version",
 )
@@ -193,6 +193,22 @@ def ispa_absorb_error(stats: Sequence[Stats], w_o: Sequence[torch.Tensor], w_dty
     rc = lib().ispa_absorb_error(arr, L, wp, w_dtype, dp, _p(eps), _p(err_terms), _p(ws),
                                  0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "ispa_absorb_error")
+
+
+def ispa_quantize_w8(w: torch.Tensor, w_dtype: int, wq_t: torch.Tensor, w_scale: torch.Tensor, stream=None) -> None:
+    d_in, d_out = w.shape
+    rc = lib().ispa_quantize_w8(_p(w), w_dtype, d_in, d_out, _p(wq_t), _p(w_scale), _stream(stream))
+    _check(rc, "ispa_quantize_w8")
+
+
+def ispa_project_w8a8(a: torch.Tensor, wq_t: torch.Tensor, w_scale: torch.Tensor, y: torch.Tensor,
+                      ws: Optional[torch.Tensor] = None, stream=None) -> None:
+    n = a.shape[0]
+    d_in = a.numel() // max(1, n)
+    d_out = wq_t.shape[0]
+    rc = lib().ispa_project_w8a8(_p(a), n, d_in, _p(wq_t), _p(w_scale), d_out, _p(y), _p(ws),
+                                 0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "ispa_project_w8a8")
 
 
 def ispa_select_layers(eps: Sequence[float], K: int):

@@ -34,7 +34,7 @@ class IspaSession:
     MIN_RISE = 0.02    # ... and above that minimum + MIN_RISE
 
     def __init__(self, layers: int, heads: int, head_dim: int, lam: float, K: int, dtype: str = "bf16",
-                 device: str = "cuda"):
+                 device: str = "cuda", w8a8: bool = False):
         self.layers, self.heads, self.head_dim = layers, heads, head_dim
         self.D = heads * head_dim
         self.lam, self.K = float(lam), int(K)
@@ -55,6 +55,10 @@ class IspaSession:
         self.idx: List[int] = []
         self.eps_host: List[float] = []
         self.transitions = 0
+        # W8A8 projection of the L-layers (int8 codes of W_new, transposed, and column scales)
+        self.w8a8 = bool(w8a8) and dtype == "bf16"
+        self.wq: List[Optional[torch.Tensor]] = [None] * layers
+        self.wq_scale: List[Optional[torch.Tensor]] = [None] * layers
         self.monitor: List[Optional[ispa.Stats]] = [None] * layers
         self.live_history: List[Dict[int, float]] = []
         self._eps_live = torch.empty(layers, dtype=torch.float32, device=device)
@@ -112,12 +116,16 @@ class IspaSession:
         ispa.ispa_attn_split(desc, q, k, v, o, lse, o_loc, lse_loc, o_hist, lse_hist, stats=st, ws=ws, stream=stream)
 
     def local_attention(self, layer: int, q, k_loc, v_loc, o, lse=None, y=None, stream=None) -> None:
-        """An L-layer call: sink + chunk rows only; y = O W_new when y is given."""
+        """An L-layer call: sink + chunk rows only; y = O W_new when y is given (through the
+        int8 W8A8 path when the session was created with w8a8=True)."""
         n_q, n_kv = q.shape[0], k_loc.shape[0]
         desc = ispa.make_desc(n_q, n_kv, self.heads, self.head_dim, dtype=self.code)
-        w = self.W_new[layer] if y is not None else None
-        ws = self._attn_ws(desc) if lse is None else None
-        ispa.ispa_local_attn(desc, q, k_loc, v_loc, o, lse, w, y, ws=ws, stream=stream)
+        quant = self.w8a8 and y is not None
+        w = self.W_new[layer] if (y is not None and not quant) else None
+        ws = self._attn_ws(desc) if (lse is None or quant) else None
+        ispa.ispa_local_attn(desc, q, k_loc, v_loc, o, lse, w, None if quant else y, ws=ws, stream=stream)
+        if quant:
+            ispa.ispa_project_w8a8(o, self.wq[layer], self.wq_scale[layer], y, ws=ws, stream=stream)
 
     # ---------------------------------------------------------------- the switch
     def transition(self, K: Optional[int] = None, stream=None) -> List[int]:
@@ -132,6 +140,12 @@ class IspaSession:
         self.is_local = [int(f) for f in flags]
         self.transitions += 1
         self._reset_monitor(stream)
+        if self.w8a8:
+            for l in self.idx:
+                if self.wq[l] is None:
+                    self.wq[l] = torch.empty(self.D, self.D, dtype=torch.int8, device=self.device)
+                    self.wq_scale[l] = torch.empty(self.D, dtype=torch.float32, device=self.device)
+                ispa.ispa_quantize_w8(self.W_new[l], self.code, self.wq[l], self.wq_scale[l], stream)
         if any(s != ispa.ISPA_OK for s in status):
             bad = [l for l, s in enumerate(status) if s != ispa.ISPA_OK]
             raise ispa.IspaError(ispa.ISPA_ERR_NOT_SPD, "transition", f"G + lambda I not SPD in layers {bad}")

@@ -91,3 +91,17 @@ def test_set_attn_kernel_choice_round_trips():
         assert ispa.ispa_set_attn_kernel(ispa.ISPA_ATTN_AUTO) == ispa.ISPA_ATTN_SINGLE
     finally:
         ispa.ispa_set_attn_kernel(prev)
+
+
+def test_w8a8_arguments_are_checked_before_any_launch():
+    L = ispa.lib()
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: every call below fails its checks first
+    assert L.ispa_quantize_w8(None, ispa.ISPA_BF16, 128, 128, fake, fake, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_quantize_w8(fake, ispa.ISPA_BF16, 96, 128, fake, fake, None) == ispa.ISPA_ERR_UNSUPPORTED
+    assert L.ispa_quantize_w8(fake, 7, 128, 128, fake, fake, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_project_w8a8(fake, 10, 128, fake, fake, 200, fake, None, 0, None) == ispa.ISPA_ERR_UNSUPPORTED
+    assert L.ispa_project_w8a8(fake, 10, 128, fake, fake, 128, fake, None, 0, None) == ispa.ISPA_ERR_WORKSPACE
+    assert L.ispa_project_w8a8(None, 10, 128, fake, fake, 128, fake, None, 0, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_project_w8a8(fake, 0, 128, fake, fake, 128, fake, None, 0, None) == ispa.ISPA_OK
+    # the workspace covers the row codes and scales
+    assert ispa.workspace_bytes(None, 4680, 1536) >= 4680 * 1536 + 4 * 4680

@@ -366,3 +366,49 @@ def test_live_error_fires_at_the_scene_cut_only():
         prev.append(live)
     planted_f = [l for l in range(cfg.layers) if cfg.planted(l) and l not in out["transitions"][0]["idx"]]
     assert planted_f and fired[3] == [] and fired[4] == [] and fired[5] == planted_f
+
+
+# ------------------------------------------------------------------ W8A8 projection
+def test_int8_quantization_hand_cases():
+    q, s = oracle.quantize_int8(np.array([[1.0, -2.0, 0.5], [0.0, 0.0, 0.0]]), axis=1)
+    assert q.tolist() == [[64, -127, 32], [0, 0, 0]]            # 63.5 rounds to even (64); 31.75 -> 32
+    assert s[0] == np.float32(2.0) / np.float32(127.0) and s[1] == 0.0
+    qc, sc = oracle.quantize_int8(np.array([[1.0, 4.0], [-3.0, 2.0]]), axis=0)
+    assert qc.tolist() == [[42, 127], [-127, 64]]               # columns: amax 3 and 4; 42.33 -> 42, 63.5 -> 64
+    assert sc.tolist() == [np.float32(3.0) / np.float32(127.0), np.float32(4.0) / np.float32(127.0)]
+
+
+def test_int8_quantization_error_bound():
+    rng = np.random.default_rng(4)
+    x = (rng.standard_normal((40, 96)) * np.exp(rng.normal(0, 2, (40, 1)))).astype(np.float32)
+    q, s = oracle.quantize_int8(x, axis=1)
+    err = np.abs(x.astype(np.float64) - q.astype(np.float64) * s[:, None].astype(np.float64))
+    assert np.all(err <= 0.5 * s[:, None] * (1 + 1e-5) + 1e-30)
+    assert np.all(np.abs(q).max(axis=1) == 127)                 # the largest element of a row maps to 127
+
+
+def test_w8a8_scale_invariances_and_error_bound():
+    """Per-row activation scales and per-column weight scales: doubling a row of A or a
+    column of W doubles exactly that row or column of y; y is within the quantisation
+    bound of the float64 product."""
+    rng = np.random.default_rng(5)
+    n, K, N = 24, 64, 40
+    A = synth_bf16(rng.standard_normal((n, K)))
+    W = synth_bf16(rng.standard_normal((K, N)) / 8)
+    y = oracle.project_w8a8(A, W)
+    A2 = A.copy(); A2[3] *= 2
+    W2 = W.copy(); W2[:, 7] *= 2
+    y2 = oracle.project_w8a8(A2, W)
+    y3 = oracle.project_w8a8(A, W2)
+    assert np.array_equal(y2[3], 2 * y[3]) and np.array_equal(np.delete(y2, 3, 0), np.delete(y, 3, 0))
+    assert np.array_equal(y3[:, 7], 2 * y[:, 7]) and np.array_equal(np.delete(y3, 7, 1), np.delete(y, 7, 1))
+    exact = A.astype(np.float64) @ W.astype(np.float64)
+    sa = np.abs(A).max(axis=1, keepdims=True) / 127
+    sw = np.abs(W).max(axis=0, keepdims=True) / 127
+    # |A W - Aq Wq| <= sum_k (|a_k| e_w + |w_k| e_a + e_a e_w), e = half a step; plus bf16 rounding
+    bound = (np.abs(A) @ np.ones((K, N))) * 0.5 * sw + 0.5 * sa * (np.ones((n, K)) @ np.abs(W)) + K * 0.25 * sa * sw
+    assert np.all(np.abs(y - exact) <= bound * (1 + 1e-6) + np.abs(exact) * 2.0 ** -8 + 1e-12)
+
+
+def synth_bf16(x):
+    return oracle.bf16_round(np.asarray(x, np.float64)).astype(np.float32)
