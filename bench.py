@@ -376,6 +376,18 @@ def reference_arm(args, cfg, rank):
     return 0
 
 
+def kv_block(cfg, is_local):
+    """K/V bytes held per replica before the transition (every layer F) and after it (the
+    selected L-layers keep only the sink and the chunk)."""
+    from streaming_video_attention_b200.session import kv_cache_bytes
+    hist = cfg.kv_window - cfg.sink_frames
+    args = (hist, cfg.chunk_frames, cfg.sink_frames, cfg.tpf, cfg.D, 2)
+    before = kv_cache_bytes([0] * cfg.layers, *args)
+    after = kv_cache_bytes(is_local, *args)
+    return {"before_bytes": before, "after_bytes": after, "removed_frac": (before - after) / before,
+            "l_layers": int(sum(is_local))}
+
+
 def config_block(cfg, n):
     return {
         "workload": (f"{cfg.name}: ISPA episode, {cfg.layers} layers x {cfg.heads} heads x {cfg.head_dim}, "
@@ -491,6 +503,7 @@ def ispa_arm(args, cfg, rank, world, local_rank):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_block(cfg, world),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches), "clocks": clk,
             "selection": {"idx": sess.idx, "margin": sess.selection_margin()},
+            "kv_cache": kv_block(cfg, sess.is_local),
             "input_generation_s": gen_s,
         }
         print(json.dumps(line), flush=True)

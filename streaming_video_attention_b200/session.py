@@ -29,6 +29,20 @@ import torch
 from . import ispa
 
 
+def kv_cache_bytes(is_local: Sequence[int], history_frames: int, chunk_frames: int, sink_frames: int,
+                   tokens_per_frame: int, D: int, elem_bytes: int = 2) -> int:
+    """Bytes of K and V held across the layers [ISPA §3.1 step 3: an L-layer keeps only the sink
+    and the current chunk, its history is evicted; an F-layer keeps the sink, its recent history
+    frames and the chunk]. history_frames counts the frames an F-layer holds besides the sink and
+    the chunk."""
+    per_frame = 2 * tokens_per_frame * D * elem_bytes
+    total = 0
+    for loc in is_local:
+        frames = sink_frames + chunk_frames + (0 if loc else history_frames)
+        total += frames * per_frame
+    return total
+
+
 class IspaSession:
     RATIO = 4.0        # live error above RATIO x its minimum since the transition ...
     MIN_RISE = 0.02    # ... and above that minimum + MIN_RISE

@@ -37,3 +37,19 @@ def test_rule_matches_oracle_on_random_histories():
             hist.append({l: float(np.exp(rng.normal(-3.0, 2.0))) for l in present})
         want = oracle.rewarm_trigger(hist[:-1], hist[-1])
         assert _session_rule(hist) == want, hist
+
+
+def test_kv_cache_accounting():
+    from streaming_video_attention_b200.session import kv_cache_bytes
+    # one frame of K and V at the 1.3B shape: 2 x 1560 tokens x 1536 x 2 bytes
+    frame = 2 * 1560 * 1536 * 2
+    assert kv_cache_bytes([0], 20, 3, 1, 1560, 1536) == 24 * frame          # sink + 20 history + chunk
+    assert kv_cache_bytes([1], 20, 3, 1, 1560, 1536) == 4 * frame           # sink + chunk
+    before = kv_cache_bytes([0] * 30, 20, 3, 1, 1560, 1536)
+    after = kv_cache_bytes([1] * 15 + [0] * 15, 20, 3, 1, 1560, 1536)
+    assert after == 15 * 24 * frame + 15 * 4 * frame
+    assert abs((before - after) / before - 20 / 48) < 1e-12               # half the layers: 41.7 % removed
+    # with a long history the removed share approaches the absorbed share of layers
+    long_b = kv_cache_bytes([0] * 30, 119, 3, 1, 1560, 1536)
+    long_a = kv_cache_bytes([1] * 15 + [0] * 15, 119, 3, 1, 1560, 1536)
+    assert 0.48 < (long_b - long_a) / long_b < 0.5
