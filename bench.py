@@ -56,39 +56,47 @@ def parse_args(argv=None):
                          "the batched solve alone (kernel-level timing, also the target of ncu captures)")
     ap.add_argument("--w8a8", action="store_true",
                     help="local mode: the L-layer projection through int8 weights and activations")
-    ap.add_argument("--attn-kernel", choices=["auto", "single", "pair"], default="auto",
-                    help="bf16 head_dim-128 attention kernel: one CTA per query tile, or CTA pairs "
-                         "(cta_group::2); auto = the library's default")
+    ap.add_argument("--attn-kernel", choices=["auto", "single", "pair", "two_group"], default="auto",
+                    help="bf16 head_dim-128 attention kernel: one CTA per query tile, CTA pairs "
+                         "(cta_group::2), or one CTA with two softmax groups; auto = the library's default")
     return ap.parse_args(argv)
 
 
 # DRAM bytes per fused call at the 1.3B shape (dram__bytes_read.sum + dram__bytes_write.sum,
-# one ncu capture per kernel: the split attention 276.8 MB, the statistics GEMM 50.5 MB; see
-# profiles/attn_split_sm100_1p3b_layer.md and profiles/stats_gemm_sm100_1p3b_layer.md). The
-# figure holds only for the kernel sources it was taken from: any other source reports null.
+# one ncu capture per kernel; profiles/attn_split_2g_sm100_1p3b_layer.md,
+# profiles/attn_split_sm100_1p3b_layer.md and profiles/stats_gemm_sm100_1p3b_layer.md). A figure
+# holds only for the kernel sources it was taken from: any other source reports null.
+_PTX = ("streaming_video_attention_b200/csrc/ptx.cuh",
+        "0353fca5187d1129c0e7936a8baa86b17e79672c07a933ea5a5f127e77d94af0")
 CAPTURED_TRAFFIC = {
     "workload": "1p3b_bf16",
-    "bytes_per_call": 276.8e6 + 50.5e6,
-    "sources": {
-        "streaming_video_attention_b200/csrc/attn_sm100.cu":
-            "d529641e0543692a54f49c730bd94b44bb0d8126a3e4bdeb0cd0e0acf6b451df",
-        "streaming_video_attention_b200/csrc/stats_sm100.cu":
-            "16c2ff9f411eae42daa66a16d81e6a84d3fe5185d2c3049a072bbda0027ade4d",
-        "streaming_video_attention_b200/csrc/ptx.cuh":
-            "0353fca5187d1129c0e7936a8baa86b17e79672c07a933ea5a5f127e77d94af0",
+    "stats": (50.5e6, dict([_PTX, ("streaming_video_attention_b200/csrc/stats_sm100.cu",
+                                   "16c2ff9f411eae42daa66a16d81e6a84d3fe5185d2c3049a072bbda0027ade4d")])),
+    "attention": {
+        "single": (276.8e6, dict([_PTX, ("streaming_video_attention_b200/csrc/attn_sm100.cu",
+                                         "d529641e0543692a54f49c730bd94b44bb0d8126a3e4bdeb0cd0e0acf6b451df")])),
+        "two_group": (278.8e6, dict([_PTX, ("streaming_video_attention_b200/csrc/attn2g_sm100.cu",
+                                            "e066d3338ea9828fafcb4f8ff1d06734d7d1aab058f5c35d1410770d602a7170")])),
     },
 }
 
 
 def captured_traffic(cfg, attn_kernel: str):
+    """DRAM bytes of one fused call (attention kernel + statistics GEMM), or None."""
     import hashlib
-    if cfg.name != CAPTURED_TRAFFIC["workload"] or attn_kernel == "pair":
+    kernel = "two_group" if attn_kernel == "auto" else attn_kernel
+    if cfg.name != CAPTURED_TRAFFIC["workload"] or kernel not in CAPTURED_TRAFFIC["attention"]:
         return None
-    for rel, digest in CAPTURED_TRAFFIC["sources"].items():
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest() != digest:
-                return None
-    return CAPTURED_TRAFFIC["bytes_per_call"]
+    total = 0.0
+    for nbytes, sources in (CAPTURED_TRAFFIC["attention"][kernel], CAPTURED_TRAFFIC["stats"]):
+        if nbytes is None:
+            return None
+        for rel, digest in sources.items():
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest() != digest:
+                    return None
+        total += nbytes
+    return total
 
 
 def peaks():
@@ -457,6 +465,7 @@ def ispa_arm(args, cfg, rank, world, local_rank):
     roof = {"bound": "tensor", "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
             "frac": achieved / sustained, "traffic": captured_traffic(cfg, args.attn_kernel),
             "kernel": "ispa_attn_split with fused statistics (split attention + Gram GEMM)",
+            "attn_kernel": "two_group" if args.attn_kernel == "auto" else args.attn_kernel,
             "peak_kind": f"{peak_kind} sustained bf16 (timed inside a long step)",
             "frac_of_burst_peak": achieved / burst,
             "per_call_ms": secs / max(1, len(timers)) * 1e3}
@@ -637,7 +646,8 @@ def main(argv=None):
     if args.impl != "reference":
         from streaming_video_attention_b200 import ispa
         ispa.ispa_set_attn_kernel({"auto": ispa.ISPA_ATTN_AUTO, "single": ispa.ISPA_ATTN_SINGLE,
-                                   "pair": ispa.ISPA_ATTN_PAIR}[args.attn_kernel])
+                                   "pair": ispa.ISPA_ATTN_PAIR,
+                                   "two_group": ispa.ISPA_ATTN_TWO_GROUP}[args.attn_kernel])
     if args.mode != "episode":
         return unit_arm(args, cfg)
     world = int(os.environ.get("WORLD_SIZE", "1"))

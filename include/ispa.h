@@ -231,17 +231,27 @@ int ispa_selftest_exp2_poly(const float *x, float *y, int n, ispa_stream_t strea
 
 /* ispa_set_attn_kernel -- choose the tensor-core kernel that bf16 attention calls with
  * head_dim 128 use (ispa_attn_split, ispa_attn_split_noalloc, ispa_local_attn), for this
- * process and every device. Both compute the same result:
- *   ISPA_ATTN_AUTO (0)      the faster one on sm_100a (the single-CTA kernel; on a 1.3B
- *                           layer call the pair kernel measured 1.8x slower);
- *   ISPA_ATTN_SINGLE (1)    one CTA per 128-query tile, all MMAs cta_group::1;
+ * process and every device. All compute the same result:
+ *   ISPA_ATTN_AUTO (0)      the fastest one on sm_100a: the two-group kernel (on a 1.3B
+ *                           layer call 13 % faster than the single-group one, which is
+ *                           1.8x faster than the pair kernel);
+ *   ISPA_ATTN_SINGLE (1)    one CTA per 128-query tile, one softmax group, all MMAs
+ *                           cta_group::1;
  *   ISPA_ATTN_PAIR (2)      two CTAs (a cluster of 2 on two SMs) per pair of 128-query
  *                           tiles of one head: 256-row cta_group::2 MMAs, each SM loading
- *                           half of every K/V tile.
- * head_dim 64 always uses the single-CTA kernel. Returns the previous choice, or
+ *                           half of every K/V tile;
+ *   ISPA_ATTN_TWO_GROUP (3) one CTA per 128-query tile with two softmax groups that take
+ *                           alternate KV tiles, each with its own S buffer and accumulator
+ *                           in tensor memory, merged by log-sum-exp at the end.
+ * head_dim 64 always uses the single-group kernel. Returns the previous choice, or
  * ISPA_ERR_INVALID_ARG (nothing changed) for any other value. Not synchronised with
  * launches in flight: set it before the calls it should affect. */
-typedef enum { ISPA_ATTN_AUTO = 0, ISPA_ATTN_SINGLE = 1, ISPA_ATTN_PAIR = 2 } ispa_attn_kernel;
+typedef enum {
+    ISPA_ATTN_AUTO = 0,
+    ISPA_ATTN_SINGLE = 1,
+    ISPA_ATTN_PAIR = 2,
+    ISPA_ATTN_TWO_GROUP = 3
+} ispa_attn_kernel;
 int ispa_set_attn_kernel(int choice);
 
 /* ispa_kernel_launches -- number of kernels this library has launched in this process

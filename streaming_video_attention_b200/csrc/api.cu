@@ -224,10 +224,17 @@ int run_attention(const ispa_attn_desc *d, const void *q, const void *k, const v
     cudaError_t e;
     if (d->dtype == ISPA_FP32)
         e = launch_attn_simt_f32(a, s);
-    else if (d->head_dim == 128 && g_attn_kernel.load(std::memory_order_relaxed) == ISPA_ATTN_PAIR)
-        e = launch_attn_bf16_2sm(a, s);
-    else
+    else if (d->head_dim != 128)
         e = launch_attn_bf16(a, s);
+    else {
+        const int choice = g_attn_kernel.load(std::memory_order_relaxed);
+        if (choice == ISPA_ATTN_PAIR)
+            e = launch_attn_bf16_2sm(a, s);
+        else if (choice == ISPA_ATTN_SINGLE)
+            e = launch_attn_bf16(a, s);
+        else
+            e = launch_attn_bf16_2g(a, s);   // ISPA_ATTN_AUTO, ISPA_ATTN_TWO_GROUP
+    }
     if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
     return ISPA_OK;
 }
@@ -587,7 +594,8 @@ int ispa_local_attn(const ispa_attn_desc *desc, const void *q, const void *k_loc
 }
 
 int ispa_set_attn_kernel(int choice) {
-    if (choice != ISPA_ATTN_AUTO && choice != ISPA_ATTN_SINGLE && choice != ISPA_ATTN_PAIR)
+    if (choice != ISPA_ATTN_AUTO && choice != ISPA_ATTN_SINGLE && choice != ISPA_ATTN_PAIR &&
+        choice != ISPA_ATTN_TWO_GROUP)
         return fail(ISPA_ERR_INVALID_ARG, "ispa_set_attn_kernel: unknown choice %d", choice);
     return g_attn_kernel.exchange(choice);
 }

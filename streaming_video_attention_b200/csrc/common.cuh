@@ -64,6 +64,7 @@ cudaError_t launch_attn_simt_f32(const AttnArgs &a, cudaStream_t s);
 cudaError_t launch_attn_simt_bf16(const AttnArgs &a, cudaStream_t s);
 cudaError_t launch_attn_bf16(const AttnArgs &a, cudaStream_t s);   // tcgen05 path
 cudaError_t launch_attn_bf16_2sm(const AttnArgs &a, cudaStream_t s);   // tcgen05 CTA-pair path, head_dim 128
+cudaError_t launch_attn_bf16_2g(const AttnArgs &a, cudaStream_t s);    // tcgen05, two softmax groups, head_dim 128
 
 // Batched SIMT GEMM: C_z[m][n] = alpha * sum_k A_z(m,k) B_z(k,n) + beta * C_z[m][n].
 // A_z(m,k) = A[m*lda + k] if a_kcontig else A[k*lda + m]; B_z(k,n) = B[n*ldb + k] if

@@ -236,7 +236,7 @@ def ispa_selftest_exp2_poly(x: torch.Tensor, y: torch.Tensor, stream=None) -> No
     _check(lib().ispa_selftest_exp2_poly(_p(x), _p(y), x.numel(), _stream(stream)), "ispa_selftest_exp2_poly")
 
 
-ISPA_ATTN_AUTO, ISPA_ATTN_SINGLE, ISPA_ATTN_PAIR = 0, 1, 2
+ISPA_ATTN_AUTO, ISPA_ATTN_SINGLE, ISPA_ATTN_PAIR, ISPA_ATTN_TWO_GROUP = 0, 1, 2, 3
 
 
 def ispa_set_attn_kernel(choice: int) -> int:

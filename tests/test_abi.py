@@ -88,7 +88,8 @@ def test_set_attn_kernel_choice_round_trips():
         assert ispa.ispa_set_attn_kernel(ispa.ISPA_ATTN_SINGLE) == ispa.ISPA_ATTN_PAIR
         with pytest.raises(ispa.IspaError):
             ispa.ispa_set_attn_kernel(7)
-        assert ispa.ispa_set_attn_kernel(ispa.ISPA_ATTN_AUTO) == ispa.ISPA_ATTN_SINGLE
+        assert ispa.ispa_set_attn_kernel(ispa.ISPA_ATTN_TWO_GROUP) == ispa.ISPA_ATTN_SINGLE
+        assert ispa.ispa_set_attn_kernel(ispa.ISPA_ATTN_AUTO) == ispa.ISPA_ATTN_TWO_GROUP
     finally:
         ispa.ispa_set_attn_kernel(prev)
 

@@ -1,10 +1,12 @@
-"""GPU parity of both bf16 head_dim-128 split-attention kernels (one CTA per query tile, and
-CTA pairs with cta_group::2 MMAs), each against the CPU oracle on the same seeded inputs.
+"""GPU parity of the three bf16 head_dim-128 split-attention kernels (one CTA per query tile;
+CTA pairs with cta_group::2 MMAs; one CTA with two softmax groups on alternate KV tiles), each
+against the CPU oracle on the same seeded inputs.
 
 Tolerances: as for every bf16 attention check, 2e-2 relative Frobenius per output tensor and
 2e-2 absolute on lse; the fused statistics 2e-2 relative. The two kernels against each other
-on a full 1.3B-shaped layer: 1e-2 relative (both round P and the outputs to bf16; they
-differ only in accumulation order inside the MMAs).
+on a full 1.3B-shaped layer: 1e-2 relative (all round P and the outputs to bf16; they differ
+in accumulation order, and the two-group kernel also rounds each group's normalised local part
+to bf16 before merging them).
 """
 import math
 
@@ -20,7 +22,7 @@ from tests.test_gpu_parity import _attn_case, _check_attn, _run_split
 
 pytestmark = pytest.mark.gpu
 
-KERNELS = {"single": ispa.ISPA_ATTN_SINGLE, "pair": ispa.ISPA_ATTN_PAIR}
+KERNELS = {"single": ispa.ISPA_ATTN_SINGLE, "pair": ispa.ISPA_ATTN_PAIR, "two_group": ispa.ISPA_ATTN_TWO_GROUP}
 
 
 @pytest.fixture(params=sorted(KERNELS))
@@ -54,6 +56,8 @@ def test_kernel_matches_oracle(attn_kernel, layout):
     (129, 129, (0, 64), (65, 129)),      # a 1-row query tail; a 1-row KV tail
     (256, 700, (0, 0), (300, 700)),      # exactly one tile pair; no sink
     (5, 3, (0, 1), (1, 3)),              # fewer keys than anything
+    (128, 300, (0, 0), (200, 300)),      # one local tile, then history: the odd group hands over first
+    (200, 1000, (0, 64), (900, 1000)),   # two local tiles; the history tiles alternate between groups
 ])
 def test_kernel_edge_sizes(attn_kernel, n_q, n_kv, sink, chunk):
     q, k, v = _attn_case(77, n_q, n_kv, 2, 128, "bf16")
@@ -78,7 +82,7 @@ def test_kernel_fused_stats(attn_kernel):
 
 
 def test_kernels_agree_on_full_1p3b_layer():
-    """Both kernels on one 1.3B-shaped layer call (n_q 4680, n_kv 37440, 12 heads): every
+    """Every kernel against the single-CTA one on a 1.3B-shaped layer call (n_q 4680, n_kv 37440, 12 heads): every
     output element, not a sample."""
     cfg = synth.CONFIGS["1p3b_bf16"]
     t, layer = cfg.warmup_chunks - 1, 5
@@ -95,12 +99,13 @@ def test_kernels_agree_on_full_1p3b_layer():
             res[name] = _run_split(q, k, v, sink, chunk, "bf16")
         finally:
             ispa.ispa_set_attn_kernel(prev)
-    for key in res["single"]:
-        a, b = res["single"][key], res["pair"][key]
-        if key.startswith("A_"):
-            assert rel_fro(b, a) < 1e-2, key
-        else:
-            assert np.array_equal(np.isfinite(a), np.isfinite(b)), key
-            fin = np.isfinite(a)
-            assert np.max(np.abs(a[fin] - b[fin])) < 1e-2, key
+    for other in sorted(set(KERNELS) - {"single"}):
+        for key in res["single"]:
+            a, b = res["single"][key], res[other][key]
+            if key.startswith("A_"):
+                assert rel_fro(b, a) < 1e-2, (other, key)
+            else:
+                assert np.array_equal(np.isfinite(a), np.isfinite(b)), (other, key)
+                fin = np.isfinite(a)
+                assert np.max(np.abs(a[fin] - b[fin])) < 1e-2, (other, key)
 
