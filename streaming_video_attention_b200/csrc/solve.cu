@@ -3,7 +3,12 @@
 //
 //   M = G + lambda I                          fill_shifted
 //   M = L L^T (blocked, right-looking)        potrf_diag + trsm_panel + GEMM trailing update
-//   dW = L^-T L^-1 (C W)                      GEMM, then trsv_block + GEMM per block, both ways
+//   dW = L^-T L^-1 (C W)                      with D a multiple of 128: X = L^-1 by blocked
+//                                             forward substitution on the identity (the
+//                                             updates skip X's zero upper part), then
+//                                             Z = X (C W) and dW = X^T Z on the tensor
+//                                             cores (3xTF32); otherwise trsv_block + GEMM
+//                                             per block, both ways, on (C W) itself
 //   five traces -> E^2, T^2, eps              GEMMs G dW, H W, G W, then dot_partials
 //
 // Block size nb = 64 (D must be a multiple of 64). The diagonal blocks are factored and
@@ -186,6 +191,14 @@ __global__ void add_delta_kernel(PtrBatch W, PtrBatch dW, PtrBatch out, size_t n
         oz[i] = from_f32<TW>(to_f32(Wz[i]) + dz[i]);
 }
 
+__global__ void fill_identity_kernel(PtrBatch dst, int D) {
+    const int z = blockIdx.y;
+    float *d = static_cast<float *>(dst.p[z]);
+    const size_t n = (size_t)D * D;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        d[i] = (i / D == i % D) ? 1.f : 0.f;
+}
+
 __global__ void copy_f32_kernel(PtrBatch src, PtrBatch dst, size_t n) {
     const int z = blockIdx.y;
     const float4 *s = static_cast<const float4 *>(src.p[z]);
@@ -302,8 +315,10 @@ cudaError_t error_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
 }
 
 // Solve for one batch of layers. All pointers are device pointers, one per layer.
-//   G, C, H: statistics; W: weights of type wt; dW: output; M, Y: D*D float scratch each;
-//   P: D*D float scratch; terms: 5 * batch * nparts doubles; status: batch ints (zeroed).
+//   G, C, H: statistics; W: weights of type wt; dW: output (the batch's matrices contiguous,
+//   dW.p[z] = dW.p[0] + z*D*D); M, Y: D*D float scratch each; P: D*D float scratch; Yc, Pc:
+//   the Y and P blocks as contiguous batches; terms: 5 * batch * nparts doubles; status:
+//   batch ints (zeroed).
 cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H, const PtrBatch &W, ElemType wt,
                         const PtrBatch &dW, const PtrBatch &M, const PtrBatch &Y, const PtrBatch &P, float *Yc,
                         float *Pc, float *split, double *terms, int nparts, int *status, float *eps,
@@ -319,10 +334,8 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
     fill_shifted_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(G, M, D, lambda); note_launch();
     ISPA_TRY(cudaGetLastError());
 
-    // Y = C W, and dW <- Y (solved in place below)
+    // Y = C W
     ISPA_TRY(c_times_w(C, W, wt, Y, Yc, split, D, batch, err_flag, tc, s));
-    copy_f32_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(Y, dW, n); note_launch();
-    ISPA_TRY(cudaGetLastError());
 
     // Cholesky factorisation, blocked
     const int nblk = D / NB;
@@ -341,30 +354,61 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
         ISPA_TRY(launch_gemm_simt(d, make_gemm_batch(M, offA, M, offA, M, offC, batch, 4, 4), s));
     }
 
-    // Forward substitution L Z = Y (in dW)
-    const dim3 tgrid((D + 127) / 128, batch);
-    for (int kb = 0; kb < nblk; ++kb) {
-        const int k0 = kb * NB;
-        trsv_block_kernel<false><<<tgrid, 128, 0, s>>>(M, dW, D, k0); note_launch();
+    if (tc) {
+        // X = L^-1 in P: forward substitution L X = I. Block row k of X is nonzero only in its
+        // first k0 + NB columns, so the diagonal solve and the update below stop there.
+        fill_identity_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(P, D); note_launch();
         ISPA_TRY(cudaGetLastError());
-        const int rest = D - k0 - NB;
-        if (rest <= 0) break;
-        GemmDesc d{rest, D, NB, D, D, D, true, false, ElemType::F32, ElemType::F32, ElemType::F32, -1.f, 1.f,
-                   false, batch};
-        ISPA_TRY(launch_gemm_simt(
-            d, make_gemm_batch(M, (size_t)(k0 + NB) * D + k0, dW, (size_t)k0 * D, dW, (size_t)(k0 + NB) * D, batch, 4, 4),
-            s));
-    }
-    // Backward substitution L^T X = Z
-    for (int kb = nblk - 1; kb >= 0; --kb) {
-        const int k0 = kb * NB;
-        trsv_block_kernel<true><<<tgrid, 128, 0, s>>>(M, dW, D, k0); note_launch();
+        for (int kb = 0; kb < nblk; ++kb) {
+            const int k0 = kb * NB;
+            const int cols = k0 + NB;
+            trsv_block_kernel<false><<<dim3((cols + 127) / 128, batch), 128, 0, s>>>(M, P, D, k0); note_launch();
+            ISPA_TRY(cudaGetLastError());
+            const int rest = D - k0 - NB;
+            if (rest <= 0) break;
+            GemmDesc d{rest, cols, NB, D, D, D, true, false, ElemType::F32, ElemType::F32, ElemType::F32, -1.f, 1.f,
+                       false, batch};
+            ISPA_TRY(launch_gemm_simt(
+                d, make_gemm_batch(M, (size_t)(k0 + NB) * D + k0, P, (size_t)k0 * D, P, (size_t)(k0 + NB) * D, batch, 4, 4),
+                s));
+        }
+        // Z = X Y into dW, then dW = X^T Z (3xTF32; B operands are split transposed)
+        const size_t bn = (size_t)batch * n;
+        float *Ahi = split, *Alo = split + bn, *Bhi = split + 2 * bn, *Blo = split + 3 * bn;
+        float *dWc = static_cast<float *>(dW.p[0]);
+        ISPA_TRY(launch_split_tf32(P, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
+        ISPA_TRY(launch_split_tf32(Y, ElemType::F32, Bhi, Blo, D, D, true, batch, s));
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Bhi, Blo, dWc, D, D, D, batch, err_flag, s));
+        ISPA_TRY(launch_split_tf32(P, ElemType::F32, Ahi, Alo, D, D, true, batch, s));
+        ISPA_TRY(launch_split_tf32(dW, ElemType::F32, Bhi, Blo, D, D, true, batch, s));
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Bhi, Blo, dWc, D, D, D, batch, err_flag, s));
+    } else {
+        // dW <- Y, solved in place: forward substitution L Z = Y, then backward L^T X = Z
+        copy_f32_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(Y, dW, n); note_launch();
         ISPA_TRY(cudaGetLastError());
-        if (k0 == 0) break;
-        // X[0:k0, :] -= (L[k0:k0+NB, 0:k0])^T X_k
-        GemmDesc d{k0, D, NB, D, D, D, false, false, ElemType::F32, ElemType::F32, ElemType::F32, -1.f, 1.f, false,
-                   batch};
-        ISPA_TRY(launch_gemm_simt(d, make_gemm_batch(M, (size_t)k0 * D, dW, (size_t)k0 * D, dW, 0, batch, 4, 4), s));
+        const dim3 tgrid((D + 127) / 128, batch);
+        for (int kb = 0; kb < nblk; ++kb) {
+            const int k0 = kb * NB;
+            trsv_block_kernel<false><<<tgrid, 128, 0, s>>>(M, dW, D, k0); note_launch();
+            ISPA_TRY(cudaGetLastError());
+            const int rest = D - k0 - NB;
+            if (rest <= 0) break;
+            GemmDesc d{rest, D, NB, D, D, D, true, false, ElemType::F32, ElemType::F32, ElemType::F32, -1.f, 1.f,
+                       false, batch};
+            ISPA_TRY(launch_gemm_simt(
+                d, make_gemm_batch(M, (size_t)(k0 + NB) * D + k0, dW, (size_t)k0 * D, dW, (size_t)(k0 + NB) * D, batch, 4, 4),
+                s));
+        }
+        for (int kb = nblk - 1; kb >= 0; --kb) {
+            const int k0 = kb * NB;
+            trsv_block_kernel<true><<<tgrid, 128, 0, s>>>(M, dW, D, k0); note_launch();
+            ISPA_TRY(cudaGetLastError());
+            if (k0 == 0) break;
+            // X[0:k0, :] -= (L[k0:k0+NB, 0:k0])^T X_k
+            GemmDesc d{k0, D, NB, D, D, D, false, false, ElemType::F32, ElemType::F32, ElemType::F32, -1.f, 1.f, false,
+                       batch};
+            ISPA_TRY(launch_gemm_simt(d, make_gemm_batch(M, (size_t)k0 * D, dW, (size_t)k0 * D, dW, 0, batch, 4, 4), s));
+        }
     }
 
     // Reconstruction error terms
