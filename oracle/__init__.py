@@ -22,4 +22,8 @@ from .ispa_oracle import (  # noqa: F401
     rewarm_trigger,
     quantize_int8,
     project_w8a8,
+    kv_blocks,
+    quantize_i8_q,
+    quantize_i8_k,
+    split_attention_i8,
 )

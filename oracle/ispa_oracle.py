@@ -244,6 +244,79 @@ def project_w8a8(A: np.ndarray, W: np.ndarray) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------------------
+# 8-bit split attention [ISPA §3.4: the decomposition is built on 8-bit attention kernels
+# (SageAttention, SageAttention2), whose scheme the pages do not give]. Reading: as in
+# SageAttention, S = scale * Q K^T is taken from int8 copies of Q and K, everything after
+# it (softmax, P, P V, the partition merge, the statistics operands) exactly as in the bf16
+# path. Q is quantised per (token, head); K per (block, head), a block being 128 rows of
+# one partition segment (the sink range, the chunk range and the history runs around them,
+# each cut into blocks from its first row; the last block of a segment is shorter). Each
+# scale is symmetric, as in quantize_int8: amax / 127, with q = rint(x * (127 / amax)) in
+# float32 (ties to even), clamped to +-127. Then S_ij = scale * s_q,i * s_k,b(j) * (q8_i . k8_j),
+# the dot product exact in integers. No smoothing of K: the softmax ignores a per-row
+# shift, but the log-sum-exp output would have to be corrected for it.
+# --------------------------------------------------------------------------------------
+def kv_blocks(n_kv: int, sink: Tuple[int, int], chunk: Tuple[int, int], rows: int = 128) -> List[Tuple[int, int]]:
+    """(begin, end) of the K quantisation blocks, in row order."""
+    loc = sorted(r for r in (tuple(sink), tuple(chunk)) if r[1] > r[0])
+    segs = list(loc)
+    cur = 0
+    for b, e in loc:
+        if b > cur:
+            segs.append((cur, b))
+        cur = max(cur, e)
+    if cur < n_kv:
+        segs.append((cur, n_kv))
+    blocks = []
+    for b, e in sorted(segs):
+        blocks += [(r, min(r + rows, e)) for r in range(b, e, rows)]
+    return blocks
+
+
+def _i8_symmetric(x: np.ndarray, amax: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    amax = np.asarray(amax, dtype=np.float32)
+    inv = np.zeros_like(amax)
+    nz = amax > 0
+    inv[nz] = np.float32(127.0) / amax[nz]
+    q = np.clip(np.rint(x * inv), -127, 127).astype(np.int8)
+    return q, (amax / np.float32(127.0)).astype(np.float32)
+
+
+def quantize_i8_q(q: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Q [n, h, d] -> (q8 [n, h, d] int8, s_q [h, n] float32)."""
+    x = np.asarray(q, dtype=np.float32)
+    q8, sc = _i8_symmetric(x, np.max(np.abs(x), axis=2, keepdims=True) if x.size else np.zeros(x.shape[:2] + (1,)))
+    return q8, np.ascontiguousarray(sc[:, :, 0].T)
+
+
+def quantize_i8_k(k: np.ndarray, blocks: Sequence[Tuple[int, int]]) -> Tuple[np.ndarray, np.ndarray]:
+    """K [n, h, d] -> (k8 [n, h, d] int8, s_k [h, n_blocks] float32), blocks from kv_blocks."""
+    x = np.asarray(k, dtype=np.float32)
+    n, h, d = x.shape
+    k8 = np.zeros((n, h, d), dtype=np.int8)
+    sk = np.zeros((h, len(blocks)), dtype=np.float32)
+    for i, (b, e) in enumerate(blocks):
+        amax = np.max(np.abs(x[b:e]), axis=(0, 2)).reshape(1, h, 1)
+        k8[b:e], sc = _i8_symmetric(x[b:e], amax)
+        sk[:, i] = sc[0, :, 0]
+    return k8, sk
+
+
+def split_attention_i8(q, k, v, sink: Tuple[int, int], chunk: Tuple[int, int], scale: float) -> Dict[str, np.ndarray]:
+    """split_attention with S taken from the int8 copies: S = scale * s_q s_k (q8 . k8)."""
+    blocks = kv_blocks(k.shape[0], sink, chunk)
+    q8, sq = quantize_i8_q(q)
+    k8, sk = quantize_i8_k(k, blocks)
+    q_deq = q8.astype(np.float64) * sq.T.astype(np.float64)[:, :, None]
+    k_deq = np.zeros(k8.shape, dtype=np.float64)
+    for i, (b, e) in enumerate(blocks):
+        k_deq[b:e] = k8[b:e].astype(np.float64) * sk[:, i].astype(np.float64)[None, :, None]
+    out = split_attention(q_deq, k_deq, v, sink, chunk, scale)
+    out.update(q8=q8, q_scale=sq, k8=k8, k_scale=sk, blocks=blocks)
+    return out
+
+
+# --------------------------------------------------------------------------------------
 # A whole streaming run, chunk by chunk [ISPA §3.1, §3.3 re-triggered warmup].
 # --------------------------------------------------------------------------------------
 def live_error(A_loc, A_full, dtype: str, W, dW) -> float:

@@ -412,3 +412,71 @@ def test_w8a8_scale_invariances_and_error_bound():
 
 def synth_bf16(x):
     return oracle.bf16_round(np.asarray(x, np.float64)).astype(np.float32)
+
+
+# ------------------------------------------------------------------ 8-bit (int8) split attention
+def test_kv_blocks_cover_the_rows_once_and_respect_partitions():
+    for n_kv, sink, chunk in [(1000, (0, 64), (900, 1000)), (300, (0, 0), (200, 300)), (640, (0, 130), (130, 640)),
+                              (5, (0, 1), (1, 3)), (37440, (0, 1560), (32760, 37440))]:
+        blocks = oracle.kv_blocks(n_kv, sink, chunk)
+        rows = np.concatenate([np.arange(b, e) for b, e in blocks])
+        assert np.array_equal(rows, np.arange(n_kv))                     # in order, each row once
+        assert all(0 < e - b <= 128 for b, e in blocks)
+        _, local, _ = oracle.partition_masks(n_kv, sink, chunk)
+        for b, e in blocks:
+            assert local[b:e].all() or not local[b:e].any()               # one partition per block
+            in_sink = (sink[0] <= b < sink[1]) == (sink[0] <= e - 1 < sink[1])
+            assert in_sink                                                # never across the sink edge
+    assert oracle.kv_blocks(300, (0, 0), (200, 300)) == [(0, 128), (128, 200), (200, 300)]
+    assert oracle.kv_blocks(1000, (0, 64), (900, 1000))[:3] == [(0, 64), (64, 192), (192, 320)]
+
+
+def test_i8_quantizers_hand_cases_and_bounds():
+    q = np.zeros((2, 1, 4), np.float32)
+    q[0, 0] = [1.0, -2.0, 0.5, 0.25]
+    q8, sq = oracle.quantize_i8_q(q)
+    assert q8[0, 0].tolist() == [64, -127, 32, 16] and q8[1, 0].tolist() == [0, 0, 0, 0]   # 63.5 -> 64 (even)
+    assert sq.shape == (1, 2) and sq[0, 0] == np.float32(2.0) / np.float32(127.0) and sq[0, 1] == 0.0
+    rng = np.random.default_rng(9)
+    k = synth_bf16(rng.standard_normal((300, 3, 64)) * np.exp(rng.normal(0, 1, (300, 1, 1))))
+    blocks = oracle.kv_blocks(300, (0, 40), (200, 300))
+    k8, sk = oracle.quantize_i8_k(k, blocks)
+    assert sk.shape == (3, len(blocks))
+    for i, (b, e) in enumerate(blocks):
+        amax = np.abs(k[b:e]).max(axis=(0, 2))
+        assert np.all(sk[:, i] == (amax / np.float32(127.0)).astype(np.float32))
+        assert np.all(np.abs(k8[b:e]).max(axis=(0, 2)) == 127)        # the largest element maps to 127
+        err = np.abs(k8[b:e].astype(np.float64) * sk[:, i][None, :, None] - k[b:e])
+        assert np.all(err <= 0.5 * sk[:, i][None, :, None] * (1 + 1e-5))
+
+
+def test_i8_attention_reduces_to_the_exact_one_on_the_grid():
+    """Integer inputs whose per-row (Q) and per-block (K) maxima are 127 quantise to themselves
+    with scale 1: the 8-bit split attention then equals the plain one exactly."""
+    rng = np.random.default_rng(10)
+    n_q, n_kv, h, d = 9, 300, 2, 32
+    q = rng.integers(-126, 127, (n_q, h, d)).astype(np.float64)
+    k = rng.integers(-126, 127, (n_kv, h, d)).astype(np.float64)
+    q[:, :, 0] = 127.0
+    for b, e in oracle.kv_blocks(n_kv, (0, 5), (200, 300)):
+        k[b, :, 0] = -127.0
+    v = synth_bf16(rng.standard_normal((n_kv, h, d)))
+    scale = 1.0 / (127.0 * 127.0 * d)
+    got = oracle.split_attention_i8(q, k, v, (0, 5), (200, 300), scale)
+    want = oracle.split_attention(q, k, v, (0, 5), (200, 300), scale)
+    assert np.all(got["q_scale"] == 1.0) and np.all(got["k_scale"] == 1.0)
+    for key in ("A_full", "A_loc", "A_hist", "lse_full", "lse_loc", "lse_hist"):
+        assert np.array_equal(got[key], want[key]), key
+
+
+def test_i8_attention_error_against_unquantised():
+    """On N(0,1) inputs with the 1/sqrt(d) scale the int8 scores move the outputs by about
+    1 %: the bound here is the 2e-2 used for bf16 attention."""
+    rng = np.random.default_rng(11)
+    n_q, n_kv, h, d = 64, 300, 2, 128
+    q, k, v = (synth_bf16(rng.standard_normal((n, h, d))) for n in (n_q, n_kv, n_kv))
+    got = oracle.split_attention_i8(q, k, v, (0, 40), (200, 300), 1 / math.sqrt(d))
+    want = oracle.split_attention(q, k, v, (0, 40), (200, 300), 1 / math.sqrt(d))
+    for key in ("A_full", "A_loc", "A_hist"):
+        rel = np.linalg.norm(got[key] - want[key]) / np.linalg.norm(want[key])
+        assert rel < 2e-2, (key, rel)
