@@ -54,6 +54,8 @@ def parse_args(argv=None):
                     help="episode: the full step (default). call / local / solve: one layer's fused split "
                          "attention at the last warmup chunk, one L-layer local attention with projection, or "
                          "the batched solve alone (kernel-level timing, also the target of ncu captures)")
+    ap.add_argument("--i8", action="store_true",
+                    help="call mode: the 8-bit split attention (int8 Q and K, quantised inside the timed call)")
     ap.add_argument("--w8a8", action="store_true",
                     help="local mode: the L-layer projection through int8 weights and activations")
     ap.add_argument("--attn-kernel", choices=["auto", "single", "pair", "two_group"], default="auto",
@@ -75,8 +77,8 @@ CAPTURED_TRAFFIC = {
     "attention": {
         "single": (276.8e6, dict([_PTX, ("streaming_video_attention_b200/csrc/attn_sm100.cu",
                                          "d529641e0543692a54f49c730bd94b44bb0d8126a3e4bdeb0cd0e0acf6b451df")])),
-        "two_group": (278.8e6, dict([_PTX, ("streaming_video_attention_b200/csrc/attn2g_sm100.cu",
-                                            "e066d3338ea9828fafcb4f8ff1d06734d7d1aab058f5c35d1410770d602a7170")])),
+        "two_group": (281.2e6, dict([_PTX, ("streaming_video_attention_b200/csrc/attn2g_sm100.cu",
+                                            "3bed3806f2e152d01cb932a529d3f79da812540a4b19e6fbb52febc93f129433")])),
     },
 }
 
@@ -594,6 +596,24 @@ def unit_arm(args, cfg):
             fn = lambda: sess.full_attention(0, q, k, v, sink, chunk, o, lse, collect=True)
             flops = 4.0 * cfg.n_q * n_kv * cfg.head_dim * cfg.heads + 4.0 * cfg.n_q * D * D
             what = f"fused split attention + statistics, one layer, n_q {cfg.n_q}, n_kv {n_kv}"
+            if args.i8:
+                desc = ispa.make_desc(cfg.n_q, n_kv, cfg.heads, cfg.head_dim, sink, chunk)
+                q8 = torch.empty(q.shape, dtype=torch.int8, device=device)
+                k8 = torch.empty(k.shape, dtype=torch.int8, device=device)
+                qs = torch.empty((cfg.n_q, cfg.heads), dtype=torch.float32, device=device)
+                ks = torch.empty((cfg.heads, ispa.ispa_k_blocks(desc)), dtype=torch.float32, device=device)
+                ws = ispa.alloc_workspace(ispa.workspace_bytes(desc, 0, 0))
+                st = sess.stats[0]
+
+                def attn_only():
+                    ispa.ispa_attn_split_i8(desc, q8, qs, k8, ks, v, o, lse, stats=st, ws=ws)
+
+                def fn():
+                    ispa.ispa_quantize_q_i8(q, q8, qs)
+                    ispa.ispa_quantize_k_i8(desc, k, k8, ks)
+                    attn_only()
+                what = ("8-bit split attention (int8 Q/K quantised in the call) + statistics, one layer, "
+                        f"n_q {cfg.n_q}, n_kv {n_kv}")
         else:
             sess.is_local = [1]
             if args.w8a8:
@@ -634,9 +654,22 @@ def unit_arm(args, cfg):
     burst, sustained, hbm, kind = peaks()
     dt = statistics.median(times)
     tf = flops / dt / 1e12
+    extra = {}
+    if args.mode == "call" and args.i8:
+        # the same call without the two quantisers (int8 Q/K already resident)
+        t2 = []
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            attn_only()
+            e1.record()
+            torch.cuda.synchronize()
+            t2.append(e0.elapsed_time(e1))
+        extra = {"ms_without_quantisation": statistics.median(t2)}
     print(json.dumps({"mode": args.mode, "what": what, "ms": dt * 1e3, "ms_all": [x * 1e3 for x in times],
                       "tflops": tf, "frac_of_burst_peak": tf / burst, "peak_kind": kind,
-                      "query_tokens_per_s": cfg.n_q / dt if args.mode != "solve" else None}), flush=True)
+                      "query_tokens_per_s": cfg.n_q / dt if args.mode != "solve" else None} | extra), flush=True)
     return 0
 
 

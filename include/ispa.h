@@ -100,6 +100,35 @@ int ispa_attn_split(const ispa_attn_desc *desc, const void *q, const void *k, co
                     float *lse_hist, const ispa_stats *stats, void *ws, size_t ws_bytes,
                     ispa_stream_t stream);
 
+/* 8-bit split attention [ISPA §3.4: the decomposition is built on 8-bit attention kernels,
+ * SageAttention]: ispa_attn_split with S = scale * Q K^T taken from int8 copies of Q and K;
+ * V, P, P V, the merge, the outputs and the fused statistics as in ispa_attn_split.
+ * Quantisation (symmetric, float32, ties to even): s = amax / 127 and
+ * x8 = clamp(rint(x * (127 / amax)), -127, 127), x8 = 0 and s = 0 where amax = 0; then
+ * S_ij = scale * q_scale[i] * k_scale[block(j)] * (q8_i . k8_j), the dot product exact in int32.
+ *
+ * ispa_quantize_q_i8 -- q [n, heads, 128] bf16 -> q8 (same layout, int8), q_scale [n, heads]
+ *   float32: one scale per (token, head). Device pointers; q, q8 16-byte aligned.
+ * ispa_k_blocks -- number of K blocks of desc's layout (the size of a k_scale row): the KV
+ *   rows cut at the partition boundaries into segments (the sink range, the chunk range and
+ *   the history runs around them), each segment into blocks of 128 rows from its first row;
+ *   blocks are numbered in row order. Returns the count (>= 0) or an error code.
+ * ispa_quantize_k_i8 -- k [n_kv, heads, 128] bf16 -> k8 (same layout, int8), k_scale
+ *   [heads, ispa_k_blocks(desc)] float32: one scale per (block, head).
+ * ispa_attn_split_i8 -- as ispa_attn_split, with q8/q_scale and k8/k_scale from the two
+ *   quantisers (k8 for the same desc) and v bf16. desc->dtype must be ISPA_BF16 and
+ *   head_dim 128 (otherwise ISPA_ERR_UNSUPPORTED); the outputs are bf16. Workspace as for
+ *   ispa_attn_split. */
+int ispa_quantize_q_i8(const void *q, int n, int heads, int head_dim, signed char *q8, float *q_scale,
+                       ispa_stream_t stream);
+int ispa_k_blocks(const ispa_attn_desc *desc);
+int ispa_quantize_k_i8(const ispa_attn_desc *desc, const void *k, signed char *k8, float *k_scale,
+                       ispa_stream_t stream);
+int ispa_attn_split_i8(const ispa_attn_desc *desc, const signed char *q8, const float *q_scale,
+                       const signed char *k8, const float *k_scale, const void *v, void *o_full, float *lse_full,
+                       void *o_loc, float *lse_loc, void *o_hist, float *lse_hist, const ispa_stats *stats,
+                       void *ws, size_t ws_bytes, ispa_stream_t stream);
+
 /* ispa_attn_split_noalloc -- ispa_attn_split with fused statistics for callers that cannot
  * allocate device memory (for example code running inside a host framework that owns all
  * device memory and passes only its inputs and outputs, or a plugin interface without a

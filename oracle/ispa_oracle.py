@@ -283,10 +283,10 @@ def _i8_symmetric(x: np.ndarray, amax: np.ndarray) -> Tuple[np.ndarray, np.ndarr
 
 
 def quantize_i8_q(q: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
-    """Q [n, h, d] -> (q8 [n, h, d] int8, s_q [h, n] float32)."""
+    """Q [n, h, d] -> (q8 [n, h, d] int8, s_q [n, h] float32)."""
     x = np.asarray(q, dtype=np.float32)
     q8, sc = _i8_symmetric(x, np.max(np.abs(x), axis=2, keepdims=True) if x.size else np.zeros(x.shape[:2] + (1,)))
-    return q8, np.ascontiguousarray(sc[:, :, 0].T)
+    return q8, np.ascontiguousarray(sc[:, :, 0])
 
 
 def quantize_i8_k(k: np.ndarray, blocks: Sequence[Tuple[int, int]]) -> Tuple[np.ndarray, np.ndarray]:
@@ -307,7 +307,7 @@ def split_attention_i8(q, k, v, sink: Tuple[int, int], chunk: Tuple[int, int], s
     blocks = kv_blocks(k.shape[0], sink, chunk)
     q8, sq = quantize_i8_q(q)
     k8, sk = quantize_i8_k(k, blocks)
-    q_deq = q8.astype(np.float64) * sq.T.astype(np.float64)[:, :, None]
+    q_deq = q8.astype(np.float64) * sq.astype(np.float64)[:, :, None]
     k_deq = np.zeros(k8.shape, dtype=np.float64)
     for i, (b, e) in enumerate(blocks):
         k_deq[b:e] = k8[b:e].astype(np.float64) * sk[:, i].astype(np.float64)[None, :, None]

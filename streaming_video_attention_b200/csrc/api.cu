@@ -205,9 +205,10 @@ int check_ws(void *ws, size_t have, size_t need) {
 // Kernel used by bf16 head_dim-128 attention (ispa_set_attn_kernel).
 std::atomic<int> g_attn_kernel{ISPA_ATTN_AUTO};
 
+// q_scale / k_scale non-null: q and k are int8 (the 8-bit split attention).
 int run_attention(const ispa_attn_desc *d, const void *q, const void *k, const void *v, void *o_full, float *lse_full,
                   void *o_loc, float *lse_loc, void *o_hist, float *lse_hist, void *a_ops, void *r_ops,
-                  bool local_only, cudaStream_t s) {
+                  bool local_only, cudaStream_t s, const float *q_scale = nullptr, const float *k_scale = nullptr) {
     int *flag = nullptr;
     int rc = device_error_flag(&flag);
     if (rc != ISPA_OK) return rc;
@@ -222,7 +223,9 @@ int run_attention(const ispa_attn_desc *d, const void *q, const void *k, const v
     a.segs = make_segments(d, local_only);
     a.err_flag = flag;
     cudaError_t e;
-    if (d->dtype == ISPA_FP32)
+    if (q_scale)
+        e = launch_attn_i8_2g(a, q_scale, k_scale, s);
+    else if (d->dtype == ISPA_FP32)
         e = launch_attn_simt_f32(a, s);
     else if (d->head_dim != 128)
         e = launch_attn_bf16(a, s);
@@ -303,12 +306,11 @@ size_t ispa_workspace_bytes(const ispa_attn_desc *desc, int n, int D) {
     return need;
 }
 
-int ispa_attn_split(const ispa_attn_desc *desc, const void *q, const void *k, const void *v, void *o_full,
-                    float *lse_full, void *o_loc, float *lse_loc, void *o_hist, float *lse_hist,
-                    const ispa_stats *stats, void *ws, size_t ws_bytes, ispa_stream_t stream) {
-    g_last_error.clear();
-    int rc = check_desc(desc, true);
-    if (rc != ISPA_OK) return rc;
+static int attn_split_impl(const ispa_attn_desc *desc, const void *q, const void *k, const void *v, void *o_full,
+                           float *lse_full, void *o_loc, float *lse_loc, void *o_hist, float *lse_hist,
+                           const ispa_stats *stats, void *ws, size_t ws_bytes, ispa_stream_t stream,
+                           const float *q_scale, const float *k_scale) {
+    int rc;
     if (desc->n_q > 0 && (!q || !o_full || !lse_full)) return fail(ISPA_ERR_INVALID_ARG, "q, o_full and lse_full are required");
     if (desc->n_kv > 0 && (!k || !v)) return fail(ISPA_ERR_INVALID_ARG, "k and v are required");
     for (const void *p : {q, k, v, (const void *)o_full, (const void *)o_loc, (const void *)o_hist})
@@ -325,7 +327,8 @@ int ispa_attn_split(const ispa_attn_desc *desc, const void *q, const void *k, co
         r_ops = static_cast<char *>(ws) + align_up((size_t)desc->n_q * D * elem_size(desc->dtype), 256);
     }
     if (desc->n_q > 0) {
-        rc = run_attention(desc, q, k, v, o_full, lse_full, o_loc, lse_loc, o_hist, lse_hist, a_ops, r_ops, false, s);
+        rc = run_attention(desc, q, k, v, o_full, lse_full, o_loc, lse_loc, o_hist, lse_hist, a_ops, r_ops, false, s,
+                           q_scale, k_scale);
         if (rc != ISPA_OK) return rc;
     }
     if (stats) {
@@ -335,6 +338,87 @@ int ispa_attn_split(const ispa_attn_desc *desc, const void *q, const void *k, co
         return accumulate(stats, a_ops, r_ops, desc->n_q, desc->dtype, flag, s);
     }
     return ISPA_OK;
+}
+
+int ispa_attn_split(const ispa_attn_desc *desc, const void *q, const void *k, const void *v, void *o_full,
+                    float *lse_full, void *o_loc, float *lse_loc, void *o_hist, float *lse_hist,
+                    const ispa_stats *stats, void *ws, size_t ws_bytes, ispa_stream_t stream) {
+    g_last_error.clear();
+    int rc = check_desc(desc, true);
+    if (rc != ISPA_OK) return rc;
+    return attn_split_impl(desc, q, k, v, o_full, lse_full, o_loc, lse_loc, o_hist, lse_hist, stats, ws, ws_bytes,
+                           stream, nullptr, nullptr);
+}
+
+// K blocks of the 8-bit split attention: the KV segments in row order, each cut into
+// blocks of 128 rows from its first row.
+static SegmentList row_order_segments(const ispa_attn_desc *d) {
+    SegmentList L = make_segments(d, false);
+    std::sort(L.seg, L.seg + L.count, [](const Segment &a, const Segment &b) { return a.begin < b.begin; });
+    return L;
+}
+
+static int count_k_blocks(const ispa_attn_desc *d) {
+    const SegmentList L = row_order_segments(d);
+    int n = 0;
+    for (int i = 0; i < L.count; ++i) n += (L.seg[i].end - L.seg[i].begin + 127) / 128;
+    return n;
+}
+
+static int check_i8_desc(const ispa_attn_desc *desc) {
+    int rc = check_desc(desc, true);
+    if (rc != ISPA_OK) return rc;
+    if (desc->dtype != ISPA_BF16 || desc->head_dim != 128)
+        return fail(ISPA_ERR_UNSUPPORTED, "8-bit split attention: bf16 V and outputs, head_dim 128 only");
+    return ISPA_OK;
+}
+
+int ispa_k_blocks(const ispa_attn_desc *desc) {
+    g_last_error.clear();
+    int rc = check_desc(desc, true);
+    if (rc != ISPA_OK) return rc;
+    return count_k_blocks(desc);
+}
+
+int ispa_quantize_q_i8(const void *q, int n, int heads, int head_dim, signed char *q8, float *q_scale,
+                       ispa_stream_t stream) {
+    g_last_error.clear();
+    if (n < 0 || heads <= 0) return fail(ISPA_ERR_INVALID_ARG, "bad sizes n=%d heads=%d", n, heads);
+    if (head_dim != 128) return fail(ISPA_ERR_UNSUPPORTED, "head_dim %d (supported: 128)", head_dim);
+    if (n == 0) return ISPA_OK;
+    if (!q || !q8 || !q_scale) return fail(ISPA_ERR_INVALID_ARG, "q, q8 and q_scale are required");
+    if (!aligned(q, 16) || !aligned(q8, 16)) return fail(ISPA_ERR_INVALID_ARG, "q and q8 must be 16-byte aligned");
+    cudaError_t e = launch_quant_q_i8(q, n, heads, reinterpret_cast<int8_t *>(q8), q_scale,
+                                      reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "quantize q");
+    return ISPA_OK;
+}
+
+int ispa_quantize_k_i8(const ispa_attn_desc *desc, const void *k, signed char *k8, float *k_scale,
+                       ispa_stream_t stream) {
+    g_last_error.clear();
+    int rc = check_i8_desc(desc);
+    if (rc != ISPA_OK) return rc;
+    if (desc->n_kv == 0) return ISPA_OK;
+    if (!k || !k8 || !k_scale) return fail(ISPA_ERR_INVALID_ARG, "k, k8 and k_scale are required");
+    if (!aligned(k, 16) || !aligned(k8, 16)) return fail(ISPA_ERR_INVALID_ARG, "k and k8 must be 16-byte aligned");
+    cudaError_t e = launch_quant_k_i8(k, desc->heads, row_order_segments(desc), count_k_blocks(desc),
+                                      reinterpret_cast<int8_t *>(k8), k_scale, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "quantize k");
+    return ISPA_OK;
+}
+
+int ispa_attn_split_i8(const ispa_attn_desc *desc, const signed char *q8, const float *q_scale,
+                       const signed char *k8, const float *k_scale, const void *v, void *o_full, float *lse_full,
+                       void *o_loc, float *lse_loc, void *o_hist, float *lse_hist, const ispa_stats *stats, void *ws,
+                       size_t ws_bytes, ispa_stream_t stream) {
+    g_last_error.clear();
+    int rc = check_i8_desc(desc);
+    if (rc != ISPA_OK) return rc;
+    if (desc->n_q > 0 && !q_scale) return fail(ISPA_ERR_INVALID_ARG, "q_scale is required");
+    if (desc->n_kv > 0 && !k_scale) return fail(ISPA_ERR_INVALID_ARG, "k_scale is required");
+    return attn_split_impl(desc, q8, k8, v, o_full, lse_full, o_loc, lse_loc, o_hist, lse_hist, stats, ws, ws_bytes,
+                           stream, q_scale, k_scale);
 }
 
 int ispa_accum_stats(const ispa_stats *stats, const void *a_loc, const void *a_full, int n_rows, ispa_dtype dtype,

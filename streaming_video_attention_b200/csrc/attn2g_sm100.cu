@@ -35,6 +35,14 @@
 // of the two groups through shared memory (the Q area, no longer read), and each group merges
 // and stores half of the output columns.
 //
+// 8-bit variant (kI8) [ISPA §3.4 builds on 8-bit attention kernels, SageAttention]: Q and K
+// arrive as int8 with a scale per (token, head) for Q and per (128-row block of a partition
+// segment, head) for K; S = Q8 K8^T runs as tcgen05 kind::i8 (exact int32 accumulation, half
+// the bytes and twice the rate of the bf16 MMA); V, P, PV and everything after stay as in the
+// bf16 path. The softmax reads each int32 score as the float bits of 1.5 * 2^23 + s (one
+// integer add; exact while |s| < 2^22, and |s| <= 128 * 127 * 127) and folds the offset and
+// the per-row, per-tile scale s_q s_k into the FMA that forms the exponent.
+//
 // Every mbarrier wait is bounded; on timeout the CTA records ISPA_ERR_TIMEOUT in the device
 // flag and every role leaves its loop.
 #include <cuda.h>
@@ -59,21 +67,29 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr unsigned kPolyPairs = 0x22;   // column pairs (index mod 8) on the FMA-pipe exponential
 
-constexpr int kQBytes = kBlockM * HD * 2;
-constexpr int kKVBytes = kBlockN * HD * 2;
-constexpr int kSpillBytes = kBlockM * HD * 4;   // fp32 local state
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQBytes;
-constexpr int kOffV = kOffK + kStages * kKVBytes;
-constexpr int kOffSpill = kOffV + kStages * kKVBytes;
-constexpr int kOffSpillML = kOffSpill + kSpillBytes;   // float m[128], l[128]
-constexpr int kOffBar = kOffSpillML + 2 * kBlockM * 4;
-// q, k full/empty, v full/empty, s_full[2], p_full[2], spill, done
-constexpr int kNumBars = 1 + 4 * kStages + 2 * 2 + 1 + 1;
-constexpr int kOffSeg = kOffBar + kNumBars * 8;
-constexpr int kOffMisc = kOffSeg + 4 * kMaxSegments * 4;
-constexpr int kSmem = kOffMisc + 16 + 1024;   // + slack for 1024-byte alignment
-static_assert(kSmem <= 232448, "shared memory budget");
+// Shared-memory layout; Q and K tiles hold 1-byte (kI8) or 2-byte elements.
+template <bool kI8>
+struct Layout {
+    static constexpr int kQKElem = kI8 ? 1 : 2;
+    static constexpr int kQBytes = kBlockM * HD * kQKElem;
+    static constexpr int kKBytes = kBlockN * HD * kQKElem;
+    static constexpr int kVBytes = kBlockN * HD * 2;
+    static constexpr int kBoxes = HD * kQKElem / 128;     // 128-byte-wide TMA boxes per Q/K row
+    static constexpr int kSSteps = HD * kQKElem / 32;     // S MMAs per tile: 32 bytes of K each
+    static constexpr int kSpillBytes = kBlockM * HD * 4;   // fp32 local state
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + kQBytes;
+    static constexpr int kOffV = kOffK + kStages * kKBytes;
+    static constexpr int kOffSpill = kOffV + kStages * kVBytes;
+    static constexpr int kOffSpillML = kOffSpill + kSpillBytes;   // float m[128], l[128]
+    static constexpr int kOffBar = kOffSpillML + 2 * kBlockM * 4;
+    // q, k full/empty, v full/empty, s_full[2], p_full[2], spill, done
+    static constexpr int kNumBars = 1 + 4 * kStages + 2 * 2 + 1 + 1;
+    static constexpr int kOffSeg = kOffBar + kNumBars * 8;
+    static constexpr int kOffMisc = kOffSeg + 4 * kMaxSegments * 4;
+    static constexpr int kSmem = kOffMisc + 16 + 1024;   // + slack for 1024-byte alignment
+};
+static_assert(Layout<false>::kSmem <= 232448 && Layout<true>::kSmem <= 232448, "shared memory budget");
 
 struct Split2gParams {
     void *o_full;
@@ -88,6 +104,11 @@ struct Split2gParams {
     float scale_log2;
     SegmentList segs;   // local segments first, then history segments
     int *err_flag;
+    // 8-bit variant: Q scales [n_q][heads], K scales [heads][n_blocks], and for each segment
+    // (in the order above) the row-order index of its first K block
+    const float *q_scale, *k_scale;
+    int n_blocks;
+    int seg_block0[kMaxSegments];
 };
 
 struct TileCursor {
@@ -103,11 +124,28 @@ struct TileCursor {
         if (row0 >= end && ++si < nseg) load();
     }
     __device__ __forceinline__ int valid() const { return min(kBlockN, end - row0); }
+    __device__ __forceinline__ int block(const int *blk0) const { return blk0[si] + (row0 - sb[si]) / kBlockN; }
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Instruction descriptor, kind::i8: D s32, A and B signed 8-bit, both K-major.
+__host__ __device__ constexpr uint32_t make_idesc_s8(int M, int N) {
+    return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_s8_ss_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
 __device__ __forceinline__ void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow)); }
@@ -133,15 +171,17 @@ __device__ __forceinline__ uint32_t spill_off(int r, int c) {
     return (uint32_t)r * (HD * 4) + (uint32_t)((c ^ (r & 7)) * 16);
 }
 
+template <bool kI8>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_split_2g_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const Split2gParams p) {
+    using L = Layout<kI8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sQ = smem + kOffQ;
-    uint8_t *sK = smem + kOffK;
-    uint8_t *sV = smem + kOffV;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+    uint8_t *sQ = smem + L::kOffQ;
+    uint8_t *sK = smem + L::kOffK;
+    uint8_t *sV = smem + L::kOffV;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
     uint64_t *q_full = bars;
     uint64_t *k_full = q_full + 1;         // [kStages]
     uint64_t *k_empty = k_full + kStages;  // [kStages]
@@ -151,11 +191,12 @@ attn_split_2g_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     uint64_t *p_full = s_full + 2;         // [2] per group (4 warps each)
     uint64_t *spill_bar = p_full + 2;      // the first group's local state is in the buffer
     uint64_t *done_bar = spill_bar + 1;
-    int *seg_begin = reinterpret_cast<int *>(smem + kOffSeg);
+    int *seg_begin = reinterpret_cast<int *>(smem + L::kOffSeg);
     int *seg_end = seg_begin + kMaxSegments;
     int *seg_part = seg_end + kMaxSegments;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
+    int *seg_blk0 = seg_part + kMaxSegments;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int q0 = blockIdx.x * kBlockM;
@@ -179,6 +220,7 @@ attn_split_2g_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             seg_begin[s] = p.segs.seg[s].begin;
             seg_end[s] = p.segs.seg[s].end;
             seg_part[s] = p.segs.seg[s].part;
+            seg_blk0[s] = p.seg_block0[s];
         }
         ptx::mbar_init(q_full, 1);
         for (int i = 0; i < kStages; ++i) {
@@ -215,6 +257,10 @@ attn_split_2g_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         // warp 0: Q, then K; warp 2: V. All lanes run the loop, one elected lane issues.
         const bool is_k = warp == 0;
         const CUtensorMap *tm = is_k ? &tmK : &tmV;
+        // a K tile is kBoxes boxes of 128 bytes x 128 rows, a V tile two (bf16)
+        const int tile_bytes = is_k ? L::kKBytes : L::kVBytes;
+        const int boxes = is_k ? L::kBoxes : 2;
+        const int box_cols = is_k ? 128 / L::kQKElem : 64;
         uint8_t *ring = is_k ? sK : sV;
         uint64_t *full = is_k ? k_full : v_full;
         uint64_t *empty = is_k ? k_empty : v_empty;
@@ -222,10 +268,11 @@ attn_split_2g_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         if (lane == 0) ptx::tma_prefetch_desc(tm);
         if (is_k) {
             if (lane == 0) ptx::tma_prefetch_desc(&tmQ);
-            ptx::mbar_arrive_expect_tx_warp(q_full, kQBytes);
+            ptx::mbar_arrive_expect_tx_warp(q_full, L::kQBytes);
 #pragma unroll
-            for (int b = 0; b < HD / 64; ++b)
-                ptx::tma_load_3d_warp(sQ + b * (kBlockM * 128), &tmQ, q_full, b * 64, head, q0, ptx::policy_evict_first());
+            for (int b = 0; b < L::kBoxes; ++b)
+                ptx::tma_load_3d_warp(sQ + b * (kBlockM * 128), &tmQ, q_full, b * (128 / L::kQKElem), head, q0,
+                                      ptx::policy_evict_first());
         }
         TileCursor cur;
         cur.init(seg_begin, seg_end, seg_part, nseg);
@@ -236,11 +283,10 @@ attn_split_2g_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             ok = ptx::mbar_wait_bounded(&empty[st], ((j / kStages) & 1) ^ 1, kWaitLimitNs, p.err_flag, abort_flag);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
-            ptx::mbar_arrive_expect_tx_warp(&full[st], kKVBytes);
-#pragma unroll
-            for (int b = 0; b < HD / 64; ++b)
-                ptx::tma_load_3d_warp(ring + st * kKVBytes + b * (kBlockN * 128), tm, &full[st], b * 64, head, cur.row0,
-                                      pol_kv);
+            ptx::mbar_arrive_expect_tx_warp(&full[st], tile_bytes);
+            for (int b = 0; b < boxes; ++b)
+                ptx::tma_load_3d_warp(ring + st * tile_bytes + b * (kBlockN * 128), tm, &full[st], b * box_cols, head,
+                                      cur.row0, pol_kv);
             issued = j;
         }
         if (!ok) {
@@ -252,7 +298,8 @@ attn_split_2g_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (converged)
         regs_dec();
-        constexpr uint32_t idesc_qk = ptx::make_idesc_bf16(kBlockM, kBlockN, false, false);
+        constexpr uint32_t idesc_qk =
+            kI8 ? make_idesc_s8(kBlockM, kBlockN) : ptx::make_idesc_bf16(kBlockM, kBlockN, false, false);
         constexpr uint32_t idesc_pv = ptx::make_idesc_bf16(kBlockM, HD, false, true);
         const uint32_t aQ = ptx::smem_u32(sQ), aK = ptx::smem_u32(sK), aV = ptx::smem_u32(sV);
         bool ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(q_full, 0, kWaitLimitNs, p.err_flag, abort_flag));
@@ -262,11 +309,14 @@ attn_split_2g_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             if (!__all_sync(0xffffffffu, w)) return false;
             ptx::tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < HD / 16; ++kk) {
+            for (int kk = 0; kk < L::kSSteps; ++kk) {
                 const uint32_t koff = (kk / 4) * (kBlockM * 128) + (kk % 4) * 32;
-                ptx::umma_f16_ss_warp(tS(g), ptx::make_sdesc_sw128(aQ + koff, 16, 1024),
-                                      ptx::make_sdesc_sw128(aK + ks * kKVBytes + koff, 16, 1024), idesc_qk,
-                                      kk > 0 ? 1u : 0u);
+                const uint64_t da = ptx::make_sdesc_sw128(aQ + koff, 16, 1024);
+                const uint64_t db = ptx::make_sdesc_sw128(aK + ks * L::kKBytes + koff, 16, 1024);
+                if constexpr (kI8)
+                    umma_s8_ss_warp(tS(g), da, db, idesc_qk, kk > 0 ? 1u : 0u);
+                else
+                    ptx::umma_f16_ss_warp(tS(g), da, db, idesc_qk, kk > 0 ? 1u : 0u);
             }
             ptx::umma_commit_warp(&s_full[g]);
             ptx::umma_commit_warp(&k_empty[ks]);
@@ -289,7 +339,7 @@ attn_split_2g_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
 #pragma unroll
             for (int kk = 0; kk < kBlockN / 16; ++kk)
                 ptx::umma_f16_ts_warp(tO(g), tS(g) + kk * 8,
-                                      ptx::make_sdesc_sw128(aV + vs * kKVBytes + kk * 2048, kBlockN * 128, 1024),
+                                      ptx::make_sdesc_sw128(aV + vs * L::kVBytes + kk * 2048, kBlockN * 128, 1024),
                                       idesc_pv, kk > 0 ? 1u : acc0);
             ptx::umma_commit_warp(&v_empty[vs]);
             if (j + 2 < n_tiles) ok = issue_s(j + 2);
@@ -305,12 +355,17 @@ attn_split_2g_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         const int wq = warp % 4;                     // TMEM lane quarter
         const int row = wq * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-        uint8_t *spill = smem + kOffSpill;
-        float *spill_m = reinterpret_cast<float *>(smem + kOffSpillML);
+        uint8_t *spill = smem + L::kOffSpill;
+        float *spill_m = reinterpret_cast<float *>(smem + L::kOffSpillML);
         float *spill_l = spill_m + kBlockM;
         // the group of the first history tile hands its local state over first
         const int first_group = n_local & 1;
         const bool has_history = n_local < n_tiles;
+        // exponent factor of a score (log2 units): the softmax scale, times s_q s_k for int8
+        constexpr float kOff = kI8 ? 12582912.0f : 0.0f;   // 1.5 * 2^23: an int32 score's float offset
+        float rsq = p.scale_log2;
+        if constexpr (kI8)
+            if (q0 + row < p.n_q) rsq *= p.q_scale[(size_t)(q0 + row) * p.heads + head];
         float m_run = -INFINITY, l_run = 0.f;    // this group's partition being walked
         int part_run = -1;
         TileCursor cur;
@@ -319,6 +374,11 @@ attn_split_2g_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         bool ok = true;
         for (int j = g; j < n_tiles && ok; j += 2, cur.advance(), cur.advance()) {
             const int valid = cur.valid();
+            float rs = rsq;
+            // a zero scale comes only with all-zero scores (an all-zero Q row or K block): any
+            // positive factor gives them the same exponent, and keeps -inf * rs = -inf on the
+            // masked columns of a ragged tile (0 * -inf would be NaN)
+            if constexpr (kI8) rs = fmaxf(rs * p.k_scale[(size_t)head * p.n_blocks + cur.block(seg_blk0)], 1.17549435e-38f);
             bool to_history = false, had_local = false;
             float m_prev = -INFINITY, l_prev = 0.f;
             if (cur.part != part_run) {
@@ -339,6 +399,10 @@ attn_split_2g_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             for (int c = 0; c < kBlockN / 32; ++c)
                 ptx::tmem_ld32(tS(g) + lane_off + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
             ptx::tmem_wait_ld();
+            if constexpr (kI8) {
+#pragma unroll
+                for (int c = 0; c < kBlockN; ++c) sr[c] += 0x4B400000u;   // float bits of 1.5 * 2^23 + score
+            }
             float *s = reinterpret_cast<float *>(sr);
             if (valid < kBlockN) {
 #pragma unroll
@@ -353,8 +417,9 @@ attn_split_2g_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 for (int c = 1; c < 15; c += 2) mx8[u] = ptx::max3(mx8[u], s[16 * u + c], s[16 * u + c + 1]);
                 mx8[u] = fmaxf(mx8[u], s[16 * u + 15]);
             }
-            const float mx = ptx::max3(ptx::max3(mx8[0], mx8[1], mx8[2]), ptx::max3(mx8[3], mx8[4], mx8[5]),
-                                       fmaxf(mx8[6], mx8[7])) * p.scale_log2;
+            const float mxr = ptx::max3(ptx::max3(mx8[0], mx8[1], mx8[2]), ptx::max3(mx8[3], mx8[4], mx8[5]),
+                                        fmaxf(mx8[6], mx8[7]));
+            const float mx = (kI8 ? mxr - kOff : mxr) * rs;
             float alpha = 1.f;
             bool rescale = false;
             if (mx > m_run + kRescaleThreshold || m_run == -INFINITY) {
@@ -366,8 +431,10 @@ attn_split_2g_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             }
             uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
             uint32_t pk[kBlockN / 2];
-            const uint64_t sc2 = ptx::f2_pack(p.scale_log2, p.scale_log2);
-            const uint64_t nm2 = ptx::f2_pack(-m_run, -m_run);
+            // x = (s - kOff) rs - m as one FMA: s rs - (kOff rs + m)
+            const float nm = kI8 ? -fmaf(kOff, rs, m_run) : -m_run;
+            const uint64_t sc2 = ptx::f2_pack(rs, rs);
+            const uint64_t nm2 = ptx::f2_pack(nm, nm);
 #pragma unroll
             for (int q = 0; q < kBlockN / 2; ++q) {
                 const uint64_t x2 = ptx::f2_fma(ptx::f2_pack(s[2 * q], s[2 * q + 1]), sc2, nm2);
@@ -607,31 +674,32 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [rows, heads, 128] bf16, box = 128 rows x 64 columns of one head, 128-byte swizzle.
-bool make_rows_map(CUtensorMap *m, const void *ptr, int rows, int heads) {
+// [rows, heads, 128] of 1-byte (int8) or 2-byte (bf16) elements; box = 128 bytes of one row of
+// one head x 128 rows, 128-byte swizzle.
+bool make_rows_map(CUtensorMap *m, const void *ptr, int rows, int heads, int esize) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)heads, (cuuint64_t)rows};
-    cuuint64_t strides[2] = {(cuuint64_t)HD * 2, (cuuint64_t)heads * HD * 2};
-    cuuint32_t box[3] = {64, 1, 128};
+    cuuint64_t strides[2] = {(cuuint64_t)HD * esize, (cuuint64_t)heads * HD * esize};
+    cuuint32_t box[3] = {(cuuint32_t)(128 / esize), 1, 128};
     cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    return fn(m, esize == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+              const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
-
-// head_dim 128 only.
-cudaError_t launch_attn_bf16_2g(const AttnArgs &a, cudaStream_t s) {
+template <bool kI8>
+cudaError_t launch_2g(const AttnArgs &a, const float *q_scale, const float *k_scale, cudaStream_t s) {
+    using L = Layout<kI8>;
     if (a.n_q == 0) return cudaSuccess;
     if (a.head_dim != HD) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv;
     const void *kp = a.n_kv > 0 ? a.k : a.q;
     const void *vp = a.n_kv > 0 ? a.v : a.q;
     const int kv_rows = a.n_kv > 0 ? a.n_kv : a.n_q;
-    if (!make_rows_map(&mq, a.q, a.n_q, a.heads) || !make_rows_map(&mk, kp, kv_rows, a.heads) ||
-        !make_rows_map(&mv, vp, kv_rows, a.heads))
+    if (!make_rows_map(&mq, a.q, a.n_q, a.heads, L::kQKElem) || !make_rows_map(&mk, kp, kv_rows, a.heads, L::kQKElem) ||
+        !make_rows_map(&mv, vp, kv_rows, a.heads, 2))
         return cudaErrorInvalidValue;
     Split2gParams p;
     p.o_full = a.o_full; p.lse_full = a.lse_full;
@@ -646,22 +714,44 @@ cudaError_t launch_attn_bf16_2g(const AttnArgs &a, cudaStream_t s) {
             if (a.segs.seg[i].part == part) p.segs.seg[p.segs.count++] = a.segs.seg[i];
     if (p.segs.count != a.segs.count) return cudaErrorInvalidValue;
     p.err_flag = a.err_flag;
-    cudaError_t e = cudaFuncSetAttribute(attn_split_2g_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    // K blocks are numbered in row order: each segment's first block index
+    p.q_scale = q_scale;
+    p.k_scale = k_scale;
+    p.n_blocks = 0;
+    for (int i = 0; i < p.segs.count; ++i) {
+        int first = 0;
+        for (int j = 0; j < p.segs.count; ++j)
+            if (p.segs.seg[j].begin < p.segs.seg[i].begin)
+                first += (p.segs.seg[j].end - p.segs.seg[j].begin + kBlockN - 1) / kBlockN;
+        p.seg_block0[i] = first;
+        p.n_blocks += (p.segs.seg[i].end - p.segs.seg[i].begin + kBlockN - 1) / kBlockN;
+    }
+    cudaError_t e = cudaFuncSetAttribute(attn_split_2g_kernel<kI8>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
     if (e != cudaSuccess) return e;
     // setmaxnreg.inc waits until the registers it asks for are free in the CTA's own
     // allocation: refuse to launch unless the split fits what the kernel is launched with
     static int launch_regs = -1;
     if (launch_regs < 0) {
         cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, attn_split_2g_kernel);
+        e = cudaFuncGetAttributes(&fa, attn_split_2g_kernel<kI8>);
         if (e != cudaSuccess) return e;
         launch_regs = fa.numRegs;
     }
     if (launch_regs * kThreads < kRegsNeeded) return cudaErrorInvalidConfiguration;
     dim3 grid((a.n_q + kBlockM - 1) / kBlockM, a.heads);
-    attn_split_2g_kernel<<<grid, kThreads, kSmem, s>>>(mq, mk, mv, p);
+    attn_split_2g_kernel<kI8><<<grid, kThreads, L::kSmem, s>>>(mq, mk, mv, p);
     note_launch();
     return cudaGetLastError();
+}
+
+}  // namespace
+
+// head_dim 128 only.
+cudaError_t launch_attn_bf16_2g(const AttnArgs &a, cudaStream_t s) { return launch_2g<false>(a, nullptr, nullptr, s); }
+
+// int8 Q and K (a.q, a.k) with their scales, bf16 V; head_dim 128 only.
+cudaError_t launch_attn_i8_2g(const AttnArgs &a, const float *q_scale, const float *k_scale, cudaStream_t s) {
+    return launch_2g<true>(a, q_scale, k_scale, s);
 }
 
 }  // namespace ispa

@@ -65,6 +65,8 @@ cudaError_t launch_attn_simt_bf16(const AttnArgs &a, cudaStream_t s);
 cudaError_t launch_attn_bf16(const AttnArgs &a, cudaStream_t s);   // tcgen05 path
 cudaError_t launch_attn_bf16_2sm(const AttnArgs &a, cudaStream_t s);   // tcgen05 CTA-pair path, head_dim 128
 cudaError_t launch_attn_bf16_2g(const AttnArgs &a, cudaStream_t s);    // tcgen05, two softmax groups, head_dim 128
+// int8 Q/K (a.q, a.k; scales [n_q][heads] and [heads][K blocks]), bf16 V; head_dim 128
+cudaError_t launch_attn_i8_2g(const AttnArgs &a, const float *q_scale, const float *k_scale, cudaStream_t s);
 
 // Batched SIMT GEMM: C_z[m][n] = alpha * sum_k A_z(m,k) B_z(k,n) + beta * C_z[m][n].
 // A_z(m,k) = A[m*lda + k] if a_kcontig else A[k*lda + m]; B_z(k,n) = B[n*ldb + k] if
@@ -96,6 +98,9 @@ cudaError_t launch_gemm_bf16(const void *A, const void *W, void *y, int M, int N
 
 // W8A8 projection (w8a8_sm100.cu): weights [K][N] -> int8 [N][K] + column scales; then
 // y[M][N] (bf16) from activations A [M][K] (bf16) quantised by rows into q_a / s_a.
+cudaError_t launch_quant_q_i8(const void *q, int n, int heads, int8_t *q8, float *q_scale, cudaStream_t s);
+cudaError_t launch_quant_k_i8(const void *k, int heads, const SegmentList &segs, int n_blocks, int8_t *k8,
+                              float *k_scale, cudaStream_t s);
 cudaError_t launch_quant_cols(const void *w, ElemType t, int K, int N, int8_t *qt, float *scale, cudaStream_t s);
 cudaError_t launch_project_w8a8(const void *A, int M, int K, const int8_t *qt, const float *col_scale, int N,
                                 void *y, int8_t *q_a, float *s_a, int *err_flag, cudaStream_t s);

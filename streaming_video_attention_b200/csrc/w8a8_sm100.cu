@@ -80,6 +80,65 @@ __global__ void quant_rows_kernel(const bf16 *__restrict__ x, int n, int K, int8
     if (lane == 0) scale[warp] = __fdiv_rn(amax, 127.f);
 }
 
+// K of the 8-bit split attention: one scale per (block, head), a block being up to 128 rows
+// of one KV segment (segments in row order, each cut into blocks from its first row).
+// k [n_kv][heads][128] bf16 -> k8 (same layout) + k_scale [heads][n_blocks]. One CTA per
+// (block, head); thread t handles 8 columns (one 16-byte vector) of rows t/16, t/16 + 16, ...
+__global__ void __launch_bounds__(256) quant_kblocks_kernel(const bf16 *__restrict__ k, int heads, SegmentList segs,
+                                                            int n_blocks, int8_t *__restrict__ k8,
+                                                            float *__restrict__ k_scale) {
+    const int blk = blockIdx.x, head = blockIdx.y;
+    int first = 0, r0 = 0, r1 = 0;
+    for (int i = 0; i < segs.count; ++i) {
+        const int nb = (segs.seg[i].end - segs.seg[i].begin + 127) / 128;
+        if (blk < first + nb) {
+            r0 = segs.seg[i].begin + (blk - first) * 128;
+            r1 = min(r0 + 128, segs.seg[i].end);
+            break;
+        }
+        first += nb;
+    }
+    const int v = threadIdx.x % 16, rb = threadIdx.x / 16;
+    uint4 val[8];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int r = r0 + rb + 16 * i;
+        val[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (r < r1) val[i] = *reinterpret_cast<const uint4 *>(k + ((size_t)r * heads + head) * 128 + v * 8);
+        const uint32_t w[4] = {val[i].x, val[i].y, val[i].z, val[i].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            amax = fmaxf(amax, fabsf(__uint_as_float(w[j] << 16)));
+            amax = fmaxf(amax, fabsf(__uint_as_float(w[j] & 0xFFFF0000u)));
+        }
+    }
+    __shared__ float red[8];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = amax;
+    __syncthreads();
+    amax = red[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+    const float inv = amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int r = r0 + rb + 16 * i;
+        if (r >= r1) continue;
+        const uint32_t w[4] = {val[i].x, val[i].y, val[i].z, val[i].w};
+        uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int lo = quant1(__uint_as_float(w[j] << 16), inv);
+            const int hi = quant1(__uint_as_float(w[j] & 0xFFFF0000u), inv);
+            packed[j / 2] |= ((uint32_t)(lo & 0xFF) | ((uint32_t)(hi & 0xFF) << 8)) << (16 * (j % 2));
+        }
+        *reinterpret_cast<uint2 *>(k8 + ((size_t)r * heads + head) * 128 + v * 8) = make_uint2(packed[0], packed[1]);
+    }
+    if (threadIdx.x == 0) k_scale[(size_t)head * n_blocks + blk] = __fdiv_rn(amax, 127.f);
+}
+
 // Weights w [K][N] row-major -> codes qt [N][K] and column scales [N]. CTA = 32 columns x 8
 // row groups; pass 1 finds each column's amax, pass 2 quantises 32 x 128 tiles through shared
 // memory so that both the reads of w and the writes of qt are coalesced.
@@ -325,6 +384,26 @@ cudaError_t launch_project_w8a8(const void *A, int M, int K, const int8_t *qt, c
     e = cudaFuncSetAttribute(gemm_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     gemm_i8_kernel<<<dim3(N / kTile, (M + kTile - 1) / kTile), kThreads, kSmem, s>>>(ta, tb, p);
+    note_launch();
+    return cudaGetLastError();
+}
+
+// Q of the 8-bit split attention: q [n][heads][128] bf16 -> q8 (same layout) + q_scale
+// [n][heads], one symmetric scale per (token, head): the row quantiser on n * heads rows.
+cudaError_t launch_quant_q_i8(const void *q, int n, int heads, int8_t *q8, float *q_scale, cudaStream_t s) {
+    const int rows = n * heads;
+    if (rows <= 0) return cudaSuccess;
+    quant_rows_kernel<<<(rows + 7) / 8, 256, 0, s>>>(static_cast<const bf16 *>(q), rows, 128, q8, q_scale);
+    note_launch();
+    return cudaGetLastError();
+}
+
+// K of the 8-bit split attention; segs in row order, n_blocks = their 128-row blocks.
+cudaError_t launch_quant_k_i8(const void *k, int heads, const SegmentList &segs, int n_blocks, int8_t *k8,
+                              float *k_scale, cudaStream_t s) {
+    if (n_blocks <= 0) return cudaSuccess;
+    quant_kblocks_kernel<<<dim3(n_blocks, heads), 256, 0, s>>>(static_cast<const bf16 *>(k), heads, segs, n_blocks, k8,
+                                                                k_scale);
     note_launch();
     return cudaGetLastError();
 }

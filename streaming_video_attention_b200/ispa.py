@@ -30,6 +30,7 @@ ISPA_FP32 = 1
 EXPORTS = (
     "ispa_attn_split", "ispa_attn_split_noalloc", "ispa_accum_stats", "ispa_stats_reset", "ispa_solve_absorb",
     "ispa_absorb_error", "ispa_quantize_w8", "ispa_project_w8a8", "ispa_select_layers",
+    "ispa_quantize_q_i8", "ispa_k_blocks", "ispa_quantize_k_i8", "ispa_attn_split_i8",
     "ispa_local_attn", "ispa_workspace_bytes", "ispa_device_status", "ispa_selftest_bounded_wait",
     "ispa_selftest_exp2_poly", "ispa_set_attn_kernel", "ispa_kernel_launches", "ispa_last_error", "ispa_version",
 )
@@ -70,6 +71,11 @@ def lib() -> ctypes.CDLL:
                                       ctypes.POINTER(CStats), vp, sz, vp]
         L.ispa_attn_split_noalloc.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                               ctypes.POINTER(CStats), vp]
+        L.ispa_attn_split_i8.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                         ctypes.POINTER(CStats), vp, sz, vp]
+        L.ispa_quantize_q_i8.argtypes = [vp, i, i, i, vp, vp, vp]
+        L.ispa_k_blocks.argtypes = [ctypes.POINTER(AttnDesc)]
+        L.ispa_quantize_k_i8.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp]
         L.ispa_accum_stats.argtypes = [ctypes.POINTER(CStats), vp, vp, i, i, vp, sz, vp]
         L.ispa_stats_reset.argtypes = [ctypes.POINTER(CStats), vp]
         L.ispa_solve_absorb.argtypes = [ctypes.POINTER(CStats), i, ctypes.POINTER(vp), i, f, vp, vp, vp,
@@ -148,6 +154,35 @@ def ispa_attn_split(desc, q, k, v, o_full, lse_full, o_loc=None, lse_loc=None, o
                                _p(lse_loc), _p(o_hist), _p(lse_hist), cs, _p(ws),
                                0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "ispa_attn_split")
+
+
+def ispa_quantize_q_i8(q: torch.Tensor, q8: torch.Tensor, q_scale: torch.Tensor, stream=None) -> None:
+    """q [n, heads, 128] bf16 -> q8 int8 (same shape), q_scale [n, heads] float32."""
+    n, heads, hd = q.shape
+    _check(lib().ispa_quantize_q_i8(_p(q), n, heads, hd, _p(q8), _p(q_scale), _stream(stream)), "ispa_quantize_q_i8")
+
+
+def ispa_k_blocks(desc) -> int:
+    rc = lib().ispa_k_blocks(ctypes.byref(desc))
+    if rc < 0:
+        _check(rc, "ispa_k_blocks")
+    return rc
+
+
+def ispa_quantize_k_i8(desc, k: torch.Tensor, k8: torch.Tensor, k_scale: torch.Tensor, stream=None) -> None:
+    """k [n_kv, heads, 128] bf16 -> k8 int8 (same shape), k_scale [heads, ispa_k_blocks(desc)] float32."""
+    _check(lib().ispa_quantize_k_i8(ctypes.byref(desc), _p(k), _p(k8), _p(k_scale), _stream(stream)),
+           "ispa_quantize_k_i8")
+
+
+def ispa_attn_split_i8(desc, q8, q_scale, k8, k_scale, v, o_full, lse_full, o_loc=None, lse_loc=None, o_hist=None,
+                       lse_hist=None, stats: Optional[Stats] = None, ws: Optional[torch.Tensor] = None,
+                       stream=None) -> None:
+    cs = ctypes.byref(stats.c()) if stats is not None else None
+    rc = lib().ispa_attn_split_i8(ctypes.byref(desc), _p(q8), _p(q_scale), _p(k8), _p(k_scale), _p(v), _p(o_full),
+                                  _p(lse_full), _p(o_loc), _p(lse_loc), _p(o_hist), _p(lse_hist), cs, _p(ws),
+                                  0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "ispa_attn_split_i8")
 
 
 def ispa_attn_split_noalloc(desc, q, k, v, o_full, lse_full, o_loc=None, lse_loc=None, o_hist=None,

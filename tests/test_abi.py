@@ -106,3 +106,28 @@ def test_w8a8_arguments_are_checked_before_any_launch():
     assert L.ispa_project_w8a8(fake, 0, 128, fake, fake, 128, fake, None, 0, None) == ispa.ISPA_OK
     # the workspace covers the row codes and scales
     assert ispa.workspace_bytes(None, 4680, 1536) >= 4680 * 1536 + 4 * 4680
+
+
+def test_k_blocks_count_matches_oracle():
+    import oracle
+    for n_kv, sink, chunk in [(1000, (0, 64), (900, 1000)), (300, (0, 0), (200, 300)), (640, (0, 130), (130, 640)),
+                              (5, (0, 1), (1, 3)), (37440, (0, 1560), (32760, 37440)), (0, (0, 0), (0, 0))]:
+        desc = ispa.make_desc(10, n_kv, 2, 128, sink, chunk)
+        assert ispa.ispa_k_blocks(desc) == len(oracle.kv_blocks(n_kv, sink, chunk)), (n_kv, sink, chunk)
+
+
+def test_i8_arguments_are_checked_before_any_launch():
+    L = ispa.lib()
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: every call below fails its checks first
+    d64 = ispa.make_desc(10, 100, 2, 64, (0, 10), (50, 100))
+    dfp32 = ispa.make_desc(10, 100, 2, 128, (0, 10), (50, 100), dtype=ispa.ISPA_FP32)
+    d128 = ispa.make_desc(10, 100, 2, 128, (0, 10), (50, 100))
+    assert L.ispa_quantize_q_i8(fake, 10, 2, 64, fake, fake, None) == ispa.ISPA_ERR_UNSUPPORTED
+    assert L.ispa_quantize_q_i8(fake, 10, 2, 128, None, fake, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_quantize_k_i8(ctypes.byref(d64), fake, fake, fake, None) == ispa.ISPA_ERR_UNSUPPORTED
+    assert L.ispa_quantize_k_i8(ctypes.byref(d128), fake, fake, None, None) == ispa.ISPA_ERR_INVALID_ARG
+    args = (fake, fake, fake, fake, fake, fake, fake, None, None, None, None, None, None, 0, None)
+    assert L.ispa_attn_split_i8(ctypes.byref(dfp32), *args) == ispa.ISPA_ERR_UNSUPPORTED
+    assert L.ispa_attn_split_i8(ctypes.byref(d64), *args) == ispa.ISPA_ERR_UNSUPPORTED
+    no_qs = (fake, None) + args[2:]
+    assert L.ispa_attn_split_i8(ctypes.byref(d128), *no_qs) == ispa.ISPA_ERR_INVALID_ARG

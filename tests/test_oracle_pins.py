@@ -436,7 +436,7 @@ def test_i8_quantizers_hand_cases_and_bounds():
     q[0, 0] = [1.0, -2.0, 0.5, 0.25]
     q8, sq = oracle.quantize_i8_q(q)
     assert q8[0, 0].tolist() == [64, -127, 32, 16] and q8[1, 0].tolist() == [0, 0, 0, 0]   # 63.5 -> 64 (even)
-    assert sq.shape == (1, 2) and sq[0, 0] == np.float32(2.0) / np.float32(127.0) and sq[0, 1] == 0.0
+    assert sq.shape == (2, 1) and sq[0, 0] == np.float32(2.0) / np.float32(127.0) and sq[1, 0] == 0.0
     rng = np.random.default_rng(9)
     k = synth_bf16(rng.standard_normal((300, 3, 64)) * np.exp(rng.normal(0, 1, (300, 1, 1))))
     blocks = oracle.kv_blocks(300, (0, 40), (200, 300))
