@@ -100,6 +100,24 @@ int ispa_attn_split(const ispa_attn_desc *desc, const void *q, const void *k, co
                     float *lse_hist, const ispa_stats *stats, void *ws, size_t ws_bytes,
                     ispa_stream_t stream);
 
+/* ispa_attn_split_ops -- ispa_attn_split without the accumulation: the call's statistics
+ * operands A_loc and R = A_full - A_loc (computed on chip from the partition outputs, then
+ * rounded to desc->dtype) are written to a_ops and r_ops, each [n_q, heads*head_dim] device
+ * memory of desc->dtype, 16-byte aligned. With ispa_accum_ops this splits a warmup chunk into
+ * the attention of every layer followed by one statistics launch for all of them. */
+int ispa_attn_split_ops(const ispa_attn_desc *desc, const void *q, const void *k, const void *v,
+                        void *o_full, float *lse_full, void *o_loc, float *lse_loc, void *o_hist,
+                        float *lse_hist, void *a_ops, void *r_ops, ispa_stream_t stream);
+
+/* ispa_accum_ops -- G += A^T A, C += A^T R, H += R^T R and rows += n_rows for n_layers layers
+ * [ISPA §3.2]: a_ops and r_ops hold the layers' operands one after the other
+ * ([n_layers][n_rows][D], dtype, device, layer l at offset l*n_rows*D), per_layer[l] is layer
+ * l's statistics (all of the same D). bf16 operands with D a multiple of 128 go to the tensor
+ * cores in one launch per 48 layers, with the same tiles and the same reduction order as the
+ * fused accumulation of ispa_attn_split: the results are identical bit for bit. */
+int ispa_accum_ops(const ispa_stats *per_layer, int n_layers, const void *a_ops, const void *r_ops, int n_rows,
+                   ispa_dtype dtype, ispa_stream_t stream);
+
 /* 8-bit split attention [ISPA §3.4: the decomposition is built on 8-bit attention kernels,
  * SageAttention]: ispa_attn_split with S = scale * Q K^T taken from int8 copies of Q and K;
  * V, P, P V, the merge, the outputs and the fused statistics as in ispa_attn_split.

@@ -156,6 +156,13 @@ SegmentList make_segments(const ispa_attn_desc *d, bool local_only) {
 
 __global__ void add_rows_kernel(long long *rows, long long n) { *rows += n; }
 
+struct RowsBatch {
+    long long *r[kMaxBatch];
+};
+__global__ void add_rows_batch_kernel(RowsBatch rows, int layers, long long n) {
+    if (threadIdx.x < layers) *rows.r[threadIdx.x] += n;
+}
+
 template <typename T>
 __global__ void residual_kernel(const T *a_loc, const T *a_full, T *r, size_t n) {
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
@@ -348,6 +355,70 @@ int ispa_attn_split(const ispa_attn_desc *desc, const void *q, const void *k, co
     if (rc != ISPA_OK) return rc;
     return attn_split_impl(desc, q, k, v, o_full, lse_full, o_loc, lse_loc, o_hist, lse_hist, stats, ws, ws_bytes,
                            stream, nullptr, nullptr);
+}
+
+int ispa_attn_split_ops(const ispa_attn_desc *desc, const void *q, const void *k, const void *v, void *o_full,
+                        float *lse_full, void *o_loc, float *lse_loc, void *o_hist, float *lse_hist, void *a_ops,
+                        void *r_ops, ispa_stream_t stream) {
+    g_last_error.clear();
+    int rc = check_desc(desc, true);
+    if (rc != ISPA_OK) return rc;
+    if (desc->n_q > 0 && (!a_ops || !r_ops)) return fail(ISPA_ERR_INVALID_ARG, "a_ops and r_ops are required");
+    if ((a_ops && !aligned(a_ops, 16)) || (r_ops && !aligned(r_ops, 16)))
+        return fail(ISPA_ERR_INVALID_ARG, "a_ops and r_ops must be 16-byte aligned");
+    if (desc->n_q > 0 && (!q || !o_full || !lse_full)) return fail(ISPA_ERR_INVALID_ARG, "q, o_full and lse_full are required");
+    if (desc->n_kv > 0 && (!k || !v)) return fail(ISPA_ERR_INVALID_ARG, "k and v are required");
+    for (const void *p : {q, k, v, (const void *)o_full, (const void *)o_loc, (const void *)o_hist})
+        if (p && !aligned(p, 16)) return fail(ISPA_ERR_INVALID_ARG, "q/k/v/o buffers must be 16-byte aligned");
+    if (desc->n_q == 0) return ISPA_OK;
+    return run_attention(desc, q, k, v, o_full, lse_full, o_loc, lse_loc, o_hist, lse_hist, a_ops, r_ops, false,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+int ispa_accum_ops(const ispa_stats *per_layer, int n_layers, const void *a_ops, const void *r_ops, int n_rows,
+                   ispa_dtype dtype, ispa_stream_t stream) {
+    g_last_error.clear();
+    if (!per_layer || n_layers < 0) return fail(ISPA_ERR_INVALID_ARG, "per_layer is NULL or n_layers < 0");
+    if (dtype != ISPA_BF16 && dtype != ISPA_FP32) return fail(ISPA_ERR_INVALID_ARG, "bad dtype");
+    if (n_rows < 0) return fail(ISPA_ERR_INVALID_ARG, "n_rows < 0");
+    if (n_layers == 0) return ISPA_OK;
+    const int D = per_layer[0].D;
+    if (D <= 0) return fail(ISPA_ERR_INVALID_ARG, "D <= 0");
+    for (int l = 0; l < n_layers; ++l) {
+        int rc = check_stats(&per_layer[l], D);
+        if (rc != ISPA_OK) return fail(rc, "layer %d: %s", l, g_last_error.c_str());
+    }
+    if (n_rows > 0 && (!a_ops || !r_ops)) return fail(ISPA_ERR_INVALID_ARG, "a_ops and r_ops are required");
+    if ((a_ops && !aligned(a_ops, 16)) || (r_ops && !aligned(r_ops, 16)))
+        return fail(ISPA_ERR_INVALID_ARG, "a_ops and r_ops must be 16-byte aligned");
+    if (dtype == ISPA_BF16 && D % 64 != 0) return fail(ISPA_ERR_UNSUPPORTED, "bf16 statistics need D %% 64 == 0");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int *flag = nullptr;
+    int rc = device_error_flag(&flag);
+    if (rc != ISPA_OK) return rc;
+    const size_t per = (size_t)n_rows * D * elem_size(dtype);
+    for (int l0 = 0; l0 < n_layers; l0 += kMaxBatch) {
+        const int b = std::min(kMaxBatch, n_layers - l0);
+        const char *a = static_cast<const char *>(a_ops) + (size_t)l0 * per;
+        const char *r = static_cast<const char *>(r_ops) + (size_t)l0 * per;
+        if (dtype == ISPA_BF16 && n_rows > 0) {
+            float *G[kMaxBatch], *C[kMaxBatch], *H[kMaxBatch];
+            for (int z = 0; z < b; ++z) {
+                G[z] = per_layer[l0 + z].G; C[z] = per_layer[l0 + z].C; H[z] = per_layer[l0 + z].H;
+            }
+            CUDA_CHECK_RET(launch_stats_bf16_layers(a, r, b, n_rows, D, G, C, H, flag, s), "stats GEMM (bf16, layers)");
+            RowsBatch rows;
+            for (int z = 0; z < b; ++z) rows.r[z] = per_layer[l0 + z].rows;
+            add_rows_batch_kernel<<<1, 64, 0, s>>>(rows, b, n_rows); note_launch();
+            CUDA_CHECK_RET(cudaGetLastError(), "rows counters");
+        } else {
+            for (int z = 0; z < b; ++z) {
+                rc = accumulate(&per_layer[l0 + z], a + (size_t)z * per, r + (size_t)z * per, n_rows, dtype, flag, s);
+                if (rc != ISPA_OK) return rc;
+            }
+        }
+    }
+    return ISPA_OK;
 }
 
 // K blocks of the 8-bit split attention: the KV segments in row order, each cut into

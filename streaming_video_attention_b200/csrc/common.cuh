@@ -89,6 +89,8 @@ struct GemmDesc {
 cudaError_t launch_gemm_simt(const GemmDesc &d, const GemmBatch &b, cudaStream_t s);
 
 // Ridge statistics from bf16 operands [n, D] row-major, float32 G/C/H updated in place.
+cudaError_t launch_stats_bf16_layers(const void *a_loc, const void *r, int layers, int n, int D, float *const *G,
+                                     float *const *C, float *const *H, int *err_flag, cudaStream_t s);
 cudaError_t launch_stats_bf16(const void *a_loc, const void *r, int n, int D, float *G, float *C,
                                float *H, int *err_flag, cudaStream_t s);
 

@@ -3,8 +3,11 @@
 // from the bf16 operands A = A_loc and R = A_full - A_loc, each [n, D] row-major (the
 // layout the split-attention epilogue writes), accumulated in float32.
 //
-// One CTA owns one 128x128 output tile and reduces over all n token rows in a fixed
-// order (no atomics: results repeat bit for bit). G and H are symmetric: only tiles on or
+// One CTA owns one 128x128 output tile of one layer and reduces over all n token rows in a
+// fixed order (no atomics: results repeat bit for bit). Several layers whose operands lie
+// contiguously ([layers][n][D]) go in one launch (grid.y = layer), so that a warmup chunk's
+// statistics fill the GPU with ~30 waves instead of one short wave per layer; each tile's
+// arithmetic does not depend on the batching. G and H are symmetric: only tiles on or
 // above the block diagonal are computed, and each is written to both mirrored positions,
 // so the stored G and H are exactly symmetric.
 //
@@ -31,7 +34,7 @@ constexpr int kBarOff = kStages * kStageBytes;
 constexpr int kSmemAlloc = kBarOff + 256 + 1024;
 
 struct StatsParams {
-    float *out[3];      // G, C, H
+    float *out[kMaxBatch][3];   // per layer: G, C, H
     int D, n;
     int nb;             // D / 128
     int n_sym;          // upper-triangle tiles per symmetric matrix: nb*(nb+1)/2
@@ -64,6 +67,7 @@ stats_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int layer = blockIdx.y;
     int mat, bi, bj;
     decode_item(blockIdx.x, p.nb, p.n_sym, mat, bi, bj);
     const CUtensorMap *mapA = (mat == 2) ? &tmR : &tmA;   // left operand: A for G and C, R for H
@@ -106,9 +110,10 @@ stats_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
             ptx::mbar_arrive_expect_tx_warp(&full[s], kStageBytes);
 #pragma unroll
             for (int b = 0; b < 2; ++b) {
-                ptx::tma_load_2d_warp(base + b * (kKRows * 128), mapA, &full[s], bi * kTile + b * 64, kt * kKRows, pol);
-                ptx::tma_load_2d_warp(base + kOperandBytes + b * (kKRows * 128), mapB, &full[s], bj * kTile + b * 64,
-                                      kt * kKRows, pol);
+                ptx::tma_load_3d_warp(base + b * (kKRows * 128), mapA, &full[s], bi * kTile + b * 64, kt * kKRows,
+                                      layer, pol);
+                ptx::tma_load_3d_warp(base + kOperandBytes + b * (kKRows * 128), mapB, &full[s], bj * kTile + b * 64,
+                                      kt * kKRows, layer, pol);
             }
             issued = kt;
         }
@@ -149,7 +154,7 @@ stats_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         const bool ok = ptx::mbar_wait_bounded(acc_bar, 0, kWaitLimitNs, p.err_flag, abort_flag) && !*abort_flag;
         if (ok) {
             ptx::tc_fence_after();
-            float *M = p.out[mat];
+            float *M = p.out[layer][mat];
             const size_t D = p.D;
             const int gi = bi * kTile + r;
             const bool sym = (mat != 1);
@@ -217,41 +222,53 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [n, D] bf16 row-major, box = 64 rows x 64 columns, 128-byte swizzle.
-bool make_panel_map(CUtensorMap *m, const void *ptr, int n, int D) {
+// [layers, n, D] bf16 row-major, box = 64 rows x 64 columns of one layer, 128-byte swizzle.
+bool make_panel_map(CUtensorMap *m, const void *ptr, int layers, int n, int D) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)n};
-    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)kKRows};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)n, (cuuint64_t)layers};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)n * D * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)kKRows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
-cudaError_t launch_stats_bf16(const void *a_loc, const void *r, int n, int D, float *G, float *C, float *H,
-                              int *err_flag, cudaStream_t s) {
-    if (n <= 0) return cudaSuccess;
+// Layers [0, layers) with operands a_loc, r = [layers][n][D] contiguous and outputs
+// G[l], C[l], H[l]; layers <= kMaxBatch.
+cudaError_t launch_stats_bf16_layers(const void *a_loc, const void *r, int layers, int n, int D, float *const *G,
+                                     float *const *C, float *const *H, int *err_flag, cudaStream_t s) {
+    if (n <= 0 || layers <= 0) return cudaSuccess;
+    if (layers > kMaxBatch) return cudaErrorInvalidValue;
     if (D % kTile != 0) {
-        // D not a multiple of 128 (e.g. 64-wide single head): CUDA-core GEMM
-        GemmDesc g{D, D, n, D, D, D, false, false, ElemType::BF16, ElemType::BF16, ElemType::F32, 1.f, 1.f, false, 1};
-        GemmBatch b;
-        b.A[0] = a_loc; b.B[0] = a_loc; b.C[0] = G;
-        cudaError_t e = launch_gemm_simt(g, b, s);
-        if (e != cudaSuccess) return e;
-        b.A[0] = a_loc; b.B[0] = r; b.C[0] = C;
-        e = launch_gemm_simt(g, b, s);
-        if (e != cudaSuccess) return e;
-        b.A[0] = r; b.B[0] = r; b.C[0] = H;
-        return launch_gemm_simt(g, b, s);
+        // D not a multiple of 128 (e.g. 64-wide single head): CUDA-core GEMM, layer by layer
+        for (int l = 0; l < layers; ++l) {
+            const size_t off = (size_t)l * n * D * sizeof(bf16);
+            const void *al = static_cast<const char *>(a_loc) + off;
+            const void *rl = static_cast<const char *>(r) + off;
+            GemmDesc g{D, D, n, D, D, D, false, false, ElemType::BF16, ElemType::BF16, ElemType::F32, 1.f, 1.f, false, 1};
+            GemmBatch b;
+            b.A[0] = al; b.B[0] = al; b.C[0] = G[l];
+            cudaError_t e = launch_gemm_simt(g, b, s);
+            if (e != cudaSuccess) return e;
+            b.A[0] = al; b.B[0] = rl; b.C[0] = C[l];
+            e = launch_gemm_simt(g, b, s);
+            if (e != cudaSuccess) return e;
+            b.A[0] = rl; b.B[0] = rl; b.C[0] = H[l];
+            e = launch_gemm_simt(g, b, s);
+            if (e != cudaSuccess) return e;
+        }
+        return cudaSuccess;
     }
     CUtensorMap ma, mr;
-    if (!make_panel_map(&ma, a_loc, n, D) || !make_panel_map(&mr, r, n, D)) return cudaErrorInvalidValue;
+    if (!make_panel_map(&ma, a_loc, layers, n, D) || !make_panel_map(&mr, r, layers, n, D)) return cudaErrorInvalidValue;
     StatsParams p;
-    p.out[0] = G; p.out[1] = C; p.out[2] = H;
+    for (int l = 0; l < layers; ++l) {
+        p.out[l][0] = G[l]; p.out[l][1] = C[l]; p.out[l][2] = H[l];
+    }
     p.D = D; p.n = n;
     p.nb = D / kTile;
     p.n_sym = p.nb * (p.nb + 1) / 2;
@@ -259,8 +276,13 @@ cudaError_t launch_stats_bf16(const void *a_loc, const void *r, int n, int D, fl
     cudaError_t e = cudaFuncSetAttribute(stats_gemm_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
     if (e != cudaSuccess) return e;
     const int items = 2 * p.n_sym + p.nb * p.nb;
-    stats_gemm_sm100_kernel<<<items, kThreads, kSmemAlloc, s>>>(ma, mr, p); note_launch();
+    stats_gemm_sm100_kernel<<<dim3(items, layers), kThreads, kSmemAlloc, s>>>(ma, mr, p); note_launch();
     return cudaGetLastError();
+}
+
+cudaError_t launch_stats_bf16(const void *a_loc, const void *r, int n, int D, float *G, float *C, float *H,
+                              int *err_flag, cudaStream_t s) {
+    return launch_stats_bf16_layers(a_loc, r, 1, n, D, &G, &C, &H, err_flag, s);
 }
 
 }  // namespace ispa

@@ -31,6 +31,7 @@ EXPORTS = (
     "ispa_attn_split", "ispa_attn_split_noalloc", "ispa_accum_stats", "ispa_stats_reset", "ispa_solve_absorb",
     "ispa_absorb_error", "ispa_quantize_w8", "ispa_project_w8a8", "ispa_select_layers",
     "ispa_quantize_q_i8", "ispa_k_blocks", "ispa_quantize_k_i8", "ispa_attn_split_i8",
+    "ispa_attn_split_ops", "ispa_accum_ops",
     "ispa_local_attn", "ispa_workspace_bytes", "ispa_device_status", "ispa_selftest_bounded_wait",
     "ispa_selftest_exp2_poly", "ispa_set_attn_kernel", "ispa_kernel_launches", "ispa_last_error", "ispa_version",
 )
@@ -74,6 +75,8 @@ def lib() -> ctypes.CDLL:
         L.ispa_attn_split_i8.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                          ctypes.POINTER(CStats), vp, sz, vp]
         L.ispa_quantize_q_i8.argtypes = [vp, i, i, i, vp, vp, vp]
+        L.ispa_attn_split_ops.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.ispa_accum_ops.argtypes = [ctypes.POINTER(CStats), i, vp, vp, i, i, vp]
         L.ispa_k_blocks.argtypes = [ctypes.POINTER(AttnDesc)]
         L.ispa_quantize_k_i8.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp]
         L.ispa_accum_stats.argtypes = [ctypes.POINTER(CStats), vp, vp, i, i, vp, sz, vp]
@@ -183,6 +186,23 @@ def ispa_attn_split_i8(desc, q8, q_scale, k8, k_scale, v, o_full, lse_full, o_lo
                                   _p(lse_full), _p(o_loc), _p(lse_loc), _p(o_hist), _p(lse_hist), cs, _p(ws),
                                   0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "ispa_attn_split_i8")
+
+
+def ispa_attn_split_ops(desc, q, k, v, o_full, lse_full, a_ops, r_ops, o_loc=None, lse_loc=None, o_hist=None,
+                        lse_hist=None, stream=None) -> None:
+    """ispa_attn_split writing the statistics operands [n_q, D] to a_ops / r_ops instead of
+    accumulating them."""
+    rc = lib().ispa_attn_split_ops(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(o_full), _p(lse_full), _p(o_loc),
+                                   _p(lse_loc), _p(o_hist), _p(lse_hist), _p(a_ops), _p(r_ops), _stream(stream))
+    _check(rc, "ispa_attn_split_ops")
+
+
+def ispa_accum_ops(stats: Sequence[Stats], a_ops, r_ops, n_rows: int, dtype: int, stream=None) -> None:
+    """G += A^T A, C += A^T R, H += R^T R for len(stats) layers whose operands lie one after the
+    other in a_ops / r_ops ([layers][n_rows][D])."""
+    arr = (CStats * len(stats))(*[st.c() for st in stats])
+    _check(lib().ispa_accum_ops(arr, len(stats), _p(a_ops), _p(r_ops), n_rows, dtype, _stream(stream)),
+           "ispa_accum_ops")
 
 
 def ispa_attn_split_noalloc(desc, q, k, v, o_full, lse_full, o_loc=None, lse_loc=None, o_hist=None,

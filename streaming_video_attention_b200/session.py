@@ -11,6 +11,12 @@ weights and zeroes the statistics; the next transition replaces the old dW.
 The session owns the statistics buffers, dW, the error vector and the updated weights; the
 caller owns the KV cache (evicting the history of an L-layer is the caller freeing it).
 
+Statistics of a warmup chunk: each layer's full_attention(collect=True) writes its operands
+(A_loc, R) into the layer's slot of one [layers, n_q, D] buffer, and flush_stats() (called by
+the caller after the chunk's last layer, and by transition()) accumulates every pending layer
+in one launch -- the same sums, bit for bit, as accumulating layer by layer, without a short
+final wave per layer. batch_stats=False accumulates inside each call instead.
+
 Re-warmup trigger (the pages leave it open; reading): after a transition the F-layers still
 see their history, so full_attention(..., monitor=True) accumulates one chunk's statistics
 and live_errors() evaluates the error of the dW solved at the transition on them
@@ -48,7 +54,7 @@ class IspaSession:
     MIN_RISE = 0.02    # ... and above that minimum + MIN_RISE
 
     def __init__(self, layers: int, heads: int, head_dim: int, lam: float, K: int, dtype: str = "bf16",
-                 device: str = "cuda", w8a8: bool = False):
+                 device: str = "cuda", w8a8: bool = False, batch_stats: bool = True):
         self.layers, self.heads, self.head_dim = layers, heads, head_dim
         self.D = heads * head_dim
         self.lam, self.K = float(lam), int(K)
@@ -76,6 +82,10 @@ class IspaSession:
         self.monitor: List[Optional[ispa.Stats]] = [None] * layers
         self.live_history: List[Dict[int, float]] = []
         self._eps_live = torch.empty(layers, dtype=torch.float32, device=device)
+        # warmup statistics operands awaiting flush_stats(): layer -> rows
+        self.batch_stats = bool(batch_stats)
+        self._ops: Optional[Tuple[torch.Tensor, torch.Tensor]] = None
+        self._pending: Dict[int, int] = {}
 
     # ---------------------------------------------------------------- state
     def set_weights(self, W: Sequence[torch.Tensor]) -> None:
@@ -85,6 +95,7 @@ class IspaSession:
 
     def rewarm(self, stream=None) -> None:
         """Enter (or re-enter) the dual-stream warmup: every layer F, statistics zeroed."""
+        self._pending = {}
         for st in self.stats:
             ispa.ispa_stats_reset(st, stream)
         self.is_local = [0] * self.layers
@@ -107,9 +118,41 @@ class IspaSession:
         return self._ws_attn
 
     def reserve(self, max_n_q: int) -> None:
-        """Size the attention workspace up front (no allocation inside a timed loop)."""
+        """Size the attention workspace and the statistics operand buffer up front (no
+        allocation inside a timed loop)."""
         d = ispa.make_desc(max_n_q, 1, self.heads, self.head_dim, dtype=self.code)
         self._attn_ws(d)
+        if self.batch_stats:
+            self._ops_buffers(max_n_q)
+
+    def _ops_buffers(self, n_q: int) -> Tuple[torch.Tensor, torch.Tensor]:
+        if self._ops is None or self._ops[0].shape[1] < n_q:
+            shape = (self.layers, n_q, self.D)
+            self._ops = (torch.empty(shape, dtype=self.tdtype, device=self.device),
+                         torch.empty(shape, dtype=self.tdtype, device=self.device))
+        return self._ops
+
+    def flush_stats(self, stream=None) -> None:
+        """Accumulate the pending warmup operands: one launch per run of consecutive layers
+        with the same row count."""
+        if not self._pending:
+            return
+        a_all, r_all = self._ops
+        layers = sorted(self._pending)
+        start = 0
+        while start < len(layers):
+            end = start + 1
+            n = self._pending[layers[start]]
+            while end < len(layers) and layers[end] == layers[end - 1] + 1 and self._pending[layers[end]] == n:
+                end += 1
+            l0, l1 = layers[start], layers[end - 1] + 1
+            if a_all.shape[1] == n:
+                a, r = a_all[l0:l1], r_all[l0:l1]
+            else:   # operands were written into the first n rows of wider slots: pack them
+                a, r = a_all[l0:l1, :n].contiguous(), r_all[l0:l1, :n].contiguous()
+            ispa.ispa_accum_ops(self.stats[l0:l1], a, r, n, self.code, stream)
+            start = end
+        self._pending = {}
 
     # ---------------------------------------------------------------- per-layer calls
     def full_attention(self, layer: int, q, k, v, sink: Tuple[int, int], chunk: Tuple[int, int], o, lse,
@@ -126,6 +169,14 @@ class IspaSession:
             if self.monitor[layer] is None:
                 self.monitor[layer] = ispa.Stats(self.D, self.device)
             st = self.monitor[layer]
+        if collect and self.batch_stats:
+            if layer in self._pending:
+                self.flush_stats(stream)   # a second call for the layer before a flush
+            a_all, r_all = self._ops_buffers(n_q)
+            ispa.ispa_attn_split_ops(desc, q, k, v, o, lse, a_all[layer], r_all[layer], o_loc, lse_loc, o_hist,
+                                     lse_hist, stream=stream)
+            self._pending[layer] = n_q
+            return
         ws = self._attn_ws(desc) if st is not None else None
         ispa.ispa_attn_split(desc, q, k, v, o, lse, o_loc, lse_loc, o_hist, lse_hist, stats=st, ws=ws, stream=stream)
 
@@ -145,6 +196,7 @@ class IspaSession:
     def transition(self, K: Optional[int] = None, stream=None) -> List[int]:
         """Layer Absorb + Dynamic Layer Selection. Synchronises `stream` to read the errors."""
         K = self.K if K is None else K
+        self.flush_stats(stream)
         ispa.ispa_solve_absorb(self.stats, self.W0, self.code, self.lam, self.dW, self.eps, self.err_terms,
                                self.W_new, self.status, self.ws_solve, stream)
         eps = self.eps.to("cpu", non_blocking=False).tolist()

@@ -131,3 +131,17 @@ def test_i8_arguments_are_checked_before_any_launch():
     assert L.ispa_attn_split_i8(ctypes.byref(d64), *args) == ispa.ISPA_ERR_UNSUPPORTED
     no_qs = (fake, None) + args[2:]
     assert L.ispa_attn_split_i8(ctypes.byref(d128), *no_qs) == ispa.ISPA_ERR_INVALID_ARG
+
+
+def test_split_ops_and_accum_ops_arguments_are_checked_before_any_launch():
+    L = ispa.lib()
+    fake = ctypes.c_void_p(1 << 20)
+    d = ispa.make_desc(10, 100, 2, 128, (0, 10), (50, 100))
+    assert L.ispa_attn_split_ops(ctypes.byref(d), fake, fake, fake, fake, fake, None, None, None, None, None, fake,
+                                 None) == ispa.ISPA_ERR_INVALID_ARG              # a_ops missing
+    assert L.ispa_accum_ops(None, 1, fake, fake, 10, ispa.ISPA_BF16, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_accum_ops(None, 0, None, None, 0, ispa.ISPA_BF16, None) == ispa.ISPA_ERR_INVALID_ARG
+    st = (ispa.CStats * 2)(ispa.CStats(256, 1 << 20, 1 << 20, 1 << 20, 1 << 20),
+                           ispa.CStats(128, 1 << 20, 1 << 20, 1 << 20, 1 << 20))
+    assert L.ispa_accum_ops(st, 2, fake, fake, 10, ispa.ISPA_BF16, None) == ispa.ISPA_ERR_INVALID_ARG   # D differs
+    assert L.ispa_accum_ops(st, 0, None, None, 10, ispa.ISPA_BF16, None) == ispa.ISPA_OK                 # no layers

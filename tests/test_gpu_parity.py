@@ -295,3 +295,39 @@ def test_full_size_1p3b_layer_sampled_rows():
     assert np.all(np.diag(G) >= 0) and np.all(np.diag(H) >= 0)
     a = got["A_loc"].reshape(cfg.n_q, -1)
     assert abs(np.trace(G) - np.sum(a * a)) < 1e-4 * np.sum(a * a)
+
+
+def test_batched_statistics_equal_fused_bit_for_bit():
+    """Three layers' warmup calls: ispa_attn_split with fused statistics, layer by layer,
+    against ispa_attn_split_ops + one ispa_accum_ops launch for all three: the same tiles in the
+    same reduction order, so G, C, H and the outputs are identical bit for bit. A fourth layer
+    with another row count exercises a second launch."""
+    heads, hd = 2, 128
+    D = heads * hd
+    n_q, n_kv, sink, chunk = 300, 1000, (0, 100), (700, 1000)
+    fused = [ispa.Stats(D) for _ in range(3)]
+    batched = [ispa.Stats(D) for _ in range(3)]
+    a_all = torch.empty((3, n_q, D), dtype=torch.bfloat16, device="cuda")
+    r_all = torch.empty_like(a_all)
+    desc = ispa.make_desc(n_q, n_kv, heads, hd, sink, chunk, dtype=ispa.ISPA_BF16)
+    ws = ispa.alloc_workspace(ispa.workspace_bytes(desc, 0, 0))
+    for l in range(3):
+        q, k, v = (to_device(x, "bf16") for x in _attn_case(90 + l, n_q, n_kv, heads, hd, "bf16"))
+        o1, o2 = (torch.empty((n_q, heads, hd), dtype=torch.bfloat16, device="cuda") for _ in range(2))
+        l1, l2 = (torch.empty((heads, n_q), dtype=torch.float32, device="cuda") for _ in range(2))
+        ispa.ispa_attn_split(desc, q, k, v, o1, l1, stats=fused[l], ws=ws)
+        ispa.ispa_attn_split_ops(desc, q, k, v, o2, l2, a_all[l], r_all[l])
+        torch.cuda.synchronize()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    ispa.ispa_accum_ops(batched, a_all, r_all, n_q, ispa.ISPA_BF16)
+    torch.cuda.synchronize()
+    assert ispa.ispa_device_status() == ispa.ISPA_OK
+    for f, b in zip(fused, batched):
+        for name in ("G", "C", "H"):
+            assert torch.equal(getattr(f, name), getattr(b, name)), name
+        assert int(f.rows.item()) == int(b.rows.item()) == n_q
+    # accumulating again adds on top (a second warmup chunk), still identical
+    ispa.ispa_accum_ops(batched[1:2], a_all[1:2], r_all[1:2], n_q, ispa.ISPA_BF16)
+    ispa.ispa_accum_stats(fused[1], None, None, 0, ispa.ISPA_BF16)   # no rows: nothing changes
+    torch.cuda.synchronize()
+    assert int(batched[1].rows.item()) == 2 * n_q
