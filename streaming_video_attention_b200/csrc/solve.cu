@@ -34,70 +34,89 @@ __global__ void fill_shifted_kernel(PtrBatch src, PtrBatch dst, int D, float lam
     }
 }
 
-__global__ void potrf_diag_kernel(PtrBatch M, int D, int k0, int *status) {
-    __shared__ float A[NB][NB + 1];
+// Cholesky factor of the NB x NB diagonal block at (k0, k0), in place (lower triangle). One
+// CTA of NB threads per layer; thread i holds row i of the block in registers (the column loop
+// is unrolled so that every index is a constant). Column j: the pivot's square root, then each
+// row below scales its element of column j and publishes it, then each row subtracts its
+// rank-1 update from its remaining lower-triangle elements.
+__global__ void __launch_bounds__(NB) potrf_diag_kernel(PtrBatch M, int D, int k0, int *status) {
+    __shared__ float col[NB];
+    __shared__ float piv;
     const int z = blockIdx.x;
     float *Mz = static_cast<float *>(M.p[z]);
-    const int tid = threadIdx.x, nt = blockDim.x;
-    for (int idx = tid; idx < NB * NB; idx += nt) {
-        const int i = idx / NB, j = idx % NB;
-        A[i][j] = Mz[(size_t)(k0 + i) * D + k0 + j];
+    const int i = threadIdx.x;
+    float a[NB];
+    const float *row = Mz + (size_t)(k0 + i) * D + k0;
+#pragma unroll
+    for (int c = 0; c < NB; c += 4) {
+        const float4 v = *reinterpret_cast<const float4 *>(row + c);
+        a[c] = v.x; a[c + 1] = v.y; a[c + 2] = v.z; a[c + 3] = v.w;
     }
-    __syncthreads();
+    bool bad = false;
+#pragma unroll
     for (int j = 0; j < NB; ++j) {
-        if (tid == 0) {
-            float d = A[j][j];
+        if (i == j) {
+            float d = a[j];
             if (!(d > 0.f)) {
-                status[z] = ISPA_ERR_NOT_SPD;
+                bad = true;
                 d = __int_as_float(0x7fc00000);
             } else {
                 d = sqrtf(d);
             }
-            A[j][j] = d;
+            a[j] = d;
+            piv = d;
         }
         __syncthreads();
-        for (int i = j + 1 + tid; i < NB; i += nt) A[i][j] = A[i][j] / A[j][j];
-        __syncthreads();
-        const int w = NB - j - 1;
-        for (int idx = tid; idx < w * w; idx += nt) {
-            const int r = j + 1 + idx / w, c = j + 1 + idx % w;
-            if (c <= r) A[r][c] -= A[r][j] * A[c][j];
+        if (i > j) {
+            a[j] = a[j] / piv;
+            col[i] = a[j];
         }
         __syncthreads();
+        if (i > j) {
+#pragma unroll
+            for (int k = j + 1; k < NB; ++k)
+                if (k <= i) a[k] -= a[j] * col[k];
+        }
     }
-    for (int idx = tid; idx < NB * NB; idx += nt) {
-        const int i = idx / NB, j = idx % NB;
-        if (j <= i) Mz[(size_t)(k0 + i) * D + k0 + j] = A[i][j];
-    }
+    if (bad) status[z] = ISPA_ERR_NOT_SPD;
+    float *out = Mz + (size_t)(k0 + i) * D + k0;
+#pragma unroll
+    for (int c = 0; c < NB; ++c)
+        if (c <= i) out[c] = a[c];
 }
 
-// Rows below the diagonal block: L21 = A21 L11^-T (row-wise forward substitution).
-__global__ void trsm_panel_kernel(PtrBatch M, int D, int k0) {
-    __shared__ float Lk[NB][NB + 1];
-    __shared__ float Xs[NB][NB + 1];
+// Rows below the diagonal block: L21 = A21 L11^-T (row-wise forward substitution). One CTA of
+// NB threads per NB rows; thread i holds its row of A21 in registers (unrolled loops, constant
+// indices), the factored diagonal block sits in shared memory and is read by broadcast.
+__global__ void __launch_bounds__(NB) trsm_panel_kernel(PtrBatch M, int D, int k0) {
+    __shared__ __align__(16) float Lk[NB][NB];
     const int z = blockIdx.y;
     float *Mz = static_cast<float *>(M.p[z]);
-    const int r0 = k0 + NB + blockIdx.x * NB;
-    const int tid = threadIdx.x, nt = blockDim.x;
-    for (int idx = tid; idx < NB * NB; idx += nt) {
-        const int i = idx / NB, j = idx % NB;
-        Lk[i][j] = j <= i ? Mz[(size_t)(k0 + i) * D + k0 + j] : 0.f;
-        Xs[i][j] = (r0 + i < D) ? Mz[(size_t)(r0 + i) * D + k0 + j] : 0.f;
-    }
-    __syncthreads();
-    if (tid < NB && r0 + tid < D) {
-        const int row = tid;
-        for (int j = 0; j < NB; ++j) {
-            float x = Xs[row][j];
-            for (int c = 0; c < j; ++c) x -= Xs[row][c] * Lk[j][c];
-            Xs[row][j] = x / Lk[j][j];
+    const int i = threadIdx.x;
+    const int r = k0 + NB + blockIdx.x * NB + i;
+    // column i of the diagonal block: coalesced reads, conflict-free stores
+    for (int rr = 0; rr < NB; ++rr) Lk[rr][i] = i <= rr ? Mz[(size_t)(k0 + rr) * D + k0 + i] : 0.f;
+    float x[NB];
+    if (r < D) {
+        const float *row = Mz + (size_t)r * D + k0;
+#pragma unroll
+        for (int c = 0; c < NB; c += 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(row + c);
+            x[c] = v.x; x[c + 1] = v.y; x[c + 2] = v.z; x[c + 3] = v.w;
         }
     }
     __syncthreads();
-    for (int idx = tid; idx < NB * NB; idx += nt) {
-        const int i = idx / NB, j = idx % NB;
-        if (r0 + i < D) Mz[(size_t)(r0 + i) * D + k0 + j] = Xs[i][j];
+    if (r >= D) return;
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+        float v = x[j];
+#pragma unroll
+        for (int c = 0; c < j; ++c) v -= x[c] * Lk[j][c];
+        x[j] = v / Lk[j][j];
     }
+    float *out = Mz + (size_t)r * D + k0;
+#pragma unroll
+    for (int c = 0; c < NB; c += 4) *reinterpret_cast<float4 *>(out + c) = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
 }
 
 // X_k = L_kk^-1 X_k (forward) or L_kk^-T X_k (backward) for the NB rows of block k,
@@ -341,11 +360,11 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
     const int nblk = D / NB;
     for (int kb = 0; kb < nblk; ++kb) {
         const int k0 = kb * NB;
-        potrf_diag_kernel<<<batch, 256, 0, s>>>(M, D, k0, status); note_launch();
+        potrf_diag_kernel<<<batch, NB, 0, s>>>(M, D, k0, status); note_launch();
         ISPA_TRY(cudaGetLastError());
         const int rest = D - k0 - NB;
         if (rest <= 0) break;
-        trsm_panel_kernel<<<dim3((rest + NB - 1) / NB, batch), 256, 0, s>>>(M, D, k0); note_launch();
+        trsm_panel_kernel<<<dim3((rest + NB - 1) / NB, batch), NB, 0, s>>>(M, D, k0); note_launch();
         ISPA_TRY(cudaGetLastError());
         GemmDesc d{rest, rest, NB, D, D, D, true, true, ElemType::F32, ElemType::F32, ElemType::F32, -1.f, 1.f,
                    true, batch};
