@@ -23,44 +23,57 @@
 namespace ispa {
 namespace {
 
-constexpr int kTile = 128;         // output tile (both dimensions)
+constexpr int kTile = 128;         // output tile rows; column blocks of 128
 constexpr int kKRows = 64;         // token rows per stage
-constexpr int kStages = 3;
 constexpr int kThreads = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-constexpr int kOperandBytes = kKRows * kTile * 2;          // 16 KB: two 64x64 boxes
-constexpr int kStageBytes = 2 * kOperandBytes;
-constexpr int kBarOff = kStages * kStageBytes;
-constexpr int kSmemAlloc = kBarOff + 256 + 1024;
+
+// Tiles of 128 x kN outputs: kN = 256 halves the A-operand bytes per flop (2 stages of 48 KB,
+// two CTAs per SM); kN = 128 for D not a multiple of 256 (3 stages of 32 KB).
+template <int kN>
+struct StatsCfg {
+    static constexpr int kStages = kN == 256 ? 2 : 3;
+    static constexpr int kABytes = kKRows * kTile * 2;           // 16 KB: two 64x64 boxes
+    static constexpr int kBBytes = kKRows * kN * 2;              // kN / 64 boxes
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kBarOff = kStages * kStageBytes;
+    static constexpr int kSmemAlloc = kBarOff + 256 + 1024;
+    static constexpr int kBlocks = kN / kTile;                   // 128-column blocks per tile
+};
 
 struct StatsParams {
     float *out[kMaxBatch][3];   // per layer: G, C, H
     int D, n;
     int nb;             // D / 128
-    int n_sym;          // upper-triangle tiles per symmetric matrix: nb*(nb+1)/2
+    int ng;             // column groups per row: D / kN
+    int n_sym;          // tiles per symmetric matrix that touch its upper triangle
     int *err_flag;
 };
 
-// Work item -> (matrix, tile row bi, tile column bj). Items 0..n_sym-1: G, then C (nb*nb),
-// then H (n_sym).
-__device__ __forceinline__ void decode_item(int item, int nb, int n_sym, int &mat, int &bi, int &bj) {
+// Work item -> (matrix, tile row bi, column group g). Items 0..n_sym-1: G, then C (nb*ng),
+// then H (n_sym). A symmetric matrix keeps, in row bi, the groups whose last column block
+// is on or above the diagonal: g >= bi / kBlocks.
+template <int kBlocks>
+__device__ __forceinline__ void decode_item(int item, int nb, int ng, int n_sym, int &mat, int &bi, int &g) {
     int t;
     if (item < n_sym) { mat = 0; t = item; }
-    else if (item < n_sym + nb * nb) { mat = 1; bi = (item - n_sym) / nb; bj = (item - n_sym) % nb; return; }
-    else { mat = 2; t = item - n_sym - nb * nb; }
-    // t-th upper-triangle tile in row-major order
+    else if (item < n_sym + nb * ng) { mat = 1; bi = (item - n_sym) / ng; g = (item - n_sym) % ng; return; }
+    else { mat = 2; t = item - n_sym - nb * ng; }
     int r = 0;
-    while (t >= nb - r) { t -= nb - r; ++r; }
+    while (t >= ng - r / kBlocks) { t -= ng - r / kBlocks; ++r; }
     bi = r;
-    bj = r + t;
+    g = r / kBlocks + t;
 }
 
+template <int kN>
 __global__ void __launch_bounds__(kThreads, 2)
 stats_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmR,
                         const StatsParams p) {
+    using Cfg = StatsCfg<kN>;
+    constexpr int kStages = Cfg::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kBarOff);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOff);
     uint64_t *empty = full + kStages;
     uint64_t *acc_bar = empty + kStages;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_bar + 1);
@@ -68,8 +81,8 @@ stats_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int layer = blockIdx.y;
-    int mat, bi, bj;
-    decode_item(blockIdx.x, p.nb, p.n_sym, mat, bi, bj);
+    int mat, bi, g;
+    decode_item<Cfg::kBlocks>(blockIdx.x, p.nb, p.ng, p.n_sym, mat, bi, g);
     const CUtensorMap *mapA = (mat == 2) ? &tmR : &tmA;   // left operand: A for G and C, R for H
     const CUtensorMap *mapB = (mat == 0) ? &tmA : &tmR;   // right operand: A for G, R for C and H
     const int n_k = (p.n + kKRows - 1) / kKRows;
@@ -84,7 +97,7 @@ stats_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         ptx::fence_barrier_init();
     }
     if (warp == 1) {
-        ptx::tmem_alloc(tmem_slot, 128);
+        ptx::tmem_alloc(tmem_slot, kN);
         ptx::tmem_relinquish();
     }
     ptx::tc_fence_before();
@@ -106,15 +119,16 @@ stats_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
             const uint32_t ph = (kt / kStages) & 1;
             ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&empty[s], ph ^ 1, kWaitLimitNs, p.err_flag, abort_flag));
             if (!ok) break;
-            uint8_t *base = smem + s * kStageBytes;
-            ptx::mbar_arrive_expect_tx_warp(&full[s], kStageBytes);
+            uint8_t *base = smem + s * Cfg::kStageBytes;
+            ptx::mbar_arrive_expect_tx_warp(&full[s], Cfg::kStageBytes);
 #pragma unroll
-            for (int b = 0; b < 2; ++b) {
+            for (int b = 0; b < 2; ++b)
                 ptx::tma_load_3d_warp(base + b * (kKRows * 128), mapA, &full[s], bi * kTile + b * 64, kt * kKRows,
                                       layer, pol);
-                ptx::tma_load_3d_warp(base + kOperandBytes + b * (kKRows * 128), mapB, &full[s], bj * kTile + b * 64,
+#pragma unroll
+            for (int b = 0; b < kN / 64; ++b)
+                ptx::tma_load_3d_warp(base + Cfg::kABytes + b * (kKRows * 128), mapB, &full[s], g * kN + b * 64,
                                       kt * kKRows, layer, pol);
-            }
             issued = kt;
         }
         if (!ok) {
@@ -122,7 +136,7 @@ stats_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                 ptx::mbar_wait_bounded(&full[kt % kStages], (kt / kStages) & 1, kWaitLimitNs, nullptr, nullptr);
         }
     } else if (warp == 1) {
-        constexpr uint32_t idesc = ptx::make_idesc_bf16(kTile, kTile, true, true);
+        constexpr uint32_t idesc = ptx::make_idesc_bf16(kTile, kN, true, true);
         const uint32_t sbase = ptx::smem_u32(smem);
         bool ok = true;
         for (int kt = 0; kt < n_k && ok; ++kt) {
@@ -131,10 +145,11 @@ stats_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                             ptx::mbar_wait_bounded(&full[s], (kt / kStages) & 1, kWaitLimitNs, p.err_flag, abort_flag));
             if (!ok) break;
             ptx::tc_fence_after();
-            const uint32_t a0 = sbase + s * kStageBytes;
-            const uint32_t b0 = a0 + kOperandBytes;
+            const uint32_t a0 = sbase + s * Cfg::kStageBytes;
+            const uint32_t b0 = a0 + Cfg::kABytes;
 #pragma unroll
             for (int kk = 0; kk < kKRows / 16; ++kk) {
+                // both operands MN-major: 64-column groups kKRows * 128 bytes apart
                 const uint64_t da = ptx::make_sdesc_sw128(a0 + kk * 2048, kKRows * 128, 1024);
                 const uint64_t db = ptx::make_sdesc_sw128(b0 + kk * 2048, kKRows * 128, 1024);
                 ptx::umma_f16_ss_warp(tmem, da, db, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
@@ -158,15 +173,16 @@ stats_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
             const size_t D = p.D;
             const int gi = bi * kTile + r;
             const bool sym = (mat != 1);
-            const bool diag = sym && bi == bj;
 #pragma unroll 1
-            for (int c = 0; c < kTile / 32; ++c) {
+            for (int c = 0; c < kN / 32; ++c) {
+                const int gj0 = g * kN + c * 32;
+                const int bj = gj0 / kTile;                 // 128-column block of this chunk
+                if (sym && bj < bi) continue;               // below the diagonal: the mirror holds it
                 uint32_t v[32];
                 ptx::tmem_ld32(tmem + lane_off + c * 32, v);
                 ptx::tmem_wait_ld();
-                const int gj0 = bj * kTile + c * 32;
                 float *rowp = M + (size_t)gi * D + gj0;
-                if (!diag) {
+                if (!(sym && bj == bi)) {
 #pragma unroll
                     for (int q = 0; q < 32; q += 4) {
                         float4 o = *reinterpret_cast<const float4 *>(rowp + q);
@@ -183,7 +199,7 @@ stats_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
                         }
                     }
                 } else {
-                    // diagonal tile: the upper triangle (j >= i) is updated and mirrored
+                    // diagonal block: the upper triangle (j >= i) is updated and mirrored
 #pragma unroll
                     for (int q = 0; q < 32; ++q) {
                         const int gj = gj0 + q;
@@ -202,7 +218,7 @@ stats_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
     __syncthreads();
     if (warp == 1) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem, 128);
+        ptx::tmem_dealloc(tmem, kN);
     }
 }
 
@@ -236,6 +252,20 @@ bool make_panel_map(CUtensorMap *m, const void *ptr, int layers, int n, int D) {
 }
 
 }  // namespace
+
+template <int kN>
+cudaError_t launch_tiles(const CUtensorMap &ma, const CUtensorMap &mr, StatsParams p, int layers, cudaStream_t s) {
+    using Cfg = StatsCfg<kN>;
+    p.ng = p.D / kN;
+    p.n_sym = 0;
+    for (int bi = 0; bi < p.nb; ++bi) p.n_sym += p.ng - bi / Cfg::kBlocks;
+    cudaError_t e = cudaFuncSetAttribute(stats_gemm_sm100_kernel<kN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg::kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    const int items = 2 * p.n_sym + p.nb * p.ng;
+    stats_gemm_sm100_kernel<kN><<<dim3(items, layers), kThreads, Cfg::kSmemAlloc, s>>>(ma, mr, p); note_launch();
+    return cudaGetLastError();
+}
 
 // Layers [0, layers) with operands a_loc, r = [layers][n][D] contiguous and outputs
 // G[l], C[l], H[l]; layers <= kMaxBatch.
@@ -271,13 +301,9 @@ cudaError_t launch_stats_bf16_layers(const void *a_loc, const void *r, int layer
     }
     p.D = D; p.n = n;
     p.nb = D / kTile;
-    p.n_sym = p.nb * (p.nb + 1) / 2;
     p.err_flag = err_flag;
-    cudaError_t e = cudaFuncSetAttribute(stats_gemm_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
-    if (e != cudaSuccess) return e;
-    const int items = 2 * p.n_sym + p.nb * p.nb;
-    stats_gemm_sm100_kernel<<<dim3(items, layers), kThreads, kSmemAlloc, s>>>(ma, mr, p); note_launch();
-    return cudaGetLastError();
+    if (D % 256 == 0) return launch_tiles<256>(ma, mr, p, layers, s);
+    return launch_tiles<128>(ma, mr, p, layers, s);
 }
 
 cudaError_t launch_stats_bf16(const void *a_loc, const void *r, int n, int D, float *G, float *C, float *H,
