@@ -53,3 +53,46 @@ def test_kv_cache_accounting():
     long_b = kv_cache_bytes([0] * 30, 119, 3, 1, 1560, 1536)
     long_a = kv_cache_bytes([1] * 15 + [0] * 15, 119, 3, 1, 1560, 1536)
     assert 0.48 < (long_b - long_a) / long_b < 0.5
+
+
+def test_flush_stats_groups_consecutive_layers_with_equal_rows(monkeypatch):
+    """Warmup calls only write operands; flush_stats() accumulates each run of consecutive
+    layers with the same row count in one call, packing rows when a slot is wider; a second
+    call for a pending layer flushes first; transition() flushes before solving."""
+    import torch
+    from streaming_video_attention_b200 import ispa
+
+    calls = []
+    monkeypatch.setattr(ispa, "ispa_attn_split_ops", lambda desc, q, k, v, o, lse, a, r, *args, **kw:
+                        calls.append(("ops", desc.n_q, a.shape, a.data_ptr())))
+    monkeypatch.setattr(ispa, "ispa_accum_ops", lambda stats, a, r, n, code, stream=None:
+                        calls.append(("accum", [id(s) for s in stats], tuple(a.shape), a.is_contiguous(), n)))
+    monkeypatch.setattr(ispa, "alloc_workspace", lambda nbytes, device="cuda": None)   # no solve here
+    monkeypatch.setattr(ispa, "ispa_stats_reset", lambda st, stream=None: None)
+    sess = IspaSession(5, 2, 128, 1e-2, 2, "bf16", device="cpu")
+    ids = [id(s) for s in sess.stats]
+
+    def call(layer, n_q):
+        q = torch.zeros((n_q, 2, 128), dtype=torch.bfloat16)
+        kv = torch.zeros((300, 2, 128), dtype=torch.bfloat16)
+        sess.full_attention(layer, q, kv, kv, (0, 50), (200, 300), None, None, collect=True)
+
+    for layer, n in ((0, 10), (1, 10), (2, 10), (3, 8), (4, 10)):
+        call(layer, n)
+    assert [c[0] for c in calls] == ["ops"] * 5
+    calls.clear()
+    sess.flush_stats()
+    assert calls == [("accum", ids[0:3], (3, 10, 256), True, 10),
+                     ("accum", ids[3:4], (1, 8, 256), True, 8),
+                     ("accum", ids[4:5], (1, 10, 256), True, 10)]
+    calls.clear()
+    sess.flush_stats()                                   # nothing pending: no call
+    assert calls == []
+    call(2, 10)
+    call(2, 10)                                          # the same layer again: flush in between
+    assert [c[0] for c in calls] == ["ops", "accum", "ops"]
+    assert calls[1][1] == ids[2:3]
+    sess.rewarm()                                        # pending operands are dropped
+    calls.clear()
+    sess.flush_stats()
+    assert calls == []
