@@ -93,8 +93,9 @@ def test_split_attention_edge_sizes():
 
 # ------------------------------------------------------------------ statistics (a2)
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
-def test_accum_stats_matches_oracle_on_identical_operands(dtype):
-    n, D = 777, 256
+@pytest.mark.parametrize("D", [128, 256, 384, 512])    # bf16: 128-wide tiles for 128, 384; 256-wide for 256, 512
+def test_accum_stats_matches_oracle_on_identical_operands(dtype, D):
+    n = 777
     a_loc = synth.normal_tensor(7, (10,), (n, D), dtype, std=0.05)
     a_full = synth.normal_tensor(7, (11,), (n, D), dtype, std=0.05)
     st = ispa.Stats(D)
