@@ -158,7 +158,8 @@ class IspaSession:
     def full_attention(self, layer: int, q, k, v, sink: Tuple[int, int], chunk: Tuple[int, int], o, lse,
                        collect: bool, o_loc=None, lse_loc=None, o_hist=None, lse_hist=None, stream=None,
                        monitor: bool = False) -> None:
-        """An F-layer call; with collect=True (warmup) the ridge statistics accumulate too; with
+        """An F-layer call; with collect=True (warmup) the call's statistics operands are kept for
+        flush_stats() (batch_stats=True) or accumulated at once (batch_stats=False); with
         monitor=True (after a transition) this chunk's statistics go to the layer's monitor."""
         n_q, n_kv = q.shape[0], k.shape[0]
         desc = ispa.make_desc(n_q, n_kv, self.heads, self.head_dim, sink, chunk, dtype=self.code)
