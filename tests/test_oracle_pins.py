@@ -260,6 +260,39 @@ def test_error_traces_match_direct_norms():
         assert abs(e["eps"] - E2 / T2) < 1e-9
 
 
+def test_project_golden_two_heads():
+    """y = A W for A [n, heads, head_dim] (column h*head_dim + j) and W stored [D_in, D_out],
+    against a hand-computed case whose W is neither square nor symmetric."""
+    g = _golden("project_two_heads.json")
+    A, W = np.array(g["A"]), np.array(g["W"])
+    np.testing.assert_array_equal(oracle.project(A, W), np.array(g["y"]))
+
+
+def test_project_residual_is_the_error_numerator():
+    """||project(A_loc, W + dW) - project(A_full, W)||^2 summed over the warmup equals E^2 of
+    the trace form (itself pinned to direct norms above), for attention outputs of a real
+    split call, several heads and a non-symmetric W: a transposed W or a dropped dW in
+    project would change the left side only."""
+    n_q, n_kv, h, d = 12, 40, 3, 4
+    D = h * d
+    rng = np.random.default_rng(130)
+    W = rng.standard_normal((D, D)) / math.sqrt(D)
+    assert np.linalg.norm(W - W.T) > 0.5 * np.linalg.norm(W)
+    st = oracle.stats_init(D)
+    chunks = []
+    for t in range(3):
+        q, k, v = (rng.standard_normal(s) for s in ((n_q, h, d), (n_kv, h, d), (n_kv, h, d)))
+        res = oracle.split_attention(q, k, v, (0, 6), (28, 40), 1 / math.sqrt(d))
+        oracle.stats_update(st, res["A_loc"], res["A_full"], "fp32")
+        chunks.append(res)
+    for dW in (oracle.absorb_solve(st["G"], st["C"], W, 0.05), rng.standard_normal((D, D)) / D):
+        e = oracle.reconstruction_error(st["G"], st["C"], st["H"], W, dW)
+        E2 = sum(np.sum((oracle.project(c["A_loc"], W + dW) - oracle.project(c["A_full"], W)) ** 2) for c in chunks)
+        T2 = sum(np.sum(oracle.project(c["A_full"], W) ** 2) for c in chunks)
+        assert abs(E2 - e["E2"]) < 1e-10 * T2
+        assert abs(T2 - e["T2"]) < 1e-10 * T2
+
+
 def test_solution_minimises_the_ridge_objective():
     n, D, lam = 30, 5, 0.2
     a = _rand((n, D), 120)
