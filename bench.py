@@ -50,6 +50,8 @@ def parse_args(argv=None):
                     help="timed steps of the end-to-end leg (its first step's copies are the pipeline fill)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-shapes", action="store_true",
+                    help="skip the one-layer call timings of the 1.3B, long-history and 14B shapes")
     ap.add_argument("--cpu-rows", type=int, default=512)
     ap.add_argument("--mode", choices=["episode", "call", "local", "solve"], default="episode",
                     help="episode: the full step (default). call / local / solve: one layer's fused split "
@@ -65,33 +67,28 @@ def parse_args(argv=None):
     return ap.parse_args(argv)
 
 
-# DRAM bytes per layer call at the 1.3B shape (dram__bytes_read.sum + dram__bytes_write.sum, one
-# ncu capture per kernel, the statistics GEMM on a one-layer launch; profiles/attn_split_2g_sm100_1p3b_layer.md,
-# profiles/attn_split_sm100_1p3b_layer.md and profiles/stats_gemm_sm100_1p3b_layer.md). A figure
-# holds only for the kernel sources it was taken from: any other source reports null.
-_PTX = ("streaming_video_attention_b200/csrc/ptx.cuh",
-        "0353fca5187d1129c0e7936a8baa86b17e79672c07a933ea5a5f127e77d94af0")
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum, ncu) per launch of the kernels the
+# roofline object describes, each tied to the sha256 of the sources it was captured from: a figure
+# is reported only while those sources are unchanged, otherwise the line's traffic is null.
+# The path is the episode's: one ispa_attn_split_ops launch per warmup layer call and one batched
+# ispa_accum_ops launch per chunk, whose bytes are charged to the chunk's layers equally.
+# None: not yet captured for the current sources.
 CAPTURED_TRAFFIC = {
     "workload": "1p3b_bf16",
-    "stats": (49.6e6, dict([_PTX, ("streaming_video_attention_b200/csrc/stats_sm100.cu",
-                                   "8958228b298ce923c00635e441f0bce98ae0869e773a3171b70c6b0dedb1aa8f")])),
-    "attention": {
-        "single": (276.8e6, dict([_PTX, ("streaming_video_attention_b200/csrc/attn_sm100.cu",
-                                         "d529641e0543692a54f49c730bd94b44bb0d8126a3e4bdeb0cd0e0acf6b451df")])),
-        "two_group": (281.2e6, dict([_PTX, ("streaming_video_attention_b200/csrc/attn2g_sm100.cu",
-                                            "3bed3806f2e152d01cb932a529d3f79da812540a4b19e6fbb52febc93f129433")])),
-    },
+    "attention": {"two_group": (None, {})},
+    "stats_per_layer": (None, {}),
 }
 
 
 def captured_traffic(cfg, attn_kernel: str):
-    """DRAM bytes of one fused call (attention kernel + statistics GEMM), or None."""
+    """DRAM bytes per warmup layer call on the timed path (attention launch + its share of the
+    chunk's statistics launch), or None."""
     import hashlib
     kernel = "two_group" if attn_kernel == "auto" else attn_kernel
     if cfg.name != CAPTURED_TRAFFIC["workload"] or kernel not in CAPTURED_TRAFFIC["attention"]:
         return None
     total = 0.0
-    for nbytes, sources in (CAPTURED_TRAFFIC["attention"][kernel], CAPTURED_TRAFFIC["stats"]):
+    for nbytes, sources in (CAPTURED_TRAFFIC["attention"][kernel], CAPTURED_TRAFFIC["stats_per_layer"]):
         if nbytes is None:
             return None
         for rel, digest in sources.items():
@@ -100,6 +97,9 @@ def captured_traffic(cfg, attn_kernel: str):
                     return None
         total += nbytes
     return total
+
+
+DATASHEET_DENSE_BF16_TFLOPS = 2250.0   # B200 dense bf16 (the 2:4-sparse figure halved)
 
 
 def peaks():
@@ -321,9 +321,11 @@ def physical_gpu_index(local_rank: int) -> int:
 
 
 # --------------------------------------------------------------------------- CPU oracle sample
-def oracle_sample(cfg, rows: int):
-    """Time the oracle on a bounded sample: `rows` query rows of one layer's last warmup call
-    (split attention over explicit masks + statistics). Returns (seconds, threads, note)."""
+def oracle_parts(cfg, rows: int) -> dict:
+    """Time the oracle on one bounded sample of the episode's calls: `rows` query rows of one
+    layer's last warmup call -- the split attention over explicit masks, and the statistics of
+    those rows -- and the same rows through one L-layer call (attention over the sink and chunk
+    rows, projection with W + dW). Returns seconds per part and the sample's KV row counts."""
     import oracle
     t = cfg.warmup_chunks - 1
     frames = synth.cache_frames(cfg, t)
@@ -331,34 +333,60 @@ def oracle_sample(cfg, rows: int):
     q = synth.chunk_q(cfg, 0, t)[:rows]
     k = synth.kv_tensor(cfg, 0, frames, "k")
     v = synth.kv_tensor(cfg, 0, frames, "v")
+    s0 = cfg.chunk_start_frame(t)
+    loc = list(range(cfg.sink_frames)) + list(range(s0, s0 + cfg.chunk_frames))
+    pos = {f: i for i, f in enumerate(frames)}
+    loc_rows = np.concatenate([np.arange(pos[f] * cfg.tpf, (pos[f] + 1) * cfg.tpf) for f in loc])
+    W = synth.w_out(cfg, 0).astype(np.float64)
     t0 = time.perf_counter()
     res = oracle.split_attention(q, k, v, (lay["sink_begin"], lay["sink_end"]), (lay["chunk_begin"], lay["chunk_end"]),
                                  cfg.scale)
+    t1 = time.perf_counter()
     st = oracle.stats_init(cfg.D)
     oracle.stats_update(st, res["A_loc"], res["A_full"], cfg.dtype)
-    dt = time.perf_counter() - t0
-    return dt, lay["n_kv"]
+    t2 = time.perf_counter()
+    A, _ = oracle.local_attention(q, k[loc_rows], v[loc_rows], cfg.scale)
+    oracle.project(A, W)
+    t3 = time.perf_counter()
+    return {"attn": t1 - t0, "stats": t2 - t1, "local": t3 - t2, "n_kv": lay["n_kv"], "n_loc": len(loc_rows),
+            "rows": rows}
 
 
-def oracle_value(cfg, dt: float, rows: int, n_kv_sample: int, wl_calls) -> float:
-    """Extrapolate the sample to one episode (linear in query rows and KV rows per call) and
-    express it in the step's unit."""
+def oracle_transition(cfg) -> float:
+    """The oracle's transition in full: absorb solve (dense LU) + reconstruction error for every
+    layer and the selection, on statistics of three warmup chunks' rows built once from seeded
+    operands outside the timing. Returns seconds."""
+    import oracle
+    n = cfg.warmup_chunks * cfg.n_q
+    a = synth.normal_tensor(5, (1,), (n, cfg.D), cfg.dtype, std=0.05).astype(np.float64)
+    r = synth.normal_tensor(5, (2,), (n, cfg.D), cfg.dtype, std=0.05).astype(np.float64)
+    st = oracle.stats_init(cfg.D)
+    oracle.stats_update(st, a.reshape(n, cfg.heads, -1), (a + r).reshape(n, cfg.heads, -1), cfg.dtype)
+    Ws = [synth.w_out(cfg, l).astype(np.float64) for l in range(cfg.layers)]
+    t0 = time.perf_counter()
+    eps = []
+    for W in Ws:
+        dW = oracle.absorb_solve(st["G"], st["C"], W, cfg.lam)
+        eps.append(oracle.reconstruction_error(st["G"], st["C"], st["H"], W, dW)["eps"])
+    oracle.select_layers(eps, cfg.K)
+    return time.perf_counter() - t0
+
+
+def oracle_episode_seconds(cfg, parts: dict, t_transition: float) -> float:
+    """The oracle's time for one episode: each warmup call's attention scaled from the sample
+    linearly in query rows and KV rows, its statistics linearly in query rows (their cost does
+    not depend on the KV rows), the transition as timed, then the post-transition chunk (F-layers:
+    split attention; L-layers: local attention + projection)."""
+    per_row = cfg.n_q / parts["rows"]
     est = 0.0
-    for n_kv in wl_calls:
-        est += dt * (cfg.n_q / rows) * (n_kv / n_kv_sample)
-    tokens = (cfg.warmup_chunks + 1) * cfg.n_q
-    return tokens / est
-
-
-def episode_calls(cfg):
-    calls = []
     for t in range(cfg.warmup_chunks):
-        lay = synth.chunk_layout(cfg, synth.cache_frames(cfg, t), t)
-        calls += [lay["n_kv"]] * cfg.layers
+        n_kv = synth.chunk_layout(cfg, synth.cache_frames(cfg, t), t)["n_kv"]
+        est += cfg.layers * (parts["attn"] * per_row * n_kv / parts["n_kv"] + parts["stats"] * per_row)
+    est += t_transition
     post = synth.chunk_layout(cfg, synth.cache_frames(cfg, cfg.warmup_chunks), cfg.warmup_chunks)["n_kv"]
-    n_loc = (cfg.sink_frames + cfg.chunk_frames) * cfg.tpf
-    calls += [post] * (cfg.layers - cfg.K) + [n_loc] * cfg.K
-    return calls
+    est += (cfg.layers - cfg.K) * parts["attn"] * per_row * post / parts["n_kv"]
+    est += cfg.K * parts["local"] * per_row
+    return est
 
 
 def cpu_threads():
@@ -371,29 +399,48 @@ def cpu_threads():
 
 
 # --------------------------------------------------------------------------- arms
+def cpu_baseline_block(cfg, rows: int, parts_list, t_transition: float) -> dict:
+    """The oracle's throughput on this host's cores from sampled calls and a timed transition."""
+    parts = {key: statistics.mean(p[key] for p in parts_list) for key in ("attn", "stats", "local")}
+    parts.update(n_kv=parts_list[0]["n_kv"], n_loc=parts_list[0]["n_loc"], rows=rows)
+    episode_s = oracle_episode_seconds(cfg, parts, t_transition)
+    sampled = sum(p["attn"] + p["stats"] + p["local"] for p in parts_list)
+    sample = (f"{rows} query rows of one layer's last warmup call (n_kv {parts['n_kv']}): float64 split attention "
+              f"over explicit masks {parts['attn']:.2f} s, statistics {parts['stats']:.2f} s, L-layer local attention "
+              f"(n_kv {parts['n_loc']}) + projection {parts['local']:.2f} s (mean of {len(parts_list)}), scaled "
+              f"linearly to every call of the episode (attention in rows x KV rows, the rest in rows); the "
+              f"transition (dense-LU absorb solve + error for {cfg.layers} layers at D = {cfg.D}, selection) timed "
+              f"in full: {t_transition:.2f} s")
+    return {"value": (cfg.warmup_chunks + 1) * cfg.n_q / episode_s, "unit": UNIT, "cores": cpu_threads(),
+            "kind": "oracle", "sample": sample, "extrapolated": True, "episode_s_estimate": episode_s,
+            "sampled_s": sampled + t_transition, "transition_s": t_transition}
+
+
 def reference_arm(args, cfg, rank):
+    """The oracle timed on the host's cores. Each step is a bounded sample of the episode (one
+    layer call's sampled rows through the attention, the statistics and the L-layer call); the
+    transition is timed in full once; the line's value is the episode's query tokens over the
+    oracle's estimated episode time, and ms_per_step is the time of a sampled step as run."""
     if rank != 0:
         return 0
-    calls = episode_calls(cfg)
     rows = args.cpu_rows
     for _ in range(args.warmup):
-        oracle_sample(cfg, max(8, rows // 8))
-    times = []
+        oracle_parts(cfg, max(8, rows // 8))
+    parts_list = []
+    t0 = time.perf_counter()
     for _ in range(args.steps):
-        dt, nkv = oracle_sample(cfg, rows)
-        times.append(dt)
-    dt = sum(times) / len(times)
-    value = oracle_value(cfg, dt, rows, nkv, calls)
-    step_est_ms = (cfg.warmup_chunks + 1) * cfg.n_q / value * 1e3
-    cores = cpu_threads()
-    sample = (f"{rows} query rows of one layer's last warmup call (n_kv {nkv}), split attention over explicit "
-              f"masks + statistics in float64, extrapolated linearly in rows and KV rows to the episode")
+        parts_list.append(oracle_parts(cfg, rows))
+    step_ms = (time.perf_counter() - t0) / max(1, args.steps) * 1e3
+    t_transition = oracle_transition(cfg)
+    cpu = cpu_baseline_block(cfg, rows, parts_list, t_transition)
+    value = cpu["value"]
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_est_ms, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_block(cfg, args.gpus),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "config": config_block(cfg, args.gpus), "extrapolated": True,
+        "episode_ms_estimate": cpu["episode_s_estimate"] * 1e3,
+        "cpu_baseline": cpu,
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -489,6 +536,7 @@ def ispa_arm(args, cfg, rank, world, local_rank):
             "attn_kernel": "two_group" if args.attn_kernel == "auto" else args.attn_kernel,
             "peak_kind": f"{peak_kind} sustained bf16 (timed inside a long step)",
             "frac_of_burst_peak": achieved / burst,
+            "frac_of_datasheet_dense_bf16": achieved / DATASHEET_DENSE_BF16_TFLOPS,
             "per_call_ms": secs / max(1, args.steps * cfg.warmup_chunks * cfg.layers) * 1e3,
             "attention_ms_per_call": by_kind["attention"][0] / max(1, by_kind["attention"][1]) * 1e3,
             "statistics_ms_per_chunk_of_all_layers": by_kind["statistics"][0] / max(1, by_kind["statistics"][1]) * 1e3}
@@ -557,14 +605,14 @@ def ispa_arm(args, cfg, rank, world, local_rank):
 
     assert ispa.ispa_device_status() == ispa.ISPA_OK
 
+    shapes = None
+    if world == 1 and not args.no_shapes:
+        shapes = shape_calls(device, steps=5, warmup=3, threads=threads)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, nkv = oracle_sample(cfg, args.cpu_rows)
-        cpu = {"value": oracle_value(cfg, dt, args.cpu_rows, nkv, episode_calls(cfg)), "unit": UNIT,
-               "cores": cpu_threads(), "kind": "oracle",
-               "sample": f"{args.cpu_rows} query rows of one layer's last warmup call (n_kv {nkv}), float64 split "
-                         f"attention over explicit masks + statistics, {dt:.2f} s, extrapolated linearly in rows and "
-                         f"KV rows to the episode"}
+        parts = oracle_parts(cfg, args.cpu_rows)
+        cpu = cpu_baseline_block(cfg, args.cpu_rows, [parts], oracle_transition(cfg))
 
     if rank == 0:
         line = {
@@ -574,10 +622,75 @@ def ispa_arm(args, cfg, rank, world, local_rank):
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches), "clocks": clk,
             "selection": {"idx": sess.idx, "margin": sess.selection_margin()},
             "kv_cache": kv_block(cfg, sess.is_local),
+            "shapes": shapes,
             "input_generation_s": gen_s,
         }
         print(json.dumps(line), flush=True)
     return 0
+
+
+def kv_device(cfg, layer: int, frames, which: str, device, threads: int) -> torch.Tensor:
+    """K or V of `frames` (time order) on the device, bf16, generated frame by frame on `threads`
+    host threads (the same bytes as synth.kv_tensor)."""
+    tpf = cfg.tpf
+    host = np.empty((len(frames) * tpf, cfg.D), dtype=np.uint16)
+
+    def fill(i):
+        x = synth.frame_kv(cfg, layer, frames[i], which).reshape(tpf, cfg.D)
+        host[i * tpf:(i + 1) * tpf] = synth.bf16_bits_from_f32(x)
+
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(fill, range(len(frames))))
+    t = torch.from_numpy(host.view(np.int16)).to(device).view(torch.bfloat16)
+    return t.reshape(len(frames) * tpf, cfg.heads, cfg.head_dim)
+
+
+def shape_calls(device, steps: int, warmup: int, threads: int) -> dict:
+    """One layer's warmup call (split attention with the statistics fused, the library's call for
+    a single layer) at the last warmup chunk of each model shape, timed alone with CUDA events,
+    L2 flushed (a 256 MB write) before every call; median of `steps`. The roofline fraction takes
+    the measured burst peak (a kernel pair timed alone); hbm_gbs is the call's algorithmic bytes
+    (Q, K, V, O and lse once) over its time."""
+    from streaming_video_attention_b200.session import IspaSession
+
+    burst, _, hbm, _ = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    out = {}
+    for name in ("1p3b_bf16", "long_bf16", "14b_bf16"):
+        cfg = synth.CONFIGS[name]
+        t = cfg.warmup_chunks - 1
+        frames = synth.cache_frames(cfg, t)
+        lay = synth.chunk_layout(cfg, frames, t)
+        n_kv = lay["n_kv"]
+        q = torch.from_numpy(synth.bf16_bits_from_f32(synth.chunk_q(cfg, 0, t)).view(np.int16)).to(device)
+        q = q.view(torch.bfloat16)
+        k = kv_device(cfg, 0, frames, "k", device, threads)
+        v = kv_device(cfg, 0, frames, "v", device, threads)
+        sess = IspaSession(1, cfg.heads, cfg.head_dim, cfg.lam, 1, "bf16", str(device), batch_stats=False)
+        sess.reserve(cfg.n_q)
+        o = torch.empty((cfg.n_q, cfg.heads, cfg.head_dim), dtype=torch.bfloat16, device=device)
+        lse = torch.empty((cfg.heads, cfg.n_q), dtype=torch.float32, device=device)
+        sink, chunk = (lay["sink_begin"], lay["sink_end"]), (lay["chunk_begin"], lay["chunk_end"])
+        times = []
+        for i in range(warmup + steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            sess.full_attention(0, q, k, v, sink, chunk, o, lse, collect=True)
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= warmup:
+                times.append(e0.elapsed_time(e1) / 1e3)
+        dt = statistics.median(times)
+        flops = 4.0 * cfg.n_q * n_kv * cfg.head_dim * cfg.heads + 4.0 * cfg.n_q * cfg.D * cfg.D
+        nbytes = 2.0 * (2 * cfg.n_q + 2 * n_kv) * cfg.D + 4.0 * cfg.heads * cfg.n_q
+        out[name] = {"n_q": cfg.n_q, "n_kv": n_kv, "heads": cfg.heads, "D": cfg.D, "ms": dt * 1e3,
+                     "query_tokens_per_s": cfg.n_q / dt, "tflops": flops / dt / 1e12,
+                     "frac_of_burst_peak": flops / dt / 1e12 / burst,
+                     "hbm_gbs": nbytes / dt / 1e9, "frac_of_hbm_peak": nbytes / dt / 1e9 / hbm}
+        del q, k, v, sess, o, lse
+        torch.cuda.empty_cache()
+    return out
 
 
 def unit_arm(args, cfg):
