@@ -30,6 +30,10 @@
  *    ispa_device_status() reads and clears.
  *  - Threading: calls may come from several host threads; ispa_last_error() is
  *    per-thread.
+ *  - Device reset: the library looks up the device address of each of its own device
+ *    variables (the error flag; the static scratch of ispa_attn_split_noalloc) once per device
+ *    and keeps it for the life of the process. cudaDeviceReset frees them: after resetting a
+ *    device, make no further library call on that device in the same process.
  */
 #ifndef ISPA_H
 #define ISPA_H
@@ -157,7 +161,8 @@ int ispa_attn_split_i8(const ispa_attn_desc *desc, const signed char *q8, const 
  * float32 elements); larger calls return ISPA_ERR_UNSUPPORTED before any launch. stats is
  * required. The array is held by every GPU that loads the library until the process
  * exits. The first call on a device looks up the array's device address (make that first
- * call before any stream capture). All calls share the array: calls that overlap on the
+ * call before any stream capture); the address is kept until the process exits, so a
+ * cudaDeviceReset of that device ends the use of this call in the process. All calls share the array: calls that overlap on the
  * GPU race and must be serialised by the caller. Arguments otherwise as ispa_attn_split. */
 int ispa_attn_split_noalloc(const ispa_attn_desc *desc, const void *q, const void *k, const void *v,
                             void *o_full, float *lse_full, void *o_loc, float *lse_loc, void *o_hist,
@@ -218,6 +223,21 @@ int ispa_absorb_error(const ispa_stats *per_layer, int n_layers, const void *con
  *   is_local [n_layers] (host, 1 for a selected layer), either output may be NULL. */
 int ispa_select_layers(const float *eps_host, int n_layers, int K, int *idx_out,
                        unsigned char *is_local);
+
+/* ispa_rewarm_check -- the re-warmup trigger's decision, host only [ISPA §3.1 last paragraph,
+ * §3.3 last paragraph: the warmup is entered again when the scene changes; the pages give no
+ * trigger. Reading: after a transition each monitored F-layer's live error -- ispa_absorb_error
+ * of the transition's dW on one chunk's statistics -- is recorded per chunk; the warmup is
+ * re-entered when a layer's latest live error exceeds both ratio x and min_rise + the lowest
+ * live error that layer showed on the earlier chunks since the transition].
+ *   live_history: host float [n_chunks][n_layers], oldest chunk first, NaN where a layer was not
+ *     monitored in that chunk (an L-layer, or a layer the caller does not watch).
+ *   ratio, min_rise: the rule's constants (the session uses 4 and 0.02); compared in double.
+ *   fired: host [n_layers], set to 1 for a layer whose latest entry is a number, that has at least
+ *     one earlier number, and whose latest value exceeds both bounds; 0 otherwise.
+ * Returns the number of layers fired (>= 0), or an error code (nothing written). */
+int ispa_rewarm_check(const float *live_history, int n_chunks, int n_layers, double ratio, double min_rise,
+                      unsigned char *fired);
 
 /* ispa_local_attn -- an L-layer after the switch [ISPA §3.1 step 3, §3.3]: attention
  * over the local rows only (every one of desc->n_kv rows of k_loc/v_loc, i.e. the sink

@@ -709,6 +709,35 @@ int ispa_select_layers(const float *eps_host, int n_layers, int K, int *idx_out,
     return ISPA_OK;
 }
 
+int ispa_rewarm_check(const float *live_history, int n_chunks, int n_layers, double ratio, double min_rise,
+                      unsigned char *fired) {
+    g_last_error.clear();
+    if (n_chunks < 0 || n_layers < 0) return fail(ISPA_ERR_INVALID_ARG, "n_chunks and n_layers must be >= 0");
+    if (n_layers > 0 && !fired) return fail(ISPA_ERR_INVALID_ARG, "fired is NULL");
+    if (n_chunks > 0 && n_layers > 0 && !live_history) return fail(ISPA_ERR_INVALID_ARG, "live_history is NULL");
+    if (!(ratio >= 0.0) || !(min_rise >= 0.0)) return fail(ISPA_ERR_INVALID_ARG, "ratio and min_rise must be >= 0");
+    int count = 0;
+    for (int l = 0; l < n_layers; ++l) {
+        fired[l] = 0;
+        if (n_chunks < 2) continue;
+        const float latest = live_history[(size_t)(n_chunks - 1) * n_layers + l];
+        if (latest != latest) continue;   // not monitored in the latest chunk
+        double lowest = INFINITY;
+        bool seen = false;
+        for (int c = 0; c < n_chunks - 1; ++c) {
+            const float e = live_history[(size_t)c * n_layers + l];
+            if (e != e) continue;
+            seen = true;
+            lowest = std::min(lowest, (double)e);
+        }
+        if (seen && (double)latest > ratio * lowest && (double)latest > lowest + min_rise) {
+            fired[l] = 1;
+            ++count;
+        }
+    }
+    return count;
+}
+
 int ispa_local_attn(const ispa_attn_desc *desc, const void *q, const void *k_loc, const void *v_loc, void *o,
                     float *lse, const void *w_new, void *y, void *ws, size_t ws_bytes, ispa_stream_t stream) {
     g_last_error.clear();

@@ -11,9 +11,9 @@
 //                                             per block, both ways, on (C W) itself
 //   five traces -> E^2, T^2, eps              GEMMs G dW, H W, G W, then dot_partials
 //
-// Block size nb = 64 (D must be a multiple of 64). The diagonal blocks are factored and
-// solved by one CTA each in shared memory; everything of order D^3 runs in the batched
-// GEMM. A non-positive pivot marks the layer ISPA_ERR_NOT_SPD and turns its results to
+// Block size nb = 64 (D must be a multiple of 64). Each 64 x 64 diagonal block is factored
+// (potrf_diag) and each panel below it solved (trsm_panel) by CTAs whose threads hold one row
+// of the block in registers; everything of order D^3 runs in batched GEMMs. A non-positive pivot marks the layer ISPA_ERR_NOT_SPD and turns its results to
 // NaN; nothing traps.
 #include "common.cuh"
 

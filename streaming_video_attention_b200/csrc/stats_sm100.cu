@@ -3,8 +3,8 @@
 // from the bf16 operands A = A_loc and R = A_full - A_loc, each [n, D] row-major (the
 // layout the split-attention epilogue writes), accumulated in float32.
 //
-// One CTA owns one 128x128 output tile of one layer and reduces over all n token rows in a
-// fixed order (no atomics: results repeat bit for bit). Several layers whose operands lie
+// One CTA owns one 128 x 256 output tile (128 x 128 when D is not a multiple of 256) of one
+// layer and reduces over all n token rows in a fixed order (no atomics: results repeat bit for bit). Several layers whose operands lie
 // contiguously ([layers][n][D]) go in one launch (grid.y = layer), so that a warmup chunk's
 // statistics fill the GPU with ~30 waves instead of one short wave per layer; each tile's
 // arithmetic does not depend on the batching. G and H are symmetric: only tiles on or

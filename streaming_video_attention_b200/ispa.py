@@ -29,7 +29,7 @@ ISPA_FP32 = 1
 
 EXPORTS = (
     "ispa_attn_split", "ispa_attn_split_noalloc", "ispa_accum_stats", "ispa_stats_reset", "ispa_solve_absorb",
-    "ispa_absorb_error", "ispa_quantize_w8", "ispa_project_w8a8", "ispa_select_layers",
+    "ispa_absorb_error", "ispa_quantize_w8", "ispa_project_w8a8", "ispa_select_layers", "ispa_rewarm_check",
     "ispa_quantize_q_i8", "ispa_k_blocks", "ispa_quantize_k_i8", "ispa_attn_split_i8",
     "ispa_attn_split_ops", "ispa_accum_ops",
     "ispa_local_attn", "ispa_workspace_bytes", "ispa_device_status", "ispa_selftest_bounded_wait",
@@ -84,6 +84,8 @@ def lib() -> ctypes.CDLL:
         L.ispa_solve_absorb.argtypes = [ctypes.POINTER(CStats), i, ctypes.POINTER(vp), i, f, vp, vp, vp,
                                         ctypes.POINTER(vp), vp, vp, sz, vp]
         L.ispa_select_layers.argtypes = [ctypes.POINTER(ctypes.c_float), i, i, ctypes.POINTER(ctypes.c_int),
+                                         ctypes.POINTER(ctypes.c_ubyte)]
+        L.ispa_rewarm_check.argtypes = [ctypes.POINTER(ctypes.c_float), i, i, ctypes.c_double, ctypes.c_double,
                                          ctypes.POINTER(ctypes.c_ubyte)]
         L.ispa_local_attn.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.ispa_workspace_bytes.argtypes = [ctypes.POINTER(AttnDesc), i, i]
@@ -275,6 +277,19 @@ def ispa_select_layers(eps: Sequence[float], K: int):
     flags = (ctypes.c_ubyte * max(1, L))()
     _check(lib().ispa_select_layers(e, L, K, idx, flags), "ispa_select_layers")
     return [idx[i] for i in range(k)], [flags[i] for i in range(L)]
+
+
+def ispa_rewarm_check(history: Sequence[Sequence[float]], ratio: float, min_rise: float):
+    """The trigger's decision on a [chunks][layers] history of live errors (NaN = not monitored);
+    returns the fired flags per layer."""
+    n_chunks = len(history)
+    n_layers = len(history[0]) if n_chunks else 0
+    flat = (ctypes.c_float * max(1, n_chunks * n_layers))(*[float(x) for row in history for x in row])
+    fired = (ctypes.c_ubyte * max(1, n_layers))()
+    rc = lib().ispa_rewarm_check(flat, n_chunks, n_layers, float(ratio), float(min_rise), fired)
+    if rc < 0:
+        _check(rc, "ispa_rewarm_check")
+    return [fired[i] for i in range(n_layers)]
 
 
 def ispa_local_attn(desc, q, k_loc, v_loc, o, lse=None, w_new=None, y=None, ws=None, stream=None) -> None:

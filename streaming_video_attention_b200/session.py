@@ -12,7 +12,8 @@ The session owns the statistics buffers, dW, the error vector and the updated we
 caller owns the KV cache (evicting the history of an L-layer is the caller freeing it).
 
 Statistics of a warmup chunk: each layer's full_attention(collect=True) writes its operands
-(A_loc, R) into the layer's slot of one [layers, n_q, D] buffer, and flush_stats() (called by
+(A_loc, R) into the layer's slot of one buffer of layers x n_q x D elements (slots packed for
+the chunk's row count, so a run of layers is one contiguous operand), and flush_stats() (called by
 the caller after the chunk's last layer, and by transition()) accumulates every pending layer
 in one launch -- the same sums, bit for bit, as accumulating layer by layer, without a short
 final wave per layer. batch_stats=False accumulates inside each call instead.
@@ -126,31 +127,36 @@ class IspaSession:
             self._ops_buffers(max_n_q)
 
     def _ops_buffers(self, n_q: int) -> Tuple[torch.Tensor, torch.Tensor]:
-        if self._ops is None or self._ops[0].shape[1] < n_q:
-            shape = (self.layers, n_q, self.D)
-            self._ops = (torch.empty(shape, dtype=self.tdtype, device=self.device),
-                         torch.empty(shape, dtype=self.tdtype, device=self.device))
+        """Flat operand buffers for layers x n_q rows: layer l of a chunk with n rows per layer
+        sits at [l * n * D, (l + 1) * n * D), so consecutive layers are contiguous for any n."""
+        need = self.layers * n_q * self.D
+        if self._ops is None or self._ops[0].numel() < need:
+            self._ops = (torch.empty(need, dtype=self.tdtype, device=self.device),
+                         torch.empty(need, dtype=self.tdtype, device=self.device))
         return self._ops
 
+    def _ops_slot(self, layer: int, n: int) -> Tuple[torch.Tensor, torch.Tensor]:
+        a_all, r_all = self._ops_buffers(n)
+        lo, hi = layer * n * self.D, (layer + 1) * n * self.D
+        return a_all[lo:hi].view(n, self.D), r_all[lo:hi].view(n, self.D)
+
     def flush_stats(self, stream=None) -> None:
-        """Accumulate the pending warmup operands: one launch per run of consecutive layers
-        with the same row count."""
+        """Accumulate the pending warmup operands: one launch per run of consecutive layers (all
+        pending layers share one row count)."""
         if not self._pending:
             return
         a_all, r_all = self._ops
         layers = sorted(self._pending)
+        n = self._pending[layers[0]]
         start = 0
         while start < len(layers):
             end = start + 1
-            n = self._pending[layers[start]]
-            while end < len(layers) and layers[end] == layers[end - 1] + 1 and self._pending[layers[end]] == n:
+            while end < len(layers) and layers[end] == layers[end - 1] + 1:
                 end += 1
             l0, l1 = layers[start], layers[end - 1] + 1
-            if a_all.shape[1] == n:
-                a, r = a_all[l0:l1], r_all[l0:l1]
-            else:   # operands were written into the first n rows of wider slots: pack them
-                a, r = a_all[l0:l1, :n].contiguous(), r_all[l0:l1, :n].contiguous()
-            ispa.ispa_accum_ops(self.stats[l0:l1], a, r, n, self.code, stream)
+            lo, hi = l0 * n * self.D, l1 * n * self.D
+            ispa.ispa_accum_ops(self.stats[l0:l1], a_all[lo:hi].view(l1 - l0, n, self.D),
+                                r_all[lo:hi].view(l1 - l0, n, self.D), n, self.code, stream)
             start = end
         self._pending = {}
 
@@ -171,10 +177,10 @@ class IspaSession:
                 self.monitor[layer] = ispa.Stats(self.D, self.device)
             st = self.monitor[layer]
         if collect and self.batch_stats:
-            if layer in self._pending:
-                self.flush_stats(stream)   # a second call for the layer before a flush
-            a_all, r_all = self._ops_buffers(n_q)
-            ispa.ispa_attn_split_ops(desc, q, k, v, o, lse, a_all[layer], r_all[layer], o_loc, lse_loc, o_hist,
+            if layer in self._pending or (self._pending and next(iter(self._pending.values())) != n_q):
+                self.flush_stats(stream)   # a second call for the layer, or another row count, before a flush
+            a_op, r_op = self._ops_slot(layer, n_q)
+            ispa.ispa_attn_split_ops(desc, q, k, v, o, lse, a_op, r_op, o_loc, lse_loc, o_hist,
                                      lse_hist, stream=stream)
             self._pending[layer] = n_q
             return
@@ -235,16 +241,14 @@ class IspaSession:
         return live
 
     def rewarm_layers(self) -> List[int]:
-        """Monitored layers whose latest live error left the range seen since the transition."""
+        """Monitored layers whose latest live error left the range seen since the transition
+        (the library's ispa_rewarm_check on the recorded live errors)."""
         if len(self.live_history) < 2:
             return []
-        latest, earlier = self.live_history[-1], self.live_history[:-1]
-        out = []
-        for l, e in latest.items():
-            ref = [d[l] for d in earlier if l in d]
-            if ref and e > self.RATIO * min(ref) and e > min(ref) + self.MIN_RISE:
-                out.append(l)
-        return sorted(out)
+        nan = float("nan")
+        hist = [[d.get(l, nan) for l in range(self.layers)] for d in self.live_history]
+        fired = ispa.ispa_rewarm_check(hist, self.RATIO, self.MIN_RISE)
+        return [l for l in range(self.layers) if fired[l]]
 
     def selection_margin(self) -> Optional[float]:
         """(eps_(K+1) - eps_(K)) / eps_(K) of the last transition: how decisive the cut was."""

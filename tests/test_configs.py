@@ -3,7 +3,8 @@
 
 * tiny fp32 (1 layer, 2 x 64, 4 warmup chunks): the whole streaming run, element by element.
 * structured bf16, scaled down (4 layers, cut + re-warmup, K sweep): the whole run.
-* 1.3B shape: one planted layer through the whole warmup at full size (oracle on every row).
+* 1.3B shape: one planted and one i.i.d. layer through the whole warmup at full size (oracle on
+  every row; dW through the whole bf16 chain).
 * long history (n_kv 191,880): one layer, sampled query rows; then the L-layer call.
 * 14B shape (40 x 128, D = 5120): one layer, sampled rows; the absorb solve at D = 5120.
 
@@ -176,18 +177,37 @@ def test_structured_run_with_automatic_rewarmup():
     _compare_runs(cfg, got, want, attn_tol=2e-2, eps_tol=5e-2, y_tol=5e-2)
 
 
-def test_1p3b_planted_layer_full_warmup():
-    """The 1.3B attention shape (12 x 128, n_q 4680, H = 15, 18, 21) through the whole warmup
-    of one planted layer, the oracle on every row: statistics, eps, dW against the oracle."""
-    base = synth.CONFIGS["structured_bf16"]
-    cfg = synth.IspaConfig(**{**base.__dict__, "layers": 1, "K": 1, "cut_chunk": None,
-                              "total_chunks": base.warmup_chunks, "name": "structured_1layer"})
-    assert cfg.planted(0)
+@pytest.mark.parametrize("kind", ["planted", "iid"])
+def test_1p3b_layer_full_warmup_chain(kind):
+    """The 1.3B attention shape (12 x 128, n_q 4680, H = 15, 18, 21) through the whole warmup of
+    one layer -- planted (rank-16 template + drift) or i.i.d. N(0, 1) -- the oracle on every row:
+    attention outputs, eps, and dW through the whole bf16 chain (attention -> bf16 operands ->
+    statistics -> solve) against the oracle's own float64 chain on the same inputs.
+
+    dW bound: the GPU's A_loc and R differ from the oracle's by the bf16 rounding of P before the
+    PV product and of the outputs (about 1.6e-3 relative RMS per element, independent across
+    elements); the ridge solve carries that relative noise into C and from C into dW about one for
+    one, so dW moves by a few 1e-3 relative -- above the 1e-3 the solve meets on identical
+    statistics (test_solve_absorb_matches_oracle). Checked here at 1e-2."""
+    if kind == "planted":
+        base = synth.CONFIGS["structured_bf16"]
+        cfg = synth.IspaConfig(**{**base.__dict__, "layers": 1, "K": 1, "cut_chunk": None,
+                                  "total_chunks": base.warmup_chunks, "name": "structured_1layer"})
+        assert cfg.planted(0)
+    else:
+        base = synth.CONFIGS["1p3b_bf16"]
+        cfg = synth.IspaConfig(**{**base.__dict__, "layers": 1, "K": 1, "total_chunks": base.warmup_chunks,
+                                  "name": "1p3b_1layer"})
     got = gpu_episode(cfg, n_chunks=cfg.warmup_chunks)
     want = oracle.run_episode(cfg, n_chunks=cfg.warmup_chunks, keep_outputs=True)
     tg, tw = got["transitions"][0], want["transitions"][0]
     assert tg["rows"] == [3 * cfg.n_q]
-    assert abs(tg["eps"][0] - tw["eps"][0]) <= 5e-2 * tw["eps"][0], (tg["eps"], tw["eps"])
+    eps_err = abs(tg["eps"][0] - tw["eps"][0]) / tw["eps"][0]
+    dW_err = rel_fro(to_numpy(tg["dW"][0]), tw["dW"][0])
+    print(f"\n[{kind}] eps gpu {tg['eps'][0]:.6e} oracle {tw['eps'][0]:.6e} rel {eps_err:.3e}; "
+          f"dW rel Frobenius {dW_err:.3e}")
+    assert eps_err <= 5e-2, (tg["eps"], tw["eps"])
+    assert dW_err < 1e-2, dW_err
     for t in range(cfg.warmup_chunks):
         assert rel_fro(to_numpy(got["outputs"][t][0]["O"]), want["outputs"][t][0]["O"]) < 2e-2
 

@@ -1,5 +1,6 @@
-"""Host logic of the streaming session that needs no GPU: the re-warmup trigger rule, against
-the oracle's statement of the same rule on hand cases and random live-error histories."""
+"""Host logic of the streaming session that needs no GPU: the re-warmup trigger rule (the
+library's ispa_rewarm_check, a host-only call), against the oracle's statement of the same rule on
+hand cases and random live-error histories."""
 import types
 
 import numpy as np
@@ -9,7 +10,9 @@ from streaming_video_attention_b200.session import IspaSession
 
 
 def _session_rule(history):
-    fake = types.SimpleNamespace(live_history=history, RATIO=IspaSession.RATIO, MIN_RISE=IspaSession.MIN_RISE)
+    layers = 1 + max((l for d in history for l in d), default=0)
+    fake = types.SimpleNamespace(live_history=history, layers=layers, RATIO=IspaSession.RATIO,
+                                 MIN_RISE=IspaSession.MIN_RISE)
     return IspaSession.rewarm_layers(fake)
 
 
@@ -26,6 +29,21 @@ def test_rule_hand_cases():
     assert _session_rule([{3: 1e-4}, {3: 9e-3}]) == []
 
 
+def test_rewarm_check_abi():
+    from streaming_video_attention_b200 import ispa
+    nan = float("nan")
+    # layer 0 rises 30x; layer 1 is not monitored in the latest chunk; layer 2 has no earlier value;
+    # layer 3 rises 5x but by less than min_rise
+    hist = [[0.01, 0.5, nan, 0.001], [0.012, 0.4, nan, 0.002], [0.3, nan, 9.0, 0.005]]
+    assert ispa.ispa_rewarm_check(hist, 4.0, 0.02) == [1, 0, 0, 0]
+    assert ispa.ispa_rewarm_check(hist, 4.0, 0.0) == [1, 0, 0, 1]
+    assert ispa.ispa_rewarm_check(hist[:1], 4.0, 0.02) == [0, 0, 0, 0]
+    L = ispa.lib()
+    assert L.ispa_rewarm_check(None, 2, 3, 4.0, 0.02, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_rewarm_check(None, -1, 0, 4.0, 0.02, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_rewarm_check(None, 0, 0, 4.0, 0.02, None) == 0
+
+
 def test_rule_matches_oracle_on_random_histories():
     rng = np.random.default_rng(3)
     for _ in range(300):
@@ -34,7 +52,8 @@ def test_rule_matches_oracle_on_random_histories():
         hist = []
         for _ in range(n_chunks):
             present = [l for l in layers if rng.random() < 0.9]
-            hist.append({l: float(np.exp(rng.normal(-3.0, 2.0))) for l in present})
+            # live errors come from float32 device buffers
+            hist.append({l: float(np.float32(np.exp(rng.normal(-3.0, 2.0)))) for l in present})
         want = oracle.rewarm_trigger(hist[:-1], hist[-1])
         assert _session_rule(hist) == want, hist
 
@@ -57,8 +76,8 @@ def test_kv_cache_accounting():
 
 def test_flush_stats_groups_consecutive_layers_with_equal_rows(monkeypatch):
     """Warmup calls only write operands; flush_stats() accumulates each run of consecutive
-    layers with the same row count in one call, packing rows when a slot is wider; a second
-    call for a pending layer flushes first; transition() flushes before solving."""
+    layers in one call on contiguous operands; a call with another row count, or a second call
+    for a pending layer, flushes first; transition() flushes before solving."""
     import torch
     from streaming_video_attention_b200 import ispa
 
@@ -79,12 +98,15 @@ def test_flush_stats_groups_consecutive_layers_with_equal_rows(monkeypatch):
 
     for layer, n in ((0, 10), (1, 10), (2, 10), (3, 8), (4, 10)):
         call(layer, n)
-    assert [c[0] for c in calls] == ["ops"] * 5
+    assert [c[0] for c in calls] == ["ops", "ops", "ops", "accum", "ops", "accum", "ops"]
+    assert calls[3][1:] == (ids[0:3], (3, 10, 256), True, 10)
+    assert calls[5][1:] == (ids[3:4], (1, 8, 256), True, 8)
+    # slots of one row count are packed: layer l at l * n * D elements
+    base = calls[0][3]
+    assert [c[3] - base for c in calls[:3]] == [0, 10 * 256 * 2, 2 * 10 * 256 * 2]
     calls.clear()
     sess.flush_stats()
-    assert calls == [("accum", ids[0:3], (3, 10, 256), True, 10),
-                     ("accum", ids[3:4], (1, 8, 256), True, 8),
-                     ("accum", ids[4:5], (1, 10, 256), True, 10)]
+    assert calls == [("accum", ids[4:5], (1, 10, 256), True, 10)]
     calls.clear()
     sess.flush_stats()                                   # nothing pending: no call
     assert calls == []
