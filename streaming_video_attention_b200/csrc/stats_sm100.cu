@@ -3,18 +3,21 @@
 // from the bf16 operands A = A_loc and R = A_full - A_loc, each [n, D] row-major (the
 // layout the split-attention epilogue writes), accumulated in float32.
 //
-// One CTA owns one 128 x 256 output tile (128 x 128 when D is not a multiple of 256) of one
-// layer and reduces over all n token rows in a fixed order (no atomics: results repeat bit for bit). Several layers whose operands lie
-// contiguously ([layers][n][D]) go in one launch (grid.y = layer), so that a warmup chunk's
-// statistics fill the GPU with ~30 waves instead of one short wave per layer; each tile's
-// arithmetic does not depend on the batching. G and H are symmetric: only tiles on or
-// above the block diagonal are computed, and each is written to both mirrored positions,
-// so the stored G and H are exactly symmetric.
+// D a multiple of 256 (every model shape here): the persistent SM-pair kernel below -- a
+// cluster of two CTAs owns 256 x 256 output tiles, the leader drives both tensor cores with
+// cta_group::2 MMAs, two accumulators in tensor memory let one tile's epilogue overlap the next
+// tile's MMAs. Other D (multiples of 128): one CTA per 128 x 128 tile. Either way each tile
+// reduces over all n token rows in a fixed order (no atomics: results repeat bit for bit), and
+// several layers whose operands lie contiguously ([layers][n][D]) go in one launch, so that a
+// warmup chunk's statistics fill the GPU instead of one short wave per layer; each tile's
+// arithmetic does not depend on the batching. G and H are symmetric: only tiles on or above
+// the block diagonal are computed, and each is written to both mirrored positions, so the
+// stored G and H are exactly symmetric.
 //
 // Both MMA operands are "MN-major" slices of [n, D]: a TMA box of 64 token rows x 64
 // columns (128-byte swizzle) puts 64 columns of one token in each 128-byte row, with
 // consecutive tokens (the reduction index) 128 bytes apart. 256 threads: warp 0 TMA,
-// warp 1 MMA (lane 0), warps 4..7 epilogue (read-modify-write of the float32 tile).
+// warp 1 MMA, warps 4..7 epilogue (read-modify-write of the float32 tile).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -222,6 +225,260 @@ stats_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
     }
 }
 
+// ---------------------------------------------------------------------------------------
+// SM-pair kernel (D a multiple of 256): one cluster of two CTAs on two SMs owns a 256 x 256
+// output tile; the leader issues tcgen05.mma.cta_group::2 with M = 256 (each CTA's 128 output
+// rows in its own tensor memory) and N = 256 (each CTA holds 128 of the 256 columns of the
+// right operand). Per SM and k-step that halves the operand bytes of a 128 x 256 tile per flop
+// (64 instead of 96 B/clk read by the tensor core, 64 instead of 96 B/clk written by TMA), which
+// keeps shared memory below its 128 B/clk. The kernel is persistent: cluster c takes tiles
+// c, c + clusters, ... of all layers in order, with two accumulators of 256 columns in tensor
+// memory, so that one tile's read-modify-write epilogue overlaps the next tile's MMAs. Each
+// tile still reduces over all n token rows in a fixed order (no atomics).
+constexpr int kPairStages = 6;
+constexpr int kPairHalf = 128;                              // output rows / right-operand columns per CTA
+constexpr int kPairOpBytes = kKRows * kPairHalf * 2;        // 16 KB: two 64 x 64 boxes
+constexpr int kPairStageBytes = 2 * kPairOpBytes;           // left + right operand of this CTA
+constexpr int kPairOffBar = kPairStages * kPairStageBytes;
+constexpr int kPairNumBars = 2 * kPairStages + 2 + 2 + 1;   // full, empty, acc_full[2], acc_empty[2], done
+constexpr int kPairSmem = kPairOffBar + kPairNumBars * 8 + 16 + 1024;
+static_assert(kPairSmem <= 232448, "shared memory budget");
+
+struct PairParams {
+    float *out[kMaxBatch][3];   // per layer: G, C, H
+    int D, n;
+    int nb;                     // D / 256
+    int n_sym;                  // nb (nb + 1) / 2 tiles on or above the block diagonal
+    int items;                  // tiles per layer: G, C, H
+    int tiles;                  // items * layers
+    int *err_flag;
+};
+
+// Work item of a layer -> (matrix, tile row bi, tile column g) in 256-blocks: G's upper tiles,
+// then every C tile, then H's upper tiles.
+__device__ __forceinline__ void decode_pair_item(int item, int nb, int n_sym, int &mat, int &bi, int &g) {
+    int t;
+    if (item < n_sym) { mat = 0; t = item; }
+    else if (item < n_sym + nb * nb) { mat = 1; bi = (item - n_sym) / nb; g = (item - n_sym) % nb; return; }
+    else { mat = 2; t = item - n_sym - nb * nb; }
+    int r = 0;
+    while (t >= nb - r) { t -= nb - r; ++r; }
+    bi = r;
+    g = r + t;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+stats_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmR,
+                  const PairParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
+    // both CTAs evaluate the same condition, so either both leave here or neither does
+    if (ptx::cluster_nctarank() != 2) {
+        if (threadIdx.x == 0) raise_device_error(p.err_flag, ISPA_ERR_UNSUPPORTED);
+        return;
+    }
+    const uint32_t rank = ptx::cluster_ctarank();
+    const bool leader = rank == 0;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kPairOffBar);   // [stages] (leader's count both CTAs)
+    uint64_t *empty = full + kPairStages;                                // [stages] (multicast commit)
+    uint64_t *acc_full = empty + kPairStages;                            // [2] (multicast commit)
+    uint64_t *acc_empty = acc_full + 2;                                  // [2] (leader's: 4 warps x 2 CTAs)
+    uint64_t *done_bar = acc_empty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done_bar + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int cl = blockIdx.x / 2, ncl = gridDim.x / 2;
+    const int n_k = (p.n + kKRows - 1) / kKRows;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPairStages; ++s) {
+            ptx::mbar_init(&full[s], 1);
+            ptx::mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&acc_full[b], 1);
+            ptx::mbar_init(&acc_empty[b], 8);
+        }
+        ptx::mbar_init(done_bar, 1);
+        *abort_flag = 0;
+        ptx::fence_barrier_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc_2sm(tmem_slot, 512);
+        ptx::tmem_relinquish_2sm();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::cluster_sync();      // the peer's barriers exist before anything arrives on them
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            ptx::tma_prefetch_desc(&tmA);
+            ptx::tma_prefetch_desc(&tmR);
+        }
+        const uint64_t pol = ptx::policy_evict_last();
+        int it = 0;
+        bool ok = true;
+        for (int t = cl; t < p.tiles && ok; t += ncl) {
+            const int layer = t / p.items;
+            int mat, bi, g;
+            decode_pair_item(t % p.items, p.nb, p.n_sym, mat, bi, g);
+            const CUtensorMap *mapL = (mat == 2) ? &tmR : &tmA;   // left operand: A for G and C, R for H
+            const CUtensorMap *mapR = (mat == 0) ? &tmA : &tmR;   // right operand: A for G, R for C and H
+            const int rowL = bi * 256 + (int)rank * kPairHalf;
+            const int colR = g * 256 + (int)rank * kPairHalf;
+            for (int kt = 0; kt < n_k; ++kt, ++it) {
+                const int s = it % kPairStages;
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded_cluster(&empty[s], ((it / kPairStages) & 1) ^ 1,
+                                                                            kWaitLimitNs, p.err_flag, abort_flag));
+                if (!ok) break;
+                uint8_t *base = smem + s * kPairStageBytes;
+                const uint32_t lead_full = ptx::mapa_shared(ptx::smem_u32(&full[s]), 0);
+                if (leader) ptx::mbar_arrive_expect_tx_warp(&full[s], 2 * kPairStageBytes);
+                if (ptx::elect_one()) {
+#pragma unroll
+                    for (int b = 0; b < 2; ++b)
+                        ptx::tma_load_3d_2sm(base + b * (kKRows * 128), mapL, lead_full, rowL + b * 64, kt * kKRows,
+                                             layer, pol);
+#pragma unroll
+                    for (int b = 0; b < 2; ++b)
+                        ptx::tma_load_3d_2sm(base + kPairOpBytes + b * (kKRows * 128), mapR, lead_full, colR + b * 64,
+                                             kt * kKRows, layer, pol);
+                }
+                __syncwarp();
+            }
+        }
+        if (!ok) {
+            // let copies in flight land before the CTA can exit (bounded)
+            const uint64_t t0 = ptx::globaltimer_ns();
+            while (ptx::globaltimer_ns() - t0 < 2000000ull) {
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (leader only)
+        if (leader) {
+            constexpr uint32_t idesc = ptx::make_idesc_bf16(2 * kPairHalf, 256, true, true);
+            const uint32_t sbase = ptx::smem_u32(smem);
+            int it = 0, i = 0;
+            bool ok = true;
+            for (int t = cl; t < p.tiles && ok; t += ncl, ++i) {
+                const int b = i & 1;
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded_cluster(&acc_empty[b], ((i >> 1) & 1) ^ 1,
+                                                                            kWaitLimitNs, p.err_flag, abort_flag));
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)b * 256u;
+                for (int kt = 0; kt < n_k; ++kt, ++it) {
+                    const int s = it % kPairStages;
+                    ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded_cluster(&full[s], (it / kPairStages) & 1,
+                                                                                kWaitLimitNs, p.err_flag, abort_flag));
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    const uint32_t a0 = sbase + s * kPairStageBytes;
+                    const uint32_t b0 = a0 + kPairOpBytes;
+                    if (ptx::elect_one()) {
+#pragma unroll
+                        for (int kk = 0; kk < kKRows / 16; ++kk) {
+                            // both operands MN-major: 64-column groups kKRows * 128 bytes apart
+                            const uint64_t da = ptx::make_sdesc_sw128(a0 + kk * 2048, kKRows * 128, 1024);
+                            const uint64_t db = ptx::make_sdesc_sw128(b0 + kk * 2048, kKRows * 128, 1024);
+                            ptx::umma_f16_ss_2sm(d, da, db, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        ptx::umma_commit_2sm(&empty[s], 0x3);
+                    }
+                    __syncwarp();
+                }
+                if (!ok) break;
+                if (ptx::elect_one()) ptx::umma_commit_2sm(&acc_full[b], 0x3);
+                __syncwarp();
+            }
+            if (!ok && lane == 0) *abort_flag = 1;
+            // every MMA this CTA issued has completed before the pair releases tensor memory
+            if (ptx::elect_one()) ptx::umma_commit_2sm(done_bar, 0x1);
+            __syncwarp();
+            ptx::mbar_wait_bounded_cluster(done_bar, 0, kWaitLimitNs, p.err_flag, nullptr);
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int wq = warp - 4;                           // TMEM lane quarter: rows wq*32 .. +31 of this CTA's half
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        const uint32_t lead_empty0 = ptx::mapa_shared(ptx::smem_u32(&acc_empty[0]), 0);
+        const uint32_t lead_empty1 = ptx::mapa_shared(ptx::smem_u32(&acc_empty[1]), 0);
+        const size_t D = p.D;
+        int i = 0;
+        for (int t = cl; t < p.tiles; t += ncl, ++i) {
+            const int b = i & 1;
+            const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded_cluster(&acc_full[b], (i >> 1) & 1,
+                                                                                   kWaitLimitNs, p.err_flag,
+                                                                                   abort_flag));
+            if (!ok) break;
+            ptx::tc_fence_after();
+            const int layer = t / p.items;
+            int mat, bi, g;
+            decode_pair_item(t % p.items, p.nb, p.n_sym, mat, bi, g);
+            float *M = p.out[layer][mat];
+            const int warp_row0 = bi * 256 + (int)rank * kPairHalf + wq * 32;
+            const int gi = warp_row0 + lane;
+            const bool sym = mat != 1;
+            const bool diag = sym && bi == g;
+#pragma unroll 1
+            for (int c = 0; c < 256 / 32; ++c) {
+                const int gj0 = g * 256 + c * 32;
+                // warp-uniform: a 32 x 32 block wholly below the diagonal of a symmetric matrix is
+                // the mirror of one above it
+                if (diag && gj0 + 31 < warp_row0) continue;
+                uint32_t v[32];
+                ptx::tmem_ld32(tmem + (uint32_t)b * 256u + lane_off + c * 32, v);
+                ptx::tmem_wait_ld();
+                float *rowp = M + (size_t)gi * D + gj0;
+                if (!diag || gj0 > warp_row0 + 31) {
+#pragma unroll
+                    for (int q = 0; q < 32; q += 4) {
+                        float4 o = *reinterpret_cast<const float4 *>(rowp + q);
+                        o.x += __uint_as_float(v[q]);
+                        o.y += __uint_as_float(v[q + 1]);
+                        o.z += __uint_as_float(v[q + 2]);
+                        o.w += __uint_as_float(v[q + 3]);
+                        *reinterpret_cast<float4 *>(rowp + q) = o;
+                        if (sym) {
+                            M[(size_t)(gj0 + q) * D + gi] = o.x;
+                            M[(size_t)(gj0 + q + 1) * D + gi] = o.y;
+                            M[(size_t)(gj0 + q + 2) * D + gi] = o.z;
+                            M[(size_t)(gj0 + q + 3) * D + gi] = o.w;
+                        }
+                    }
+                } else {
+                    // a block on the diagonal: the upper triangle (j >= i) is updated and mirrored
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) {
+                        const int gj = gj0 + q;
+                        if (gj >= gi) {
+                            const float o = rowp[q] + __uint_as_float(v[q]);
+                            rowp[q] = o;
+                            if (gj > gi) M[(size_t)gj * D + gi] = o;
+                        }
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive_cluster(b ? lead_empty1 : lead_empty0);
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::cluster_sync();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc_2sm(tmem, 512);
+    }
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -267,6 +524,43 @@ cudaError_t launch_tiles(const CUtensorMap &ma, const CUtensorMap &mr, StatsPara
     return cudaGetLastError();
 }
 
+// Persistent SM-pair launch: as many clusters as can be resident (at most one per tile).
+cudaError_t launch_pairs(const CUtensorMap &ma, const CUtensorMap &mr, const StatsParams &sp, int layers,
+                         cudaStream_t s) {
+    PairParams p;
+    for (int l = 0; l < layers; ++l)
+        for (int m = 0; m < 3; ++m) p.out[l][m] = sp.out[l][m];
+    p.D = sp.D;
+    p.n = sp.n;
+    p.nb = sp.D / 256;
+    p.n_sym = p.nb * (p.nb + 1) / 2;
+    p.items = 2 * p.n_sym + p.nb * p.nb;
+    p.tiles = p.items * layers;
+    p.err_flag = sp.err_flag;
+    cudaError_t e = cudaFuncSetAttribute(stats_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
+    if (e != cudaSuccess) return e;
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    static int max_clusters[64] = {0};
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (max_clusters[dev] <= 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2, 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = kPairSmem;
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, stats_pair_kernel, &cfg);
+        if (e != cudaSuccess) return e;
+        if (n <= 0) return cudaErrorInvalidConfiguration;
+        max_clusters[dev] = n;
+    }
+    const int clusters = p.tiles < max_clusters[dev] ? p.tiles : max_clusters[dev];
+    stats_pair_kernel<<<2 * clusters, kThreads, kPairSmem, s>>>(ma, mr, p);
+    note_launch();
+    return cudaGetLastError();
+}
+
 // Layers [0, layers) with operands a_loc, r = [layers][n][D] contiguous and outputs
 // G[l], C[l], H[l]; layers <= kMaxBatch.
 cudaError_t launch_stats_bf16_layers(const void *a_loc, const void *r, int layers, int n, int D, float *const *G,
@@ -302,7 +596,7 @@ cudaError_t launch_stats_bf16_layers(const void *a_loc, const void *r, int layer
     p.D = D; p.n = n;
     p.nb = D / kTile;
     p.err_flag = err_flag;
-    if (D % 256 == 0) return launch_tiles<256>(ma, mr, p, layers, s);
+    if (D % 256 == 0) return launch_pairs(ma, mr, p, layers, s);
     return launch_tiles<128>(ma, mr, p, layers, s);
 }
 

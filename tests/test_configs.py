@@ -184,11 +184,16 @@ def test_1p3b_layer_full_warmup_chain(kind):
     attention outputs, eps, and dW through the whole bf16 chain (attention -> bf16 operands ->
     statistics -> solve) against the oracle's own float64 chain on the same inputs.
 
-    dW bound: the GPU's A_loc and R differ from the oracle's by the bf16 rounding of P before the
-    PV product and of the outputs (about 1.6e-3 relative RMS per element, independent across
-    elements); the ridge solve carries that relative noise into C and from C into dW about one for
-    one, so dW moves by a few 1e-3 relative -- above the 1e-3 the solve meets on identical
-    statistics (test_solve_absorb_matches_oracle). Checked here at 1e-2."""
+    dW bound, from an error model: the GPU's A_loc and R differ from the oracle's by the bf16
+    rounding of P before the PV product (about 1.7e-3 relative RMS per element, independent across
+    elements). Perturbing the oracle's own float64 attention outputs by noise of that size before
+    the bf16 operand rounding moves its dW by 1.7e-3 relative Frobenius on the i.i.d. layer (G's
+    eigenvalues 1.3 .. 1.7e3: the solve passes the noise through one for one) and by 5.3e-2 on the
+    planted layer (G's eigenvalues 5e-3 .. 8.2e3 against lambda = 1e-2: the rank-16 template leaves
+    weak directions in which the solve amplifies the noise about a hundredfold), while eps moves by
+    5e-6 and 1.4e-3 relative. The 1e-3 that the solve meets on identical statistics
+    (test_solve_absorb_matches_oracle) is therefore out of reach through any bf16 chain for the
+    planted layer; the bounds are twice to three times the model's figures."""
     if kind == "planted":
         base = synth.CONFIGS["structured_bf16"]
         cfg = synth.IspaConfig(**{**base.__dict__, "layers": 1, "K": 1, "cut_chunk": None,
@@ -207,7 +212,7 @@ def test_1p3b_layer_full_warmup_chain(kind):
     print(f"\n[{kind}] eps gpu {tg['eps'][0]:.6e} oracle {tw['eps'][0]:.6e} rel {eps_err:.3e}; "
           f"dW rel Frobenius {dW_err:.3e}")
     assert eps_err <= 5e-2, (tg["eps"], tw["eps"])
-    assert dW_err < 1e-2, dW_err
+    assert dW_err < (1e-1 if kind == "planted" else 5e-3), dW_err
     for t in range(cfg.warmup_chunks):
         assert rel_fro(to_numpy(got["outputs"][t][0]["O"]), want["outputs"][t][0]["O"]) < 2e-2
 
