@@ -193,7 +193,12 @@ int ispa_stats_reset(const ispa_stats *stats, ispa_stream_t stream);
  *     W + dW (rounded to bf16 in bf16 mode) [ISPA §3.1 step 3].
  *   layer_status: device [n_layers] int, ISPA_OK or ISPA_ERR_NOT_SPD per layer (dW and
  *     eps of such a layer are NaN).
- *   ws: ispa_workspace_bytes(NULL, n_layers, D) bytes. */
+ *   ws: ispa_workspace_bytes(NULL, n_layers, D) bytes.
+ * The layers run as up to three concurrent sub-batches, each in its own part of ws: the call
+ * forks from `stream` onto two streams the library creates on its first call on a device
+ * (driver objects, no device memory; make that first call before any stream capture) and joins
+ * them back into `stream` with events, so the results are ordered on `stream` as for any other
+ * call. Calls from several host threads are serialised while they enqueue. */
 int ispa_solve_absorb(const ispa_stats *per_layer, int n_layers, const void *const *w_o,
                       ispa_dtype w_dtype, float lambda, float *dW, float *eps, double *err_terms,
                       void *const *w_new, int *layer_status, void *ws, size_t ws_bytes,

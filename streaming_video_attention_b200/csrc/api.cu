@@ -87,6 +87,40 @@ int device_error_flag(int **out) {
     return ISPA_OK;
 }
 
+// Streams and events that let a batched solve run its layers as several concurrent sub-batches:
+// the Cholesky and triangular-solve chain of one sub-batch is a sequence of small, latency-bound
+// kernels, and the large products of another fill the SMs meanwhile. Created once per device
+// (driver objects, no device memory) and reused; calls that use them are serialised on the host.
+constexpr int kSolveStreams = 3;
+struct SideStreams {
+    cudaStream_t st[kSolveStreams - 1];
+    cudaEvent_t fork, join[kSolveStreams - 1];
+    bool ready;
+};
+std::mutex g_side_mutex;
+SideStreams g_side[kMaxDevices];
+
+int side_streams(SideStreams **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(ISPA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+    SideStreams &ss = g_side[dev];
+    if (!ss.ready) {
+        for (int i = 0; i < kSolveStreams - 1; ++i) {
+            e = cudaStreamCreateWithFlags(&ss.st[i], cudaStreamNonBlocking);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaStreamCreateWithFlags");
+            e = cudaEventCreateWithFlags(&ss.join[i], cudaEventDisableTiming);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaEventCreateWithFlags");
+        }
+        e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventCreateWithFlags");
+        ss.ready = true;
+    }
+    *out = &ss;
+    return ISPA_OK;
+}
+
 size_t elem_size(ispa_dtype t) { return t == ISPA_BF16 ? 2 : 4; }
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -571,25 +605,56 @@ int ispa_solve_absorb(const ispa_stats *per_layer, int n_layers, const void *con
     int *flag = nullptr;
     rc = device_error_flag(&flag);
     if (rc != ISPA_OK) return rc;
+    // Each chunk of up to kMaxBatch layers runs as up to kSolveStreams concurrent sub-batches: the
+    // first on `stream`, the others on side streams forked from and joined back into it. Every
+    // sub-batch uses its own slices of the workspace (its layers' M, Y, P and split blocks, its
+    // trace sums).
+    SideStreams *side = nullptr;
+    std::unique_lock<std::mutex> side_lock(g_side_mutex, std::defer_lock);
+    const int max_sub = std::min(kSolveStreams, n_layers);
+    if (max_sub > 1) {
+        side_lock.lock();
+        rc = side_streams(&side);
+        if (rc != ISPA_OK) return rc;
+    }
+    const size_t nD = (size_t)D * D;
     for (int l0 = 0; l0 < n_layers; l0 += kMaxBatch) {
         const int b = std::min(kMaxBatch, n_layers - l0);
-        PtrBatch G, C, H, W, DW, M, Y, P, WN;
-        for (int z = 0; z < b; ++z) {
-            const ispa_stats &st = per_layer[l0 + z];
-            G.p[z] = st.G; C.p[z] = st.C; H.p[z] = st.H;
-            W.p[z] = const_cast<void *>(w_o[l0 + z]);
-            DW.p[z] = dW + (size_t)(l0 + z) * D * D;
-            M.p[z] = Mb + (size_t)z * mat;
-            Y.p[z] = Yb + (size_t)z * mat;
-            P.p[z] = Pb + (size_t)z * mat;
-            if (w_new) WN.p[z] = w_new[l0 + z];
+        const int nsub = std::min(max_sub, b);
+        if (nsub > 1) {
+            CUDA_CHECK_RET(cudaEventRecord(side->fork, s), "cudaEventRecord (fork)");
+            for (int i = 0; i < nsub - 1; ++i)
+                CUDA_CHECK_RET(cudaStreamWaitEvent(side->st[i], side->fork, 0), "cudaStreamWaitEvent (fork)");
         }
-        cudaError_t e = solve_batch(G, C, H, W, w_dtype == ISPA_BF16 ? ElemType::BF16 : ElemType::F32, DW, M, Y, P,
-                                    reinterpret_cast<float *>(Yb), reinterpret_cast<float *>(Pb), split, terms,
-                                    kEpsParts, layer_status + l0, eps + l0,
-                                    err_terms ? err_terms + 2 * (size_t)l0 : nullptr, w_new ? &WN : nullptr, D, lambda,
-                                    b, flag, s);
-        if (e != cudaSuccess) return cuda_fail(e, "absorb solve");
+        for (int sb = 0; sb < nsub; ++sb) {
+            const int z0 = b * sb / nsub, z1 = b * (sb + 1) / nsub, bs = z1 - z0;
+            cudaStream_t ss = sb == 0 ? s : side->st[sb - 1];
+            PtrBatch G, C, H, W, DW, M, Y, P, WN;
+            for (int z = 0; z < bs; ++z) {
+                const int l = l0 + z0 + z;
+                const ispa_stats &st = per_layer[l];
+                G.p[z] = st.G; C.p[z] = st.C; H.p[z] = st.H;
+                W.p[z] = const_cast<void *>(w_o[l]);
+                DW.p[z] = dW + (size_t)l * nD;
+                M.p[z] = Mb + (size_t)(z0 + z) * mat;
+                Y.p[z] = Yb + (size_t)(z0 + z) * mat;
+                P.p[z] = Pb + (size_t)(z0 + z) * mat;
+                if (w_new) WN.p[z] = w_new[l];
+            }
+            cudaError_t e = solve_batch(G, C, H, W, w_dtype == ISPA_BF16 ? ElemType::BF16 : ElemType::F32, DW, M, Y, P,
+                                        reinterpret_cast<float *>(Yb + (size_t)z0 * mat),
+                                        reinterpret_cast<float *>(Pb + (size_t)z0 * mat), split + 6 * (size_t)z0 * nD,
+                                        terms + 5 * (size_t)z0 * kEpsParts, kEpsParts, layer_status + l0 + z0,
+                                        eps + l0 + z0, err_terms ? err_terms + 2 * (size_t)(l0 + z0) : nullptr,
+                                        w_new ? &WN : nullptr, D, lambda, bs, flag, ss);
+            if (e != cudaSuccess) return cuda_fail(e, "absorb solve");
+        }
+        if (nsub > 1) {
+            for (int i = 0; i < nsub - 1; ++i) {
+                CUDA_CHECK_RET(cudaEventRecord(side->join[i], side->st[i]), "cudaEventRecord (join)");
+                CUDA_CHECK_RET(cudaStreamWaitEvent(s, side->join[i], 0), "cudaStreamWaitEvent (join)");
+            }
+        }
     }
     return ISPA_OK;
 }

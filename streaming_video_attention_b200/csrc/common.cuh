@@ -116,6 +116,6 @@ struct PtrBatch {
 cudaError_t launch_split_tf32(const PtrBatch &src, ElemType t, float *hi, float *lo, int rows, int cols,
                               bool transpose, int batch, cudaStream_t s);
 cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh, const float *Bl, float *C, int M,
-                               int N, int K, int batch, int *err_flag, cudaStream_t s);
+                               int N, int K, int batch, int *err_flag, cudaStream_t s, int a_tri = 0);
 
 }  // namespace ispa

@@ -44,6 +44,7 @@ struct Tf32Params {
     float *C;
     int M, N, K;
     int three_terms;    // B_lo present
+    int a_tri;          // 0: A full; 1: A lower triangular (k < m0 + 128); 2: A upper triangular (k >= m0)
     int *err_flag;
 };
 
@@ -64,7 +65,12 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int n0 = blockIdx.x * kTile, m0 = blockIdx.y * kTile, z = blockIdx.z;
-    const int n_k = (p.K + kKStep - 1) / kKStep;
+    // k-steps of this output row tile: a triangular A is zero outside [kt0, kt1), and skipping
+    // exact zeros changes no sum
+    const int n_kall = (p.K + kKStep - 1) / kKStep;
+    const int kt0 = p.a_tri == 2 ? m0 / kKStep : 0;
+    const int kt1 = p.a_tri == 1 ? min(n_kall, (m0 + kTile) / kKStep) : n_kall;
+    const int n_k = kt1 - kt0;
     const uint32_t stage_tx = (p.three_terms ? 4 : 3) * kOpBytes;
 
     if (threadIdx.x == 0) {
@@ -97,7 +103,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
             if (!ok) break;
             uint8_t *base = smem + s * kStageBytes;
             ptx::mbar_arrive_expect_tx_warp(&full[s], stage_tx);
-            const int k0 = kt * kKStep;
+            const int k0 = (kt0 + kt) * kKStep;
             ptx::tma_load_3d_warp(base, &tAh, &full[s], k0, m0, z, pol);
             ptx::tma_load_3d_warp(base + kOpBytes, &tAl, &full[s], k0, m0, z, pol);
             ptx::tma_load_3d_warp(base + 2 * kOpBytes, &tBh, &full[s], k0, n0, z, pol);
@@ -269,8 +275,10 @@ cudaError_t launch_split_tf32(const PtrBatch &src, ElemType t, float *hi, float 
 
 // C[z] = A[z] B[z] for z < batch; A given as (A_hi, A_lo) [batch][M][K], B as (B_hi, B_lo or
 // null) transposed, [batch][N][K], all contiguous float32. M, N multiples of 128; K of 32.
+// a_tri: 1 when A is lower triangular, 2 when upper triangular (then M = K): the zero part of A
+// is not read.
 cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh, const float *Bl, float *C, int M,
-                               int N, int K, int batch, int *err_flag, cudaStream_t s) {
+                               int N, int K, int batch, int *err_flag, cudaStream_t s, int a_tri) {
     if (M % kTile || N % kTile || K % kKStep || batch <= 0) return cudaErrorInvalidValue;
     CUtensorMap ah, al, bh, bl;
     if (!make_map(&ah, Ah, batch, M, K, kTile) || !make_map(&al, Al, batch, M, K, kTile) ||
@@ -279,6 +287,7 @@ cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh
     Tf32Params p;
     p.C = C; p.M = M; p.N = N; p.K = K;
     p.three_terms = Bl != nullptr;
+    p.a_tri = (a_tri == 1 || a_tri == 2) && M == K ? a_tri : 0;
     p.err_flag = err_flag;
     cudaError_t e = cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;

@@ -397,10 +397,10 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
         float *dWc = static_cast<float *>(dW.p[0]);
         ISPA_TRY(launch_split_tf32(P, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
         ISPA_TRY(launch_split_tf32(Y, ElemType::F32, Bhi, Blo, D, D, true, batch, s));
-        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Bhi, Blo, dWc, D, D, D, batch, err_flag, s));
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Bhi, Blo, dWc, D, D, D, batch, err_flag, s, 1));   // X lower
         ISPA_TRY(launch_split_tf32(P, ElemType::F32, Ahi, Alo, D, D, true, batch, s));
         ISPA_TRY(launch_split_tf32(dW, ElemType::F32, Bhi, Blo, D, D, true, batch, s));
-        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Bhi, Blo, dWc, D, D, D, batch, err_flag, s));
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Bhi, Blo, dWc, D, D, D, batch, err_flag, s, 2));   // X^T upper
     } else {
         // dW <- Y, solved in place: forward substitution L Z = Y, then backward L^T X = Z
         copy_f32_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(Y, dW, n); note_launch();
