@@ -53,10 +53,13 @@ def parse_args(argv=None):
     ap.add_argument("--no-shapes", action="store_true",
                     help="skip the one-layer call timings of the 1.3B, long-history and 14B shapes")
     ap.add_argument("--cpu-rows", type=int, default=512)
-    ap.add_argument("--mode", choices=["episode", "call", "local", "solve"], default="episode",
+    ap.add_argument("--mode", choices=["episode", "call", "local", "solve", "stats"], default="episode",
                     help="episode: the full step (default). call / local / solve: one layer's fused split "
                          "attention at the last warmup chunk, one L-layer local attention with projection, or "
-                         "the batched solve alone (kernel-level timing, also the target of ncu captures)")
+                         "the batched solve alone, or one warmup chunk's batched statistics launch (kernel-level "
+                         "timing, also the target of ncu captures)")
+    ap.add_argument("--stats-layers", type=int, default=0,
+                    help="stats mode: layers in the batched statistics launch (default: the workload's layers)")
     ap.add_argument("--i8", action="store_true",
                     help="call mode: the 8-bit split attention (int8 Q and K, quantised inside the timed call)")
     ap.add_argument("--w8a8", action="store_true",
@@ -762,6 +765,17 @@ def unit_arm(args, cfg):
             flops = 4.0 * cfg.n_q * n_kv * cfg.head_dim * cfg.heads + 2.0 * cfg.n_q * D * D
             what = (f"L-layer local attention + W_new projection{' (W8A8 int8)' if args.w8a8 else ''}, "
                     f"n_q {cfg.n_q}, n_kv {n_kv}")
+    elif args.mode == "stats":
+        # one warmup chunk's statistics: the operands of every layer [layers][n_q][D] (bf16) in one
+        # ispa_accum_ops launch, as the session issues it after the chunk's attention calls
+        layers = args.stats_layers or cfg.layers
+        g = torch.Generator(device=device).manual_seed(0)
+        a_ops = (torch.randn(layers, cfg.n_q, D, device=device, generator=g) * 0.05).to(torch.bfloat16)
+        r_ops = (torch.randn(layers, cfg.n_q, D, device=device, generator=g) * 0.02).to(torch.bfloat16)
+        stats = [ispa.Stats(D, device) for _ in range(layers)]
+        fn = lambda: ispa.ispa_accum_ops(stats, a_ops, r_ops, cfg.n_q, ispa.ISPA_BF16)
+        flops = layers * 4.0 * cfg.n_q * D * D
+        what = f"batched statistics (G, C, H) of {layers} layers, n {cfg.n_q}, D {D}"
     else:
         Ws = [up(synth.w_out(cfg, l)) for l in range(cfg.layers)]
         sess.set_weights(Ws)
@@ -793,6 +807,40 @@ def unit_arm(args, cfg):
     dt = statistics.median(times)
     tf = flops / dt / 1e12
     extra = {}
+
+    def median_ms(f, steps):
+        ts = []
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            f()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    if args.mode == "local" and not args.w8a8:
+        # the L-layer step's two kernels apart (local attention; projection y = O W_new) and the
+        # step replayed from a CUDA graph (no host launch work between the two kernels)
+        att = lambda: sess.local_attention(0, q, k, v, o, lse)
+        proj = lambda: ispa.ispa_project(o, sess.W_new[0], y)
+        for f in (att, proj):
+            f()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        s_cap = torch.cuda.Stream(device=device)
+        s_cap.wait_stream(torch.cuda.current_stream(device))
+        with torch.cuda.stream(s_cap):
+            fn()
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=s_cap):
+                fn()
+        torch.cuda.current_stream(device).wait_stream(s_cap)
+        a_ms, p_ms = median_ms(att, args.steps), median_ms(proj, args.steps)
+        g_ms = median_ms(g.replay, args.steps)
+        extra = {"attention_only_ms": a_ms, "projection_only_ms": p_ms, "graph_step_ms": g_ms,
+                 "step_minus_parts_ms": dt * 1e3 - a_ms - p_ms}
     if args.mode == "call" and args.i8:
         # the same call without the two quantisers (int8 Q/K already resident)
         t2 = []
@@ -807,7 +855,8 @@ def unit_arm(args, cfg):
         extra = {"ms_without_quantisation": statistics.median(t2)}
     print(json.dumps({"mode": args.mode, "what": what, "ms": dt * 1e3, "ms_all": [x * 1e3 for x in times],
                       "tflops": tf, "frac_of_burst_peak": tf / burst, "peak_kind": kind,
-                      "query_tokens_per_s": cfg.n_q / dt if args.mode != "solve" else None} | extra), flush=True)
+                      "query_tokens_per_s": cfg.n_q / dt if args.mode in ("call", "local") else None} | extra),
+          flush=True)
     return 0
 
 

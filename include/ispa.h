@@ -255,6 +255,16 @@ int ispa_local_attn(const ispa_attn_desc *desc, const void *q, const void *k_loc
                     const void *v_loc, void *o, float *lse, const void *w_new, void *y, void *ws,
                     size_t ws_bytes, ispa_stream_t stream);
 
+/* ispa_project -- the attention output projection y = A W [ISPA §3.1 step 3: an L-layer's output
+ * goes through the updated projection W_new = W + dW] on its own, the step that ispa_local_attn
+ * runs after the attention when given w_new.
+ *   a [n][d_in] (device, dtype; for an attention output [n, heads, head_dim] with d_in =
+ *   heads*head_dim), w [d_in][d_out] (device, dtype), y [n][d_out] (device, dtype); all 16-byte
+ *   aligned. bf16 with d_in and d_out multiples of 128 runs on the tensor cores (fp32
+ *   accumulation, bf16 output); other shapes and float32 on the CUDA cores. */
+int ispa_project(const void *a, int n, int d_in, const void *w, int d_out, void *y, ispa_dtype dtype,
+                 ispa_stream_t stream);
+
 /* ispa_quantize_w8 -- int8 weights for the W8A8 projection of the L-layers [ISPA §4.4: ISPA
  * is combined with 8-bit weights and activations; the scheme is not given -- reading:
  * symmetric int8, one scale per output column]. For each output column j of w [d_in][d_out]

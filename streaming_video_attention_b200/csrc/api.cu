@@ -842,6 +842,30 @@ int ispa_local_attn(const ispa_attn_desc *desc, const void *q, const void *k_loc
     return ISPA_OK;
 }
 
+int ispa_project(const void *a, int n, int d_in, const void *w, int d_out, void *y, ispa_dtype dtype,
+                 ispa_stream_t stream) {
+    g_last_error.clear();
+    if (n < 0 || d_in <= 0 || d_out <= 0) return fail(ISPA_ERR_INVALID_ARG, "bad sizes n=%d d_in=%d d_out=%d", n, d_in, d_out);
+    if (dtype != ISPA_BF16 && dtype != ISPA_FP32) return fail(ISPA_ERR_INVALID_ARG, "bad dtype");
+    if (n == 0) return ISPA_OK;
+    if (!a || !w || !y) return fail(ISPA_ERR_INVALID_ARG, "a, w and y are required");
+    if (!aligned(a, 16) || !aligned(w, 16) || !aligned(y, 16)) return fail(ISPA_ERR_INVALID_ARG, "a, w and y must be 16-byte aligned");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == ISPA_BF16 && d_in % 128 == 0 && d_out % 128 == 0) {
+        int *flag = nullptr;
+        int rc = device_error_flag(&flag);
+        if (rc != ISPA_OK) return rc;
+        CUDA_CHECK_RET(launch_gemm_bf16(a, w, y, n, d_out, d_in, flag, s), "projection GEMM (tcgen05)");
+    } else {
+        const ElemType t = dtype == ISPA_BF16 ? ElemType::BF16 : ElemType::F32;
+        GemmDesc g{n, d_out, d_in, d_in, d_out, d_out, true, false, t, t, t, 1.f, 0.f, false, 1};
+        GemmBatch b;
+        b.A[0] = a; b.B[0] = w; b.C[0] = y;
+        CUDA_CHECK_RET(launch_gemm_simt(g, b, s), "projection GEMM");
+    }
+    return ISPA_OK;
+}
+
 int ispa_set_attn_kernel(int choice) {
     if (choice != ISPA_ATTN_AUTO && choice != ISPA_ATTN_SINGLE && choice != ISPA_ATTN_PAIR &&
         choice != ISPA_ATTN_TWO_GROUP)

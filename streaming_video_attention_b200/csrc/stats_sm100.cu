@@ -235,7 +235,7 @@ stats_gemm_sm100_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
 // c, c + clusters, ... of all layers in order, with two accumulators of 256 columns in tensor
 // memory, so that one tile's read-modify-write epilogue overlaps the next tile's MMAs. Each
 // tile still reduces over all n token rows in a fixed order (no atomics).
-constexpr int kPairStages = 6;
+constexpr int kPairStages = 7;
 constexpr int kPairHalf = 128;                              // output rows / right-operand columns per CTA
 constexpr int kPairOpBytes = kKRows * kPairHalf * 2;        // 16 KB: two 64 x 64 boxes
 constexpr int kPairStageBytes = 2 * kPairOpBytes;           // left + right operand of this CTA
@@ -425,41 +425,60 @@ stats_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
             const int gi = warp_row0 + lane;
             const bool sym = mat != 1;
             const bool diag = sym && bi == g;
+            // two 32-column chunks at a time: both chunks' accumulator values and stored values are
+            // loaded before either is used, so their memory latencies overlap
 #pragma unroll 1
-            for (int c = 0; c < 256 / 32; ++c) {
-                const int gj0 = g * 256 + c * 32;
+            for (int c2 = 0; c2 < 256 / 64; ++c2) {
+                const int gc0 = g * 256 + c2 * 64;
                 // warp-uniform: a 32 x 32 block wholly below the diagonal of a symmetric matrix is
                 // the mirror of one above it
-                if (diag && gj0 + 31 < warp_row0) continue;
-                uint32_t v[32];
-                ptx::tmem_ld32(tmem + (uint32_t)b * 256u + lane_off + c * 32, v);
+                const bool skip0 = diag && gc0 + 31 < warp_row0;
+                const bool skip1 = diag && gc0 + 63 < warp_row0;
+                if (skip0 && skip1) continue;
+                uint32_t v[2][32];
+                ptx::tmem_ld32(tmem + (uint32_t)b * 256u + lane_off + c2 * 64, v[0]);
+                ptx::tmem_ld32(tmem + (uint32_t)b * 256u + lane_off + c2 * 64 + 32, v[1]);
                 ptx::tmem_wait_ld();
-                float *rowp = M + (size_t)gi * D + gj0;
-                if (!diag || gj0 > warp_row0 + 31) {
+                float *rowp = M + (size_t)gi * D + gc0;
+                const bool full0 = !diag || gc0 > warp_row0 + 31;
+                const bool full1 = !diag || gc0 + 32 > warp_row0 + 31;
+                float4 old[2][8];
 #pragma unroll
-                    for (int q = 0; q < 32; q += 4) {
-                        float4 o = *reinterpret_cast<const float4 *>(rowp + q);
-                        o.x += __uint_as_float(v[q]);
-                        o.y += __uint_as_float(v[q + 1]);
-                        o.z += __uint_as_float(v[q + 2]);
-                        o.w += __uint_as_float(v[q + 3]);
-                        *reinterpret_cast<float4 *>(rowp + q) = o;
-                        if (sym) {
-                            M[(size_t)(gj0 + q) * D + gi] = o.x;
-                            M[(size_t)(gj0 + q + 1) * D + gi] = o.y;
-                            M[(size_t)(gj0 + q + 2) * D + gi] = o.z;
-                            M[(size_t)(gj0 + q + 3) * D + gi] = o.w;
+                for (int h = 0; h < 2; ++h)
+                    if ((h == 0 ? full0 : full1))
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) old[h][q] = *reinterpret_cast<const float4 *>(rowp + 32 * h + 4 * q);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    if (h == 0 ? skip0 : skip1) continue;
+                    const int gj0 = gc0 + 32 * h;
+                    float *rp = rowp + 32 * h;
+                    if (h == 0 ? full0 : full1) {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            float4 o = old[h][q];
+                            o.x += __uint_as_float(v[h][4 * q]);
+                            o.y += __uint_as_float(v[h][4 * q + 1]);
+                            o.z += __uint_as_float(v[h][4 * q + 2]);
+                            o.w += __uint_as_float(v[h][4 * q + 3]);
+                            *reinterpret_cast<float4 *>(rp + 4 * q) = o;
+                            if (sym) {
+                                M[(size_t)(gj0 + 4 * q) * D + gi] = o.x;
+                                M[(size_t)(gj0 + 4 * q + 1) * D + gi] = o.y;
+                                M[(size_t)(gj0 + 4 * q + 2) * D + gi] = o.z;
+                                M[(size_t)(gj0 + 4 * q + 3) * D + gi] = o.w;
+                            }
                         }
-                    }
-                } else {
-                    // a block on the diagonal: the upper triangle (j >= i) is updated and mirrored
+                    } else {
+                        // a block on the diagonal: the upper triangle (j >= i) is updated and mirrored
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) {
-                        const int gj = gj0 + q;
-                        if (gj >= gi) {
-                            const float o = rowp[q] + __uint_as_float(v[q]);
-                            rowp[q] = o;
-                            if (gj > gi) M[(size_t)gj * D + gi] = o;
+                        for (int q = 0; q < 32; ++q) {
+                            const int gj = gj0 + q;
+                            if (gj >= gi) {
+                                const float o = rp[q] + __uint_as_float(v[h][q]);
+                                rp[q] = o;
+                                if (gj > gi) M[(size_t)gj * D + gi] = o;
+                            }
                         }
                     }
                 }

@@ -32,7 +32,7 @@ EXPORTS = (
     "ispa_absorb_error", "ispa_quantize_w8", "ispa_project_w8a8", "ispa_select_layers", "ispa_rewarm_check",
     "ispa_quantize_q_i8", "ispa_k_blocks", "ispa_quantize_k_i8", "ispa_attn_split_i8",
     "ispa_attn_split_ops", "ispa_accum_ops",
-    "ispa_local_attn", "ispa_workspace_bytes", "ispa_device_status", "ispa_selftest_bounded_wait",
+    "ispa_local_attn", "ispa_project", "ispa_workspace_bytes", "ispa_device_status", "ispa_selftest_bounded_wait",
     "ispa_selftest_exp2_poly", "ispa_set_attn_kernel", "ispa_kernel_launches", "ispa_last_error", "ispa_version",
 )
 
@@ -87,6 +87,7 @@ def lib() -> ctypes.CDLL:
                                          ctypes.POINTER(ctypes.c_ubyte)]
         L.ispa_rewarm_check.argtypes = [ctypes.POINTER(ctypes.c_float), i, i, ctypes.c_double, ctypes.c_double,
                                          ctypes.POINTER(ctypes.c_ubyte)]
+        L.ispa_project.argtypes = [vp, i, i, vp, i, vp, i, vp]
         L.ispa_local_attn.argtypes = [ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.ispa_workspace_bytes.argtypes = [ctypes.POINTER(AttnDesc), i, i]
         L.ispa_workspace_bytes.restype = ctypes.c_size_t
@@ -296,6 +297,14 @@ def ispa_local_attn(desc, q, k_loc, v_loc, o, lse=None, w_new=None, y=None, ws=N
     rc = lib().ispa_local_attn(ctypes.byref(desc), _p(q), _p(k_loc), _p(v_loc), _p(o), _p(lse), _p(w_new), _p(y),
                                _p(ws), 0 if ws is None else ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "ispa_local_attn")
+
+
+def ispa_project(a: torch.Tensor, w: torch.Tensor, y: torch.Tensor, stream=None) -> None:
+    """y = A W; a [n, d_in] (or [n, heads, head_dim]), w [d_in, d_out], y [n, d_out], one dtype."""
+    n = a.shape[0]
+    d_in, d_out = w.shape
+    _check(lib().ispa_project(_p(a), n, d_in, _p(w), d_out, _p(y), dtype_code(a.dtype), _stream(stream)),
+           "ispa_project")
 
 
 def ispa_device_status(stream=None) -> int:

@@ -52,6 +52,19 @@ def test_invalid_arguments_are_rejected_before_any_launch():
     assert L.ispa_selftest_bounded_wait(0, None) == ispa.ISPA_ERR_INVALID_ARG
 
 
+def test_project_arguments_are_checked_before_any_launch():
+    L = ispa.lib()
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: every call below fails its checks first
+    assert L.ispa_project(fake, -1, 128, fake, 128, fake, ispa.ISPA_BF16, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_project(fake, 4, 0, fake, 128, fake, ispa.ISPA_BF16, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_project(fake, 4, 128, fake, 128, fake, 7, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_project(None, 4, 128, fake, 128, fake, ispa.ISPA_BF16, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_project(ctypes.c_void_p((1 << 20) + 2), 4, 128, fake, 128, fake, ispa.ISPA_BF16,
+                          None) == ispa.ISPA_ERR_INVALID_ARG
+    assert b"aligned" in L.ispa_last_error()
+    assert L.ispa_project(None, 0, 128, None, 128, None, ispa.ISPA_BF16, None) == ispa.ISPA_OK
+
+
 def test_workspace_sizes():
     d = ispa.make_desc(4680, 37440, 12, 128, dtype=ispa.ISPA_BF16)
     # fused statistics need the A_loc and R operands: 2 * n_q * D bf16

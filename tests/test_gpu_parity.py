@@ -270,6 +270,20 @@ def test_local_attention_and_projection(dtype):
     assert rel_fro(to_numpy(y), oracle.project(A, W)) < ATTN_TOL[dtype]
 
 
+@pytest.mark.parametrize("dtype,n,d_in,d_out", [("bf16", 600, 256, 384), ("bf16", 4680, 1536, 1536),
+                                                 ("bf16", 130, 192, 64), ("fp32", 300, 256, 128)])
+def test_project_matches_oracle(dtype, n, d_in, d_out):
+    """ispa_project: y = A W on the tensor cores (bf16, multiples of 128) or the CUDA cores (other
+    shapes, float32), against the oracle's projection of the same values."""
+    a = synth.normal_tensor(61, (1,), (n, d_in), dtype)
+    W = synth.normal_tensor(61, (2,), (d_in, d_out), dtype, std=1 / math.sqrt(d_in))
+    y = torch.full((n, d_out), float("nan"), dtype=torch_dtype(dtype), device="cuda")
+    ispa.ispa_project(to_device(a, dtype), to_device(W, dtype), y)
+    torch.cuda.synchronize()
+    assert ispa.ispa_device_status() == ispa.ISPA_OK
+    assert rel_fro(to_numpy(y), oracle.project(a, W)) < ATTN_TOL[dtype]
+
+
 # ------------------------------------------------------------------ full size, sampled rows
 def test_full_size_1p3b_layer_sampled_rows():
     """One 1.3B-shaped layer call at the last warmup chunk (n_q 4680, n_kv 37440, 12 heads),
