@@ -140,12 +140,15 @@ size_t w8a8_ws_bytes(int n_rows, int D) {
     return align_up((size_t)n_rows * D, 256) + align_up((size_t)n_rows * sizeof(float), 256);
 }
 
-constexpr int kEpsParts = 64;
+// Partial sums per layer and trace of the reconstruction error: with D a multiple of 128 the D x D
+// products run on the tensor cores and every 128 x 128 output tile contributes one partial from
+// its epilogue; otherwise a reduction kernel writes 64.
+int eps_parts(int D) { return D % 128 == 0 ? (D / 128) * (D / 128) : 64; }
 
 size_t solve_ws_bytes(int n_layers, int D) {
     const size_t b = (size_t)std::min(n_layers, kMaxBatch);
     const size_t mat = (size_t)D * D * sizeof(float);   // D is a multiple of 64: 256-byte multiple
-    return b * 9 * mat + align_up(5 * b * kEpsParts * sizeof(double), 256);
+    return b * 9 * mat + align_up(5 * b * (size_t)eps_parts(D) * sizeof(double), 256);
 }
 
 int check_desc(const ispa_attn_desc *d, bool need_ranges) {
@@ -644,7 +647,7 @@ int ispa_solve_absorb(const ispa_stats *per_layer, int n_layers, const void *con
             cudaError_t e = solve_batch(G, C, H, W, w_dtype == ISPA_BF16 ? ElemType::BF16 : ElemType::F32, DW, M, Y, P,
                                         reinterpret_cast<float *>(Yb + (size_t)z0 * mat),
                                         reinterpret_cast<float *>(Pb + (size_t)z0 * mat), split + 6 * (size_t)z0 * nD,
-                                        terms + 5 * (size_t)z0 * kEpsParts, kEpsParts, layer_status + l0 + z0,
+                                        terms + 5 * (size_t)z0 * eps_parts(D), eps_parts(D), layer_status + l0 + z0,
                                         eps + l0 + z0, err_terms ? err_terms + 2 * (size_t)(l0 + z0) : nullptr,
                                         w_new ? &WN : nullptr, D, lambda, bs, flag, ss);
             if (e != cudaSuccess) return cuda_fail(e, "absorb solve");
@@ -702,7 +705,7 @@ int ispa_absorb_error(const ispa_stats *per_layer, int n_layers, const void *con
         }
         cudaError_t e = error_batch(G, C, H, W, w_dtype == ISPA_BF16 ? ElemType::BF16 : ElemType::F32, DW, Y, P,
                                     reinterpret_cast<float *>(Yb), reinterpret_cast<float *>(Pb), split, terms,
-                                    kEpsParts, eps + l0, err_terms ? err_terms + 2 * (size_t)l0 : nullptr, D, b, flag,
+                                    eps_parts(D), eps + l0, err_terms ? err_terms + 2 * (size_t)l0 : nullptr, D, b, flag,
                                     s);
         if (e != cudaSuccess) return cuda_fail(e, "absorb error");
     }

@@ -116,6 +116,8 @@ struct PtrBatch {
 cudaError_t launch_split_tf32(const PtrBatch &src, ElemType t, float *hi, float *lo, int rows, int cols,
                               bool transpose, int batch, cudaStream_t s);
 cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh, const float *Bl, float *C, int M,
-                               int N, int K, int batch, int *err_flag, cudaStream_t s, int a_tri = 0);
+                               int N, int K, int batch, int *err_flag, cudaStream_t s, int a_tri = 0,
+                               const PtrBatch *dot_x = nullptr, bool dot_x_bf16 = false, double *dot_out = nullptr,
+                               bool write_c = true);
 
 }  // namespace ispa

@@ -45,6 +45,14 @@ struct Tf32Params {
     int M, N, K;
     int three_terms;    // B_lo present
     int a_tri;          // 0: A full; 1: A lower triangular (k < m0 + 128); 2: A upper triangular (k >= m0)
+    // optional trace partial: dot_out[z][tile] = sum over the tile of C_ij * X_z[i][j] (double),
+    // X_z [M][N] row-major float32 or bf16 (one pointer per batch entry); C is written only if
+    // write_c
+    PtrBatch dot_x;
+    int has_dot;
+    int dot_x_bf16;
+    double *dot_out;
+    int write_c;
     int *err_flag;
 };
 
@@ -150,16 +158,46 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
         const int r = wq * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
         const bool ok = ptx::mbar_wait_bounded(acc_bar, 0, kWaitLimitNs, p.err_flag, abort_flag) && !*abort_flag;
+        double part = 0.0;
         if (ok) {
             ptx::tc_fence_after();
             const int gm = m0 + r;
             float *crow = p.C + ((size_t)z * p.M + gm) * p.N + n0;
+            const size_t xrow = (size_t)gm * p.N + n0;
+            const void *xz = p.has_dot ? p.dot_x.p[z] : nullptr;
 #pragma unroll 1
             for (int c = 0; c < kTile / 32; ++c) {
                 uint32_t v[32];
                 ptx::tmem_ld32(tmem + lane_off + c * 32, v);
                 ptx::tmem_wait_ld();
-                if (gm < p.M) {
+                if (p.has_dot && gm < p.M) {
+                    // products of two floats are exact in double; summed in a fixed order. The row's
+                    // 32 values are read as 16-byte vectors (N is a multiple of 128).
+                    float x[32];
+                    if (p.dot_x_bf16) {
+                        const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const bf16 *>(xz) + xrow + c * 32);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const uint4 w = src[u];
+                            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                x[8 * u + 2 * e] = __uint_as_float(ww[e] << 16);
+                                x[8 * u + 2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
+                            }
+                        }
+                    } else {
+                        const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(xz) + xrow + c * 32);
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const float4 w = src[u];
+                            x[4 * u] = w.x; x[4 * u + 1] = w.y; x[4 * u + 2] = w.z; x[4 * u + 3] = w.w;
+                        }
+                    }
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) part += (double)__uint_as_float(v[q]) * (double)x[q];
+                }
+                if (p.write_c && gm < p.M) {
 #pragma unroll
                     for (int q = 0; q < 32; q += 4) {
                         if (n0 + c * 32 + q + 3 < p.N) {
@@ -173,6 +211,16 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
                     }
                 }
             }
+        }
+        if (p.has_dot) {
+            // the tile's partial: warp sums, then warp 4 adds the four warps' sums in order
+            for (int o = 16; o > 0; o >>= 1) part += __shfl_down_sync(0xffffffffu, part, o);
+            double *red = reinterpret_cast<double *>(smem + kBarOff + 64);
+            if (lane == 0) red[wq] = part;
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (wq == 0 && lane == 0)
+                p.dot_out[(size_t)z * gridDim.x * gridDim.y + blockIdx.y * gridDim.x + blockIdx.x] =
+                    ok ? ((red[0] + red[1]) + red[2]) + red[3] : 0.0;
         }
     }
     ptx::tc_fence_before();
@@ -277,8 +325,11 @@ cudaError_t launch_split_tf32(const PtrBatch &src, ElemType t, float *hi, float 
 // null) transposed, [batch][N][K], all contiguous float32. M, N multiples of 128; K of 32.
 // a_tri: 1 when A is lower triangular, 2 when upper triangular (then M = K): the zero part of A
 // is not read.
+// dot_x (optional; per batch entry z a [M][N] float32 or bf16 row-major matrix X_z): dot_out[z][t] =
+// sum over output tile t (m-tile major) of C_ij * X_z[i][j] in double; C is written only if write_c.
 cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh, const float *Bl, float *C, int M,
-                               int N, int K, int batch, int *err_flag, cudaStream_t s, int a_tri) {
+                               int N, int K, int batch, int *err_flag, cudaStream_t s, int a_tri, const PtrBatch *dot_x,
+                               bool dot_x_bf16, double *dot_out, bool write_c) {
     if (M % kTile || N % kTile || K % kKStep || batch <= 0) return cudaErrorInvalidValue;
     CUtensorMap ah, al, bh, bl;
     if (!make_map(&ah, Ah, batch, M, K, kTile) || !make_map(&al, Al, batch, M, K, kTile) ||
@@ -288,6 +339,11 @@ cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh
     p.C = C; p.M = M; p.N = N; p.K = K;
     p.three_terms = Bl != nullptr;
     p.a_tri = (a_tri == 1 || a_tri == 2) && M == K ? a_tri : 0;
+    p.has_dot = (dot_out && dot_x) ? 1 : 0;
+    if (p.has_dot) p.dot_x = *dot_x;
+    p.dot_x_bf16 = dot_x_bf16 ? 1 : 0;
+    p.dot_out = dot_out;
+    p.write_c = (write_c || !p.has_dot) ? 1 : 0;
     p.err_flag = err_flag;
     cudaError_t e = cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;

@@ -260,40 +260,41 @@ cudaError_t error_terms(const PtrBatch &G, const PtrBatch &H, const PtrBatch &W,
     float *Ahi = split, *Alo = split + bn, *Bhi = split + 2 * bn, *Blo = split + 3 * bn;
     float *Whi = split + 4 * bn, *Wlo = wt == ElemType::BF16 ? nullptr : split + 5 * bn;
     const dim3 rgrid(nparts, batch);
-    GemmDesc full{D, D, D, D, D, D, true, false, ElemType::F32, ElemType::F32, ElemType::F32, 1.f, 0.f, false, batch};
-    // t0 = tr(dW^T G dW)
+    const bool wbf = wt == ElemType::BF16;
+    double *t_dgd = terms, *t_dy = terms + (size_t)batch * nparts, *t_whw = terms + 2 * (size_t)batch * nparts,
+           *t_wgw = terms + 3 * (size_t)batch * nparts;
     if (tc) {
+        // the traces come out of the GEMM epilogues (one partial per output tile: nparts = tiles);
+        // t4 = tr(W^T Y) was taken when Y = C W was formed
         ISPA_TRY(launch_split_tf32(G, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
         ISPA_TRY(launch_split_tf32(dW, ElemType::F32, Bhi, Blo, D, D, true, batch, s));
-        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Bhi, Blo, Pc, D, D, D, batch, err_flag, s));
-    } else {
-        ISPA_TRY(launch_gemm_simt(full, make_gemm_batch(G, 0, dW, 0, P, 0, batch, 4, 4), s));
-    }
-    dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, P, n, terms + 0 * (size_t)batch * nparts); note_launch();
-    // t1 = tr(dW^T C W)
-    dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, Y, n, terms + 1 * (size_t)batch * nparts); note_launch();
-    // t3 = tr(W^T G W) first while G's split is in place, then t2 = tr(W^T H W); t4 = tr(W^T C W)
-    GemmDesc fw = full;
-    fw.b_type = wt;
-    if (tc) {
-        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Pc, D, D, D, batch, err_flag, s));
-    } else {
-        ISPA_TRY(launch_gemm_simt(fw, make_gemm_batch(G, 0, W, 0, P, 0, batch, 4, ew), s));
-    }
-    if (wt == ElemType::BF16) { dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, P, n, terms + 3 * (size_t)batch * nparts); note_launch(); }
-    else { dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, P, n, terms + 3 * (size_t)batch * nparts); note_launch(); }
-    if (tc) {
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Bhi, Blo, Pc, D, D, D, batch, err_flag, s, 0, &dW, false, t_dgd,
+                                    false));
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Pc, D, D, D, batch, err_flag, s, 0, &W, wbf, t_wgw,
+                                    false));
         ISPA_TRY(launch_split_tf32(H, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
-        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Pc, D, D, D, batch, err_flag, s));
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Pc, D, D, D, batch, err_flag, s, 0, &W, wbf, t_whw,
+                                    false));
+        dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, Y, n, t_dy); note_launch();
     } else {
+        GemmDesc full{D, D, D, D, D, D, true, false, ElemType::F32, ElemType::F32, ElemType::F32, 1.f, 0.f, false, batch};
+        // t0 = tr(dW^T G dW)
+        ISPA_TRY(launch_gemm_simt(full, make_gemm_batch(G, 0, dW, 0, P, 0, batch, 4, 4), s));
+        dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, P, n, t_dgd); note_launch();
+        // t1 = tr(dW^T C W)
+        dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, Y, n, t_dy); note_launch();
+        // t3 = tr(W^T G W), t2 = tr(W^T H W), t4 = tr(W^T C W)
+        GemmDesc fw = full;
+        fw.b_type = wt;
+        ISPA_TRY(launch_gemm_simt(fw, make_gemm_batch(G, 0, W, 0, P, 0, batch, 4, ew), s));
+        if (wbf) { dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, P, n, t_wgw); note_launch(); }
+        else { dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, P, n, t_wgw); note_launch(); }
         ISPA_TRY(launch_gemm_simt(fw, make_gemm_batch(H, 0, W, 0, P, 0, batch, 4, ew), s));
-    }
-    if (wt == ElemType::BF16) { dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, P, n, terms + 2 * (size_t)batch * nparts); note_launch(); }
-    else { dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, P, n, terms + 2 * (size_t)batch * nparts); note_launch(); }
-    if (wt == ElemType::BF16) {
-        dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, Y, n, terms + 4 * (size_t)batch * nparts); note_launch();
-    } else {
-        dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, Y, n, terms + 4 * (size_t)batch * nparts); note_launch();
+        if (wbf) { dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, P, n, t_whw); note_launch(); }
+        else { dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, P, n, t_whw); note_launch(); }
+        double *t_wy = terms + 4 * (size_t)batch * nparts;
+        if (wbf) { dot_partials_kernel<bf16><<<rgrid, 256, 0, s>>>(W, Y, n, t_wy); note_launch(); }
+        else { dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, Y, n, t_wy); note_launch(); }
     }
     ISPA_TRY(cudaGetLastError());
     finalize_eps_kernel<<<(batch + 63) / 64, 64, 0, s>>>(terms, nparts, batch, status, eps, err_terms); note_launch();
@@ -304,7 +305,7 @@ cudaError_t error_terms(const PtrBatch &G, const PtrBatch &H, const PtrBatch &W,
 
 // Y = C W for one batch of layers (W split into Whi/Wlo first when tc).
 static cudaError_t c_times_w(const PtrBatch &C, const PtrBatch &W, ElemType wt, const PtrBatch &Y, float *Yc,
-                             float *split, int D, int batch, int *err_flag, bool tc, cudaStream_t s) {
+                             float *split, double *t_wy, int D, int batch, int *err_flag, bool tc, cudaStream_t s) {
     const size_t n = (size_t)D * D;
     const size_t ew = wt == ElemType::BF16 ? 2 : 4;
     const size_t bn = (size_t)batch * n;
@@ -313,7 +314,9 @@ static cudaError_t c_times_w(const PtrBatch &C, const PtrBatch &W, ElemType wt, 
     if (tc) {
         ISPA_TRY(launch_split_tf32(W, wt, Whi, Wlo, D, D, true, batch, s));
         ISPA_TRY(launch_split_tf32(C, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
-        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Yc, D, D, D, batch, err_flag, s));
+        // Y = C W, with t4 = tr(W^T Y) from the epilogue
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Yc, D, D, D, batch, err_flag, s, 0, &W,
+                                    wt == ElemType::BF16, t_wy, true));
     } else {
         GemmDesc d{D, D, D, D, D, D, true, false, ElemType::F32, wt, ElemType::F32, 1.f, 0.f, false, batch};
         ISPA_TRY(launch_gemm_simt(d, make_gemm_batch(C, 0, W, 0, Y, 0, batch, 4, ew), s));
@@ -328,7 +331,7 @@ cudaError_t error_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
                         double *terms, int nparts, float *eps, double *err_terms, int D, int batch, int *err_flag,
                         cudaStream_t s) {
     const bool tc = (D % 128 == 0) && split != nullptr;
-    ISPA_TRY(c_times_w(C, W, wt, Y, Yc, split, D, batch, err_flag, tc, s));
+    ISPA_TRY(c_times_w(C, W, wt, Y, Yc, split, terms + 4 * (size_t)batch * nparts, D, batch, err_flag, tc, s));
     return error_terms(G, H, W, wt, dW, Y, P, Pc, split, terms, nparts, nullptr, eps, err_terms, D, batch, err_flag,
                        tc, s);
 }
@@ -354,7 +357,7 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
     ISPA_TRY(cudaGetLastError());
 
     // Y = C W
-    ISPA_TRY(c_times_w(C, W, wt, Y, Yc, split, D, batch, err_flag, tc, s));
+    ISPA_TRY(c_times_w(C, W, wt, Y, Yc, split, terms + 4 * (size_t)batch * nparts, D, batch, err_flag, tc, s));
 
     // Cholesky factorisation, blocked
     const int nblk = D / NB;
