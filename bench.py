@@ -76,10 +76,16 @@ def parse_args(argv=None):
 # The path is the episode's: one ispa_attn_split_ops launch per warmup layer call and one batched
 # ispa_accum_ops launch per chunk, whose bytes are charged to the chunk's layers equally.
 # None: not yet captured for the current sources.
+_PTX = ("streaming_video_attention_b200/csrc/ptx.cuh",
+        "0353fca5187d1129c0e7936a8baa86b17e79672c07a933ea5a5f127e77d94af0")
 CAPTURED_TRAFFIC = {
     "workload": "1p3b_bf16",
-    "attention": {"two_group": (None, {})},
-    "stats_per_layer": (None, {}),
+    # the 90 warmup launches of one timed episode, averaged (n_kv 28,080 / 32,760 / 37,440)
+    "attention": {"two_group": (240.3e6, dict([_PTX, ("streaming_video_attention_b200/csrc/attn2g_sm100.cu",
+                                                      "3bed3806f2e152d01cb932a529d3f79da812540a4b19e6fbb52febc93f129433")]))},
+    # the episode's three 30-layer statistics launches (3.08 GB each), per layer
+    "stats_per_layer": (102.75e6, dict([_PTX, ("streaming_video_attention_b200/csrc/stats_sm100.cu",
+                                               "b6b42e9369b57a364c239b9be97ce127908ae56800a6f12cfa6448475cd0e748")])),
 }
 
 
