@@ -115,9 +115,17 @@ struct PtrBatch {
 // 3xTF32 tensor-core GEMM for D x D products (gemm_tf32_sm100.cu).
 cudaError_t launch_split_tf32(const PtrBatch &src, ElemType t, float *hi, float *lo, int rows, int cols,
                               bool transpose, int batch, cudaStream_t s);
+struct Tf32Opts {
+    int a_tri = 0;                      // 1: A lower triangular, 2: A upper triangular (M = K)
+    bool sym = false;                   // B is A: only output tiles on and below the diagonal
+    const PtrBatch *dot_x = nullptr;    // trace partials against X (float32 or bf16)
+    bool dot_x_bf16 = false;
+    double *dot_out = nullptr;
+    const PtrBatch *dot_x2 = nullptr;   // a second float32 X
+    double *dot_out2 = nullptr;
+    bool write_c = true;
+};
 cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh, const float *Bl, float *C, int M,
-                               int N, int K, int batch, int *err_flag, cudaStream_t s, int a_tri = 0,
-                               const PtrBatch *dot_x = nullptr, bool dot_x_bf16 = false, double *dot_out = nullptr,
-                               bool write_c = true);
+                               int N, int K, int batch, int *err_flag, cudaStream_t s, const Tf32Opts &o = Tf32Opts());
 
 }  // namespace ispa

@@ -1,5 +1,6 @@
 // Float32-accurate batched GEMM on the sm_100a tensor cores (3xTF32), for the absorb solve's
-// D x D products [ISPA §3.2, §3.3]: Y = C W, and G dW, H W, G W for the error traces.
+// D x D products [ISPA §3.2, §3.3]: Y = C W, the two products with L^-1, and the Gram products
+// W W^T and dW dW^T whose dots with G and H give the error traces.
 //
 // Each float32 operand X is split once into X_hi = X rounded to TF32 (11 significant bits)
 // and X_lo = X - X_hi (exact in float32; the tensor core keeps its leading 11 bits). The
@@ -43,15 +44,18 @@ __host__ __device__ constexpr uint32_t make_idesc_tf32(int M, int N, bool b_mn) 
 struct Tf32Params {
     float *C;
     int M, N, K;
-    int three_terms;    // B_lo present
+    int a_lo;           // A_lo present (absent: A is exact in TF32, e.g. bf16)
+    int b_lo;           // B_lo present
     int a_tri;          // 0: A full; 1: A lower triangular (k < m0 + 128); 2: A upper triangular (k >= m0)
-    // optional trace partial: dot_out[z][tile] = sum over the tile of C_ij * X_z[i][j] (double),
-    // X_z [M][N] row-major float32 or bf16 (one pointer per batch entry); C is written only if
-    // write_c
-    PtrBatch dot_x;
-    int has_dot;
+    int sym;            // C = A A^T: only tiles with n0 <= m0 run (B is A)
+    // optional trace partials: dot_out[z][tile] = sum over the tile of C_ij * X_z[i][j] (double),
+    // X_z [M][N] row-major float32 or bf16 (one pointer per batch entry); with sym, an off-diagonal
+    // tile also adds C_ij * X_z[j][i] (its mirror's share), and the skipped tiles write 0. A second
+    // float32 X (dot_x2 -> dot_out2) may ride along. C is written only if write_c.
+    PtrBatch dot_x, dot_x2;
+    int has_dot, has_dot2;
     int dot_x_bf16;
-    double *dot_out;
+    double *dot_out, *dot_out2;
     int write_c;
     int *err_flag;
 };
@@ -73,13 +77,22 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int n0 = blockIdx.x * kTile, m0 = blockIdx.y * kTile, z = blockIdx.z;
+    const size_t part_idx = (size_t)z * gridDim.x * gridDim.y + blockIdx.y * gridDim.x + blockIdx.x;
+    if (p.sym && n0 > m0) {
+        // the mirror tile (n0, m0) accounts for this one
+        if (threadIdx.x == 0) {
+            if (p.has_dot) p.dot_out[part_idx] = 0.0;
+            if (p.has_dot2) p.dot_out2[part_idx] = 0.0;
+        }
+        return;
+    }
     // k-steps of this output row tile: a triangular A is zero outside [kt0, kt1), and skipping
     // exact zeros changes no sum
     const int n_kall = (p.K + kKStep - 1) / kKStep;
     const int kt0 = p.a_tri == 2 ? m0 / kKStep : 0;
     const int kt1 = p.a_tri == 1 ? min(n_kall, (m0 + kTile) / kKStep) : n_kall;
     const int n_k = kt1 - kt0;
-    const uint32_t stage_tx = (p.three_terms ? 4 : 3) * kOpBytes;
+    const uint32_t stage_tx = (2 + p.a_lo + p.b_lo) * kOpBytes;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -113,9 +126,9 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
             ptx::mbar_arrive_expect_tx_warp(&full[s], stage_tx);
             const int k0 = (kt0 + kt) * kKStep;
             ptx::tma_load_3d_warp(base, &tAh, &full[s], k0, m0, z, pol);
-            ptx::tma_load_3d_warp(base + kOpBytes, &tAl, &full[s], k0, m0, z, pol);
+            if (p.a_lo) ptx::tma_load_3d_warp(base + kOpBytes, &tAl, &full[s], k0, m0, z, pol);
             ptx::tma_load_3d_warp(base + 2 * kOpBytes, &tBh, &full[s], k0, n0, z, pol);
-            if (p.three_terms) ptx::tma_load_3d_warp(base + 3 * kOpBytes, &tBl, &full[s], k0, n0, z, pol);
+            if (p.b_lo) ptx::tma_load_3d_warp(base + 3 * kOpBytes, &tBl, &full[s], k0, n0, z, pol);
             issued = kt;
         }
         if (!ok)
@@ -137,13 +150,17 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
                 const uint64_t dah = ptx::make_sdesc_sw128(ah + kk * 32, 16, 1024);
                 const uint64_t dal = ptx::make_sdesc_sw128(al + kk * 32, 16, 1024);
                 const uint64_t dbh = ptx::make_sdesc_sw128(bh + kk * 32, 16, 1024);
-                const uint32_t first = (kt == 0 && kk == 0) ? 0u : 1u;
-                ptx::umma_tf32_ss_warp(tmem, dal, dbh, idesc, first);
-                if (p.three_terms) {
-                    const uint64_t dbl = ptx::make_sdesc_sw128(bl + kk * 32, 16, 1024);
-                    ptx::umma_tf32_ss_warp(tmem, dah, dbl, idesc, 1u);
+                uint32_t acc = (kt == 0 && kk == 0) ? 0u : 1u;
+                if (p.a_lo) {
+                    ptx::umma_tf32_ss_warp(tmem, dal, dbh, idesc, acc);
+                    acc = 1u;
                 }
-                ptx::umma_tf32_ss_warp(tmem, dah, dbh, idesc, 1u);
+                if (p.b_lo) {
+                    const uint64_t dbl = ptx::make_sdesc_sw128(bl + kk * 32, 16, 1024);
+                    ptx::umma_tf32_ss_warp(tmem, dah, dbl, idesc, acc);
+                    acc = 1u;
+                }
+                ptx::umma_tf32_ss_warp(tmem, dah, dbh, idesc, acc);
             }
             ptx::umma_commit_warp(&empty[s]);
         }
@@ -158,13 +175,16 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
         const int r = wq * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
         const bool ok = ptx::mbar_wait_bounded(acc_bar, 0, kWaitLimitNs, p.err_flag, abort_flag) && !*abort_flag;
-        double part = 0.0;
+        // the mirror's share of a symmetric product's off-diagonal tile
+        const bool mirror = p.sym && m0 != n0;
+        double part = 0.0, part2 = 0.0;
         if (ok) {
             ptx::tc_fence_after();
             const int gm = m0 + r;
             float *crow = p.C + ((size_t)z * p.M + gm) * p.N + n0;
             const size_t xrow = (size_t)gm * p.N + n0;
             const void *xz = p.has_dot ? p.dot_x.p[z] : nullptr;
+            const float *x2z = p.has_dot2 ? static_cast<const float *>(p.dot_x2.p[z]) : nullptr;
 #pragma unroll 1
             for (int c = 0; c < kTile / 32; ++c) {
                 uint32_t v[32];
@@ -196,6 +216,32 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
                     }
 #pragma unroll
                     for (int q = 0; q < 32; ++q) part += (double)__uint_as_float(v[q]) * (double)x[q];
+                    if (mirror) {
+                        // X[n0 + c*32 + q][gm]: the warp's 32 rows read one 128-byte run per q
+                        const float *xt = static_cast<const float *>(xz) + (size_t)(n0 + c * 32) * p.N + gm;
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) x[q] = xt[(size_t)q * p.N];
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) part += (double)__uint_as_float(v[q]) * (double)x[q];
+                    }
+                }
+                if (p.has_dot2 && gm < p.M) {
+                    float x[32];
+                    const float4 *src = reinterpret_cast<const float4 *>(x2z + xrow + c * 32);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const float4 w = src[u];
+                        x[4 * u] = w.x; x[4 * u + 1] = w.y; x[4 * u + 2] = w.z; x[4 * u + 3] = w.w;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) part2 += (double)__uint_as_float(v[q]) * (double)x[q];
+                    if (mirror) {
+                        const float *xt = x2z + (size_t)(n0 + c * 32) * p.N + gm;
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) x[q] = xt[(size_t)q * p.N];
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) part2 += (double)__uint_as_float(v[q]) * (double)x[q];
+                    }
                 }
                 if (p.write_c && gm < p.M) {
 #pragma unroll
@@ -212,15 +258,22 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
                 }
             }
         }
-        if (p.has_dot) {
-            // the tile's partial: warp sums, then warp 4 adds the four warps' sums in order
-            for (int o = 16; o > 0; o >>= 1) part += __shfl_down_sync(0xffffffffu, part, o);
+        if (p.has_dot || p.has_dot2) {
+            // the tile's partials: warp sums, then warp 4 adds the four warps' sums in order
+            for (int o = 16; o > 0; o >>= 1) {
+                part += __shfl_down_sync(0xffffffffu, part, o);
+                part2 += __shfl_down_sync(0xffffffffu, part2, o);
+            }
             double *red = reinterpret_cast<double *>(smem + kBarOff + 64);
-            if (lane == 0) red[wq] = part;
+            if (lane == 0) {
+                red[wq] = part;
+                red[4 + wq] = part2;
+            }
             asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (wq == 0 && lane == 0)
-                p.dot_out[(size_t)z * gridDim.x * gridDim.y + blockIdx.y * gridDim.x + blockIdx.x] =
-                    ok ? ((red[0] + red[1]) + red[2]) + red[3] : 0.0;
+            if (wq == 0 && lane == 0) {
+                if (p.has_dot) p.dot_out[part_idx] = ok ? ((red[0] + red[1]) + red[2]) + red[3] : 0.0;
+                if (p.has_dot2) p.dot_out2[part_idx] = ok ? ((red[4] + red[5]) + red[6]) + red[7] : 0.0;
+            }
         }
     }
     ptx::tc_fence_before();
@@ -321,29 +374,39 @@ cudaError_t launch_split_tf32(const PtrBatch &src, ElemType t, float *hi, float 
     return cudaGetLastError();
 }
 
-// C[z] = A[z] B[z] for z < batch; A given as (A_hi, A_lo) [batch][M][K], B as (B_hi, B_lo or
-// null) transposed, [batch][N][K], all contiguous float32. M, N multiples of 128; K of 32.
-// a_tri: 1 when A is lower triangular, 2 when upper triangular (then M = K): the zero part of A
-// is not read.
-// dot_x (optional; per batch entry z a [M][N] float32 or bf16 row-major matrix X_z): dot_out[z][t] =
-// sum over output tile t (m-tile major) of C_ij * X_z[i][j] in double; C is written only if write_c.
+// C[z] = A[z] B[z] for z < batch; A given as (A_hi, A_lo or null) [batch][M][K], B as (B_hi,
+// B_lo or null) transposed, [batch][N][K], all contiguous float32 (a null lo part: that operand
+// is exact in TF32). M, N multiples of 128; K of 32. Options (Tf32Opts):
+//   a_tri: 1 when A is lower triangular, 2 when upper triangular (then M = K): the zero part of
+//          A is not read;
+//   sym:   B is A (M = N): only the output tiles on and below the diagonal are formed;
+//   dot_x / dot_out (and dot_x2 / dot_out2, float32): per batch entry z a [M][N] row-major X_z;
+//          dot_out[z][t] = sum over output tile t (m-tile major) of C_ij * X_z[i][j] in double,
+//          with sym also C_ij * X_z[j][i] off the diagonal (so the partials add up to
+//          sum_ij (A A^T)_ij X_ij);
+//   write_c: C is written (always, when no dot is asked for).
 cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh, const float *Bl, float *C, int M,
-                               int N, int K, int batch, int *err_flag, cudaStream_t s, int a_tri, const PtrBatch *dot_x,
-                               bool dot_x_bf16, double *dot_out, bool write_c) {
+                               int N, int K, int batch, int *err_flag, cudaStream_t s, const Tf32Opts &o) {
     if (M % kTile || N % kTile || K % kKStep || batch <= 0) return cudaErrorInvalidValue;
+    if (o.sym && (M != N || o.dot_x_bf16 || o.a_tri)) return cudaErrorInvalidValue;
     CUtensorMap ah, al, bh, bl;
-    if (!make_map(&ah, Ah, batch, M, K, kTile) || !make_map(&al, Al, batch, M, K, kTile) ||
+    if (!make_map(&ah, Ah, batch, M, K, kTile) || !make_map(&al, Al ? Al : Ah, batch, M, K, kTile) ||
         !make_map(&bh, Bh, batch, N, K, kTile) || !make_map(&bl, Bl ? Bl : Bh, batch, N, K, kTile))
         return cudaErrorInvalidValue;
     Tf32Params p;
     p.C = C; p.M = M; p.N = N; p.K = K;
-    p.three_terms = Bl != nullptr;
-    p.a_tri = (a_tri == 1 || a_tri == 2) && M == K ? a_tri : 0;
-    p.has_dot = (dot_out && dot_x) ? 1 : 0;
-    if (p.has_dot) p.dot_x = *dot_x;
-    p.dot_x_bf16 = dot_x_bf16 ? 1 : 0;
-    p.dot_out = dot_out;
-    p.write_c = (write_c || !p.has_dot) ? 1 : 0;
+    p.a_lo = Al != nullptr;
+    p.b_lo = Bl != nullptr;
+    p.a_tri = (o.a_tri == 1 || o.a_tri == 2) && M == K ? o.a_tri : 0;
+    p.sym = o.sym ? 1 : 0;
+    p.has_dot = (o.dot_out && o.dot_x) ? 1 : 0;
+    if (p.has_dot) p.dot_x = *o.dot_x;
+    p.has_dot2 = (o.dot_out2 && o.dot_x2) ? 1 : 0;
+    if (p.has_dot2) p.dot_x2 = *o.dot_x2;
+    p.dot_x_bf16 = o.dot_x_bf16 ? 1 : 0;
+    p.dot_out = o.dot_out;
+    p.dot_out2 = o.dot_out2;
+    p.write_c = (o.write_c || !(p.has_dot || p.has_dot2)) ? 1 : 0;
     p.err_flag = err_flag;
     cudaError_t e = cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;

@@ -9,12 +9,16 @@
 //                                             Z = X (C W) and dW = X^T Z on the tensor
 //                                             cores (3xTF32); otherwise trsv_block + GEMM
 //                                             per block, both ways, on (C W) itself
-//   five traces -> E^2, T^2, eps              GEMMs G dW, H W, G W, then dot_partials
+//   five traces -> E^2, T^2, eps              tensor cores: the Gram products W W^T and
+//                                             dW dW^T (lower tiles only) dotted with G and H,
+//                                             and tr(W^T C W), tr(dW^T C W), in the GEMM
+//                                             epilogues; otherwise GEMMs G dW, H W, G W, then
+//                                             dot_partials
 //
 // Block size nb = 64 (D must be a multiple of 64). Each 64 x 64 diagonal block is factored
 // (potrf_diag) and each panel below it solved (trsm_panel) by CTAs whose threads hold one row
-// of the block in registers; everything of order D^3 runs in batched GEMMs. A non-positive pivot marks the layer ISPA_ERR_NOT_SPD and turns its results to
-// NaN; nothing traps.
+// of the block in registers; everything of order D^3 runs in batched GEMMs. A non-positive
+// pivot marks the layer ISPA_ERR_NOT_SPD and turns its results to NaN; nothing traps.
 #include "common.cuh"
 
 namespace ispa {
@@ -36,12 +40,12 @@ __global__ void fill_shifted_kernel(PtrBatch src, PtrBatch dst, int D, float lam
 
 // Cholesky factor of the NB x NB diagonal block at (k0, k0), in place (lower triangle). One
 // CTA of NB threads per layer; thread i holds row i of the block in registers (the column loop
-// is unrolled so that every index is a constant). Column j: the pivot's square root, then each
-// row below scales its element of column j and publishes it, then each row subtracts its
-// rank-1 update from its remaining lower-triangle elements.
+// is unrolled so that every index is a constant). Column j: each row publishes its element of
+// column j (double-buffered, so one barrier per column), then every row reads the pivot d,
+// subtracts a_ij a_kj / d from its elements k in (j, i] and scales its own a_ij by 1/sqrt(d)
+// (L_ij = a_ij / sqrt(d), L_jj = d / sqrt(d)).
 __global__ void __launch_bounds__(NB) potrf_diag_kernel(PtrBatch M, int D, int k0, int *status) {
-    __shared__ float col[NB];
-    __shared__ float piv;
+    __shared__ float col[2][NB];
     const int z = blockIdx.x;
     float *Mz = static_cast<float *>(M.p[z]);
     const int i = threadIdx.x;
@@ -55,47 +59,45 @@ __global__ void __launch_bounds__(NB) potrf_diag_kernel(PtrBatch M, int D, int k
     bool bad = false;
 #pragma unroll
     for (int j = 0; j < NB; ++j) {
-        if (i == j) {
-            float d = a[j];
-            if (!(d > 0.f)) {
-                bad = true;
-                d = __int_as_float(0x7fc00000);
-            } else {
-                d = sqrtf(d);
-            }
-            a[j] = d;
-            piv = d;
-        }
+        float *cj = col[j & 1];
+        if (i >= j) cj[i] = a[j];
         __syncthreads();
+        const float d = cj[j];
+        float rs = __int_as_float(0x7fc00000);
+        if (d > 0.f) rs = rsqrtf(d);
+        else bad = true;
         if (i > j) {
-            a[j] = a[j] / piv;
-            col[i] = a[j];
-        }
-        __syncthreads();
-        if (i > j) {
+            const float f = a[j] * (rs * rs);
 #pragma unroll
             for (int k = j + 1; k < NB; ++k)
-                if (k <= i) a[k] -= a[j] * col[k];
+                if (k <= i) a[k] -= f * cj[k];
+            a[j] *= rs;
+        } else if (i == j) {
+            a[j] = d * rs;
         }
     }
-    if (bad) status[z] = ISPA_ERR_NOT_SPD;
+    if (bad && i == 0) status[z] = ISPA_ERR_NOT_SPD;
     float *out = Mz + (size_t)(k0 + i) * D + k0;
 #pragma unroll
     for (int c = 0; c < NB; ++c)
         if (c <= i) out[c] = a[c];
 }
 
-// Rows below the diagonal block: L21 = A21 L11^-T (row-wise forward substitution). One CTA of
-// NB threads per NB rows; thread i holds its row of A21 in registers (unrolled loops, constant
-// indices), the factored diagonal block sits in shared memory and is read by broadcast.
+// Rows below the diagonal block: L21 = A21 L11^-T. One CTA of NB threads per NB rows; thread i
+// holds its row of A21 in registers (unrolled loops, constant indices) and substitutes forward
+// column by column, each finished element x_j (times 1/L_jj) subtracted at once from the later
+// ones (x_c -= x_j L_cj), so the dependent chain is one multiply and one FMA per column. The
+// factored diagonal block and its reciprocal pivots sit in shared memory, read by broadcast.
 __global__ void __launch_bounds__(NB) trsm_panel_kernel(PtrBatch M, int D, int k0) {
     __shared__ __align__(16) float Lk[NB][NB];
+    __shared__ float inv[NB];
     const int z = blockIdx.y;
     float *Mz = static_cast<float *>(M.p[z]);
     const int i = threadIdx.x;
     const int r = k0 + NB + blockIdx.x * NB + i;
     // column i of the diagonal block: coalesced reads, conflict-free stores
     for (int rr = 0; rr < NB; ++rr) Lk[rr][i] = i <= rr ? Mz[(size_t)(k0 + rr) * D + k0 + i] : 0.f;
+    inv[i] = 1.f / Mz[(size_t)(k0 + i) * D + k0 + i];
     float x[NB];
     if (r < D) {
         const float *row = Mz + (size_t)r * D + k0;
@@ -109,10 +111,9 @@ __global__ void __launch_bounds__(NB) trsm_panel_kernel(PtrBatch M, int D, int k
     if (r >= D) return;
 #pragma unroll
     for (int j = 0; j < NB; ++j) {
-        float v = x[j];
+        x[j] *= inv[j];
 #pragma unroll
-        for (int c = 0; c < j; ++c) v -= x[c] * Lk[j][c];
-        x[j] = v / Lk[j][j];
+        for (int c = j + 1; c < NB; ++c) x[c] -= x[j] * Lk[c][j];
     }
     float *out = Mz + (size_t)r * D + k0;
 #pragma unroll
@@ -120,10 +121,12 @@ __global__ void __launch_bounds__(NB) trsm_panel_kernel(PtrBatch M, int D, int k
 }
 
 // X_k = L_kk^-1 X_k (forward) or L_kk^-T X_k (backward) for the NB rows of block k,
-// every column of X at once (one thread per column).
+// every column of X at once (one thread per column); each finished element (times the
+// reciprocal pivot) is subtracted at once from the elements still to come.
 template <bool TRANS>
 __global__ void __launch_bounds__(128) trsv_block_kernel(PtrBatch L, PtrBatch X, int D, int k0) {
     __shared__ float Lk[NB][NB + 1];
+    __shared__ float inv[NB];
     const int z = blockIdx.y;
     const float *Lz = static_cast<const float *>(L.p[z]);
     float *Xz = static_cast<float *>(X.p[z]);
@@ -131,6 +134,7 @@ __global__ void __launch_bounds__(128) trsv_block_kernel(PtrBatch L, PtrBatch X,
         const int i = idx / NB, j = idx % NB;
         Lk[i][j] = j <= i ? Lz[(size_t)(k0 + i) * D + k0 + j] : 0.f;
     }
+    if (threadIdx.x < NB) inv[threadIdx.x] = 1.f / Lz[(size_t)(k0 + threadIdx.x) * D + k0 + threadIdx.x];
     __syncthreads();
     const int c = blockIdx.x * blockDim.x + threadIdx.x;
     if (c >= D) return;
@@ -140,18 +144,16 @@ __global__ void __launch_bounds__(128) trsv_block_kernel(PtrBatch L, PtrBatch X,
     if (!TRANS) {
 #pragma unroll
         for (int j = 0; j < NB; ++j) {
-            float v = x[j];
+            x[j] *= inv[j];
 #pragma unroll
-            for (int i = 0; i < j; ++i) v -= Lk[j][i] * x[i];
-            x[j] = v / Lk[j][j];
+            for (int i = j + 1; i < NB; ++i) x[i] -= Lk[i][j] * x[j];
         }
     } else {
 #pragma unroll
         for (int j = NB - 1; j >= 0; --j) {
-            float v = x[j];
+            x[j] *= inv[j];
 #pragma unroll
-            for (int i = j + 1; i < NB; ++i) v -= Lk[i][j] * x[i];
-            x[j] = v / Lk[j][j];
+            for (int i = 0; i < j; ++i) x[i] -= Lk[j][i] * x[j];
         }
     }
 #pragma unroll
@@ -247,35 +249,42 @@ static GemmBatch make_gemm_batch(const PtrBatch &A, size_t offA, const PtrBatch 
         if (e_ != cudaSuccess) return e_;    \
     } while (0)
 
-// The five traces of the error and eps = E^2 / T^2 for dW given, Y = C W already in Y
-// (and W already split when tc): t0 = tr(dW^T G dW), t1 = tr(dW^T Y), t2 = tr(W^T H W),
-// t3 = tr(W^T G W), t4 = tr(W^T Y).
+// The five traces of the error and eps = E^2 / T^2 for dW given, Y = C W already in Y:
+// t0 = tr(dW^T G dW), t1 = tr(dW^T Y), t2 = tr(W^T H W), t3 = tr(W^T G W), t4 = tr(W^T Y).
+// On the tensor cores (tc) the quadratic forms are taken as dots with Gram matrices,
+// tr(X^T S X) = sum_ij S_ij (X X^T)_ij: one symmetric product W W^T (its lower tiles only)
+// dotted with G and H in its epilogue gives t3 and t2, dW dW^T dotted with G gives t0; t4 was
+// taken when Y was formed and t1 too when t1_done (the solve's last product).
 cudaError_t error_terms(const PtrBatch &G, const PtrBatch &H, const PtrBatch &W, ElemType wt, const PtrBatch &dW,
                         const PtrBatch &Y, const PtrBatch &P, float *Pc, float *split, double *terms, int nparts,
                         const int *status, float *eps, double *err_terms, int D, int batch, int *err_flag, bool tc,
-                        cudaStream_t s) {
+                        bool t1_done, cudaStream_t s) {
     const size_t n = (size_t)D * D;
     const size_t ew = wt == ElemType::BF16 ? 2 : 4;
     const size_t bn = (size_t)batch * n;
-    float *Ahi = split, *Alo = split + bn, *Bhi = split + 2 * bn, *Blo = split + 3 * bn;
-    float *Whi = split + 4 * bn, *Wlo = wt == ElemType::BF16 ? nullptr : split + 5 * bn;
+    float *Ahi = split, *Alo = split + bn;
     const dim3 rgrid(nparts, batch);
     const bool wbf = wt == ElemType::BF16;
     double *t_dgd = terms, *t_dy = terms + (size_t)batch * nparts, *t_whw = terms + 2 * (size_t)batch * nparts,
            *t_wgw = terms + 3 * (size_t)batch * nparts;
     if (tc) {
-        // the traces come out of the GEMM epilogues (one partial per output tile: nparts = tiles);
-        // t4 = tr(W^T Y) was taken when Y = C W was formed
-        ISPA_TRY(launch_split_tf32(G, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
-        ISPA_TRY(launch_split_tf32(dW, ElemType::F32, Bhi, Blo, D, D, true, batch, s));
-        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Bhi, Blo, Pc, D, D, D, batch, err_flag, s, 0, &dW, false, t_dgd,
-                                    false));
-        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Pc, D, D, D, batch, err_flag, s, 0, &W, wbf, t_wgw,
-                                    false));
-        ISPA_TRY(launch_split_tf32(H, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
-        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Pc, D, D, D, batch, err_flag, s, 0, &W, wbf, t_whw,
-                                    false));
-        dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, Y, n, t_dy); note_launch();
+        // W W^T (a bf16 W is exact in TF32: one term), dotted with G -> t3 and H -> t2
+        ISPA_TRY(launch_split_tf32(W, wt, Ahi, wbf ? nullptr : Alo, D, D, false, batch, s));
+        Tf32Opts ow;
+        ow.sym = true;
+        ow.dot_x = &G; ow.dot_out = t_wgw;
+        ow.dot_x2 = &H; ow.dot_out2 = t_whw;
+        ow.write_c = false;
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, wbf ? nullptr : Alo, Ahi, wbf ? nullptr : Alo, Pc, D, D, D, batch, err_flag,
+                                    s, ow));
+        // dW dW^T dotted with G -> t0
+        ISPA_TRY(launch_split_tf32(dW, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
+        Tf32Opts od;
+        od.sym = true;
+        od.dot_x = &G; od.dot_out = t_dgd;
+        od.write_c = false;
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Ahi, Alo, Pc, D, D, D, batch, err_flag, s, od));
+        if (!t1_done) { dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, Y, n, t_dy); note_launch(); }
     } else {
         GemmDesc full{D, D, D, D, D, D, true, false, ElemType::F32, ElemType::F32, ElemType::F32, 1.f, 0.f, false, batch};
         // t0 = tr(dW^T G dW)
@@ -315,8 +324,9 @@ static cudaError_t c_times_w(const PtrBatch &C, const PtrBatch &W, ElemType wt, 
         ISPA_TRY(launch_split_tf32(W, wt, Whi, Wlo, D, D, true, batch, s));
         ISPA_TRY(launch_split_tf32(C, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
         // Y = C W, with t4 = tr(W^T Y) from the epilogue
-        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Yc, D, D, D, batch, err_flag, s, 0, &W,
-                                    wt == ElemType::BF16, t_wy, true));
+        Tf32Opts o;
+        o.dot_x = &W; o.dot_x_bf16 = wt == ElemType::BF16; o.dot_out = t_wy;
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Yc, D, D, D, batch, err_flag, s, o));
     } else {
         GemmDesc d{D, D, D, D, D, D, true, false, ElemType::F32, wt, ElemType::F32, 1.f, 0.f, false, batch};
         ISPA_TRY(launch_gemm_simt(d, make_gemm_batch(C, 0, W, 0, Y, 0, batch, 4, ew), s));
@@ -333,7 +343,7 @@ cudaError_t error_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
     const bool tc = (D % 128 == 0) && split != nullptr;
     ISPA_TRY(c_times_w(C, W, wt, Y, Yc, split, terms + 4 * (size_t)batch * nparts, D, batch, err_flag, tc, s));
     return error_terms(G, H, W, wt, dW, Y, P, Pc, split, terms, nparts, nullptr, eps, err_terms, D, batch, err_flag,
-                       tc, s);
+                       tc, false, s);
 }
 
 // Solve for one batch of layers. All pointers are device pointers, one per layer.
@@ -400,10 +410,16 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
         float *dWc = static_cast<float *>(dW.p[0]);
         ISPA_TRY(launch_split_tf32(P, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
         ISPA_TRY(launch_split_tf32(Y, ElemType::F32, Bhi, Blo, D, D, true, batch, s));
-        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Bhi, Blo, dWc, D, D, D, batch, err_flag, s, 1));   // X lower
+        Tf32Opts oz;
+        oz.a_tri = 1;   // X lower
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Bhi, Blo, dWc, D, D, D, batch, err_flag, s, oz));
         ISPA_TRY(launch_split_tf32(P, ElemType::F32, Ahi, Alo, D, D, true, batch, s));
         ISPA_TRY(launch_split_tf32(dW, ElemType::F32, Bhi, Blo, D, D, true, batch, s));
-        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Bhi, Blo, dWc, D, D, D, batch, err_flag, s, 2));   // X^T upper
+        // X^T upper; t1 = tr(dW^T Y) from the epilogue
+        Tf32Opts od;
+        od.a_tri = 2;
+        od.dot_x = &Y; od.dot_out = terms + (size_t)batch * nparts;
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Bhi, Blo, dWc, D, D, D, batch, err_flag, s, od));
     } else {
         // dW <- Y, solved in place: forward substitution L Z = Y, then backward L^T X = Z
         copy_f32_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(Y, dW, n); note_launch();
@@ -435,7 +451,7 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
 
     // Reconstruction error terms
     ISPA_TRY(error_terms(G, H, W, wt, dW, Y, P, Pc, split, terms, nparts, status, eps, err_terms, D, batch, err_flag,
-                         tc, s));
+                         tc, tc, s));
 
     if (w_new) {
         if (wt == ElemType::BF16) { add_delta_kernel<bf16><<<dim3(fill_blocks, batch), 256, 0, s>>>(W, dW, *w_new, n); note_launch(); }
