@@ -112,6 +112,11 @@ struct PtrBatch {
     void *p[kMaxBatch];
 };
 
+// M = G + lambda I = L L^T and X = L^-1 into P, float32, one cluster of CTAs per layer
+// (chol_inv_sm100.cu); status[z] = ISPA_ERR_NOT_SPD on a non-positive pivot.
+cudaError_t launch_chol_inv(const PtrBatch &G, const PtrBatch &M, const PtrBatch &P, int D, float lambda, int batch,
+                            int *status, cudaStream_t s);
+
 // 3xTF32 tensor-core GEMM for D x D products (gemm_tf32_sm100.cu).
 cudaError_t launch_split_tf32(const PtrBatch &src, ElemType t, float *hi, float *lo, int rows, int cols,
                               bool transpose, int batch, cudaStream_t s);
@@ -123,6 +128,9 @@ struct Tf32Opts {
     double *dot_out = nullptr;
     const PtrBatch *dot_x2 = nullptr;   // a second float32 X
     double *dot_out2 = nullptr;
+    float *split_hi = nullptr;          // C's TF32 split (hi, lo), [batch][M][N] or transposed
+    float *split_lo = nullptr;
+    bool split_t = false;
     bool write_c = true;
 };
 cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh, const float *Bl, float *C, int M,

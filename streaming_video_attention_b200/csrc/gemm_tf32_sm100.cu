@@ -6,15 +6,16 @@
 // and X_lo = X - X_hi (exact in float32; the tensor core keeps its leading 11 bits). The
 // product is accumulated in float32 TMEM as A_hi B_hi + A_hi B_lo + A_lo B_hi; the dropped
 // A_lo B_lo term and the truncation of the lo parts are ~2^-22 relative, i.e. float32-level
-// accuracy. A bf16 operand is exact in TF32 (lo = 0) and costs two terms instead of three.
+// accuracy. A bf16 operand is exact in TF32 (lo = 0) and drops its lo terms (two bf16 operands:
+// one term).
 //
 // Layouts: both MMA operands are K-major (32-bit K-major tiles with the 128-byte swizzle):
 // A split as [batch][M][K], B split *and transposed* as [batch][N][K] (the split kernel for B
 // writes B^T), so C = A B = A (B^T)^T. C [batch][M][N] row-major float32, overwritten. The
 // split operands are contiguous batches in the workspace, so one 3-D tensor map covers all
-// layers. CTA = one 128 x 128 tile of one batch entry; K in steps of 32 through a 3-stage
-// ring; warp 0 TMA, warp 1 lane 0 MMA (kind::tf32, K = 8 per instruction), warps 4..7
-// epilogue.
+// layers. Persistent CTAs (one per SM) walk 128 x 128 output tiles; K in steps of 32 through
+// a 3-stage ring; warp 0 TMA, warp 1 MMA (kind::tf32, K = 8 per instruction) into two TMEM
+// accumulators in turn, warps 4..7 epilogue.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -31,7 +32,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kOpBytes = kTile * kKStep * 4;    // 16 KB per operand part per stage
 constexpr int kStageBytes = 4 * kOpBytes;       // A_hi, A_lo, B_hi, B_lo
 constexpr int kBarOff = kStages * kStageBytes;
-constexpr int kSmem = kBarOff + 128;
+constexpr int kSmem = kBarOff + 256;   // barriers, TMEM slot and abort flag, then 8 doubles at +128
 
 __host__ __device__ constexpr uint32_t make_idesc_tf32(int M, int N, bool b_mn) {
     return (1u << 4)                    // D: f32
@@ -43,7 +44,7 @@ __host__ __device__ constexpr uint32_t make_idesc_tf32(int M, int N, bool b_mn) 
 
 struct Tf32Params {
     float *C;
-    int M, N, K;
+    int M, N, K, batch;
     int a_lo;           // A_lo present (absent: A is exact in TF32, e.g. bf16)
     int b_lo;           // B_lo present
     int a_tri;          // 0: A full; 1: A lower triangular (k < m0 + 128); 2: A upper triangular (k >= m0)
@@ -57,9 +58,36 @@ struct Tf32Params {
     int dot_x_bf16;
     double *dot_out, *dot_out2;
     int write_c;
+    // optional: C split for a later 3xTF32 product, hi = C rounded to TF32 and lo = C - hi,
+    // [batch][M][N] (split_t = 0) or transposed [batch][N][M] (split_t = 1)
+    float *split_hi, *split_lo;
+    int split_t;
     int *err_flag;
 };
 
+__device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u); }
+
+// Output tiles in the order the CTAs take them (t = blockIdx.x, + gridDim.x, ...): tile rows
+// outermost, the longest K ranges first when A is triangular, then batch entries, then columns.
+struct TileId {
+    int z, m, n;
+    bool skip;   // above the diagonal of a symmetric product
+};
+__device__ __forceinline__ TileId tile_of(int t, int gx, int gy, int batch, int a_tri, int sym) {
+    const int per_row = batch * gx;
+    const int mr = t / per_row, rem = t - mr * per_row;
+    TileId id;
+    id.z = rem / gx;
+    id.n = rem - id.z * gx;
+    id.m = a_tri == 1 ? gy - 1 - mr : mr;
+    id.skip = sym && id.n > id.m;
+    return id;
+}
+
+// Persistent: one CTA per SM walks its share of the output tiles. Warp 0 streams the operand
+// k-steps through the stage ring (running ahead into the next tile), warp 1 issues the MMAs
+// into one of two TMEM accumulators, warps 4..7 drain the other: the epilogue of a tile (its
+// dots, splits and stores) overlaps the MMAs of the next.
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constant__ CUtensorMap tAl,
                    const __grid_constant__ CUtensorMap tBh, const __grid_constant__ CUtensorMap tBl,
@@ -71,27 +99,17 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
     }
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + kBarOff);
     uint64_t *empty = full + kStages;
-    uint64_t *acc_bar = empty + kStages;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_bar + 1);
+    uint64_t *acc_full = empty + kStages;
+    uint64_t *acc_empty = acc_full + 2;
+    uint64_t *done_bar = acc_empty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    double *red = reinterpret_cast<double *>(smem + kBarOff + 128);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int n0 = blockIdx.x * kTile, m0 = blockIdx.y * kTile, z = blockIdx.z;
-    const size_t part_idx = (size_t)z * gridDim.x * gridDim.y + blockIdx.y * gridDim.x + blockIdx.x;
-    if (p.sym && n0 > m0) {
-        // the mirror tile (n0, m0) accounts for this one
-        if (threadIdx.x == 0) {
-            if (p.has_dot) p.dot_out[part_idx] = 0.0;
-            if (p.has_dot2) p.dot_out2[part_idx] = 0.0;
-        }
-        return;
-    }
-    // k-steps of this output row tile: a triangular A is zero outside [kt0, kt1), and skipping
-    // exact zeros changes no sum
+    const int gx = p.N / kTile, gy = p.M / kTile;
+    const int ntiles = gx * gy * p.batch;
     const int n_kall = (p.K + kKStep - 1) / kKStep;
-    const int kt0 = p.a_tri == 2 ? m0 / kKStep : 0;
-    const int kt1 = p.a_tri == 1 ? min(n_kall, (m0 + kTile) / kKStep) : n_kall;
-    const int n_k = kt1 - kt0;
     const uint32_t stage_tx = (2 + p.a_lo + p.b_lo) * kOpBytes;
 
     if (threadIdx.x == 0) {
@@ -99,12 +117,16 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
             ptx::mbar_init(&full[s], 1);
             ptx::mbar_init(&empty[s], 1);
         }
-        ptx::mbar_init(acc_bar, 1);
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&acc_full[b], 1);
+            ptx::mbar_init(&acc_empty[b], 4);
+        }
+        ptx::mbar_init(done_bar, 1);
         *abort_flag = 0;
         ptx::fence_barrier_init();
     }
     if (warp == 1) {
-        ptx::tmem_alloc(tmem_slot, 128);
+        ptx::tmem_alloc(tmem_slot, 256);
         ptx::tmem_relinquish();
     }
     ptx::tc_fence_before();
@@ -112,85 +134,143 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    // k-steps of a tile row: a triangular A is zero outside [kt0, kt1), and skipping exact zeros
+    // changes no sum
+    auto k_range = [&](int m0, int &kt0, int &n_k) {
+        kt0 = p.a_tri == 2 ? m0 / kKStep : 0;
+        const int kt1 = p.a_tri == 1 ? min(n_kall, (m0 + kTile) / kKStep) : n_kall;
+        n_k = kt1 - kt0;
+    };
+
     // producer and MMA warps stay converged; one elected lane issues (uniform registers)
     if (warp == 0) {
         const uint64_t pol = ptx::policy_evict_normal();
-        int issued = -1;
+        int it = 0;
         bool ok = true;
-        for (int kt = 0; kt < n_k; ++kt) {
-            const int s = kt % kStages;
-            ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&empty[s], ((kt / kStages) & 1) ^ 1, kWaitLimitNs,
-                                                                 p.err_flag, abort_flag));
-            if (!ok) break;
-            uint8_t *base = smem + s * kStageBytes;
-            ptx::mbar_arrive_expect_tx_warp(&full[s], stage_tx);
-            const int k0 = (kt0 + kt) * kKStep;
-            ptx::tma_load_3d_warp(base, &tAh, &full[s], k0, m0, z, pol);
-            if (p.a_lo) ptx::tma_load_3d_warp(base + kOpBytes, &tAl, &full[s], k0, m0, z, pol);
-            ptx::tma_load_3d_warp(base + 2 * kOpBytes, &tBh, &full[s], k0, n0, z, pol);
-            if (p.b_lo) ptx::tma_load_3d_warp(base + 3 * kOpBytes, &tBl, &full[s], k0, n0, z, pol);
-            issued = kt;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const TileId id = tile_of(t, gx, gy, p.batch, p.a_tri, p.sym);
+            if (id.skip) continue;
+            const int m0 = id.m * kTile, n0 = id.n * kTile;
+            int kt0, n_k;
+            k_range(m0, kt0, n_k);
+            for (int kt = 0; kt < n_k; ++kt, ++it) {
+                const int s = it % kStages;
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&empty[s], ((it / kStages) & 1) ^ 1, kWaitLimitNs,
+                                                                     p.err_flag, abort_flag));
+                if (!ok) break;
+                uint8_t *base = smem + s * kStageBytes;
+                ptx::mbar_arrive_expect_tx_warp(&full[s], stage_tx);
+                const int k0 = (kt0 + kt) * kKStep;
+                ptx::tma_load_3d_warp(base, &tAh, &full[s], k0, m0, id.z, pol);
+                if (p.a_lo) ptx::tma_load_3d_warp(base + kOpBytes, &tAl, &full[s], k0, m0, id.z, pol);
+                ptx::tma_load_3d_warp(base + 2 * kOpBytes, &tBh, &full[s], k0, n0, id.z, pol);
+                if (p.b_lo) ptx::tma_load_3d_warp(base + 3 * kOpBytes, &tBl, &full[s], k0, n0, id.z, pol);
+            }
         }
-        if (!ok)
-            for (int kt = issued - kStages + 1 > 0 ? issued - kStages + 1 : 0; kt <= issued; ++kt)
-                ptx::mbar_wait_bounded(&full[kt % kStages], (kt / kStages) & 1, kWaitLimitNs, nullptr, nullptr);
+        if (!ok) {
+            // let copies in flight land before the CTA can exit (bounded)
+            const uint64_t t0 = ptx::globaltimer_ns();
+            while (ptx::globaltimer_ns() - t0 < 2000000ull) {
+            }
+        }
     } else if (warp == 1) {
         constexpr uint32_t idesc = make_idesc_tf32(kTile, kTile, false);
         const uint32_t sbase = ptx::smem_u32(smem);
+        int it = 0, i = 0;
         bool ok = true;
-        for (int kt = 0; kt < n_k && ok; ++kt) {
-            const int s = kt % kStages;
-            ok = __all_sync(0xffffffffu,
-                            ptx::mbar_wait_bounded(&full[s], (kt / kStages) & 1, kWaitLimitNs, p.err_flag, abort_flag));
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const TileId id = tile_of(t, gx, gy, p.batch, p.a_tri, p.sym);
+            if (id.skip) continue;
+            int kt0, n_k;
+            k_range(id.m * kTile, kt0, n_k);
+            const int b = i & 1;
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&acc_empty[b], ((i >> 1) & 1) ^ 1, kWaitLimitNs,
+                                                                 p.err_flag, abort_flag));
             if (!ok) break;
             ptx::tc_fence_after();
-            const uint32_t ah = sbase + s * kStageBytes, al = ah + kOpBytes, bh = al + kOpBytes, bl = bh + kOpBytes;
+            const uint32_t d = tmem + (uint32_t)b * kTile;
+            for (int kt = 0; kt < n_k; ++kt, ++it) {
+                const int s = it % kStages;
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&full[s], (it / kStages) & 1, kWaitLimitNs,
+                                                                     p.err_flag, abort_flag));
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const uint32_t ah = sbase + s * kStageBytes, al = ah + kOpBytes, bh = al + kOpBytes, bl = bh + kOpBytes;
 #pragma unroll
-            for (int kk = 0; kk < kKStep / 8; ++kk) {
-                const uint64_t dah = ptx::make_sdesc_sw128(ah + kk * 32, 16, 1024);
-                const uint64_t dal = ptx::make_sdesc_sw128(al + kk * 32, 16, 1024);
-                const uint64_t dbh = ptx::make_sdesc_sw128(bh + kk * 32, 16, 1024);
-                uint32_t acc = (kt == 0 && kk == 0) ? 0u : 1u;
-                if (p.a_lo) {
-                    ptx::umma_tf32_ss_warp(tmem, dal, dbh, idesc, acc);
-                    acc = 1u;
+                for (int kk = 0; kk < kKStep / 8; ++kk) {
+                    const uint64_t dah = ptx::make_sdesc_sw128(ah + kk * 32, 16, 1024);
+                    const uint64_t dal = ptx::make_sdesc_sw128(al + kk * 32, 16, 1024);
+                    const uint64_t dbh = ptx::make_sdesc_sw128(bh + kk * 32, 16, 1024);
+                    uint32_t acc = (kt == 0 && kk == 0) ? 0u : 1u;
+                    if (p.a_lo) {
+                        ptx::umma_tf32_ss_warp(d, dal, dbh, idesc, acc);
+                        acc = 1u;
+                    }
+                    if (p.b_lo) {
+                        const uint64_t dbl = ptx::make_sdesc_sw128(bl + kk * 32, 16, 1024);
+                        ptx::umma_tf32_ss_warp(d, dah, dbl, idesc, acc);
+                        acc = 1u;
+                    }
+                    ptx::umma_tf32_ss_warp(d, dah, dbh, idesc, acc);
                 }
-                if (p.b_lo) {
-                    const uint64_t dbl = ptx::make_sdesc_sw128(bl + kk * 32, 16, 1024);
-                    ptx::umma_tf32_ss_warp(tmem, dah, dbl, idesc, acc);
-                    acc = 1u;
-                }
-                ptx::umma_tf32_ss_warp(tmem, dah, dbh, idesc, acc);
+                ptx::umma_commit_warp(&empty[s]);
             }
-            ptx::umma_commit_warp(&empty[s]);
+            if (!ok) break;
+            ptx::umma_commit_warp(&acc_full[b]);
+            ++i;
         }
         if (!ok) {
             if (lane == 0) *abort_flag = 1;
             __threadfence_block();
         }
-        ptx::umma_commit_warp(acc_bar);
-        ptx::mbar_wait_bounded(acc_bar, 0, kWaitLimitNs, p.err_flag, nullptr);
+        // every MMA issued has completed before tensor memory is released
+        ptx::umma_commit_warp(done_bar);
+        ptx::mbar_wait_bounded(done_bar, 0, kWaitLimitNs, p.err_flag, nullptr);
     } else if (warp >= 4) {
         const int wq = warp - 4;
         const int r = wq * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-        const bool ok = ptx::mbar_wait_bounded(acc_bar, 0, kWaitLimitNs, p.err_flag, abort_flag) && !*abort_flag;
-        // the mirror's share of a symmetric product's off-diagonal tile
-        const bool mirror = p.sym && m0 != n0;
-        double part = 0.0, part2 = 0.0;
-        if (ok) {
+        const bool has_parts = p.has_dot || p.has_dot2;
+        int i = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+            const TileId id = tile_of(t, gx, gy, p.batch, p.a_tri, p.sym);
+            const int z = id.z, m0 = id.m * kTile, n0 = id.n * kTile;
+            const size_t part_idx = ((size_t)z * gy + id.m) * gx + id.n;
+            if (id.skip) {
+                // the mirror tile (n0, m0) accounts for this one
+                if (wq == 0 && lane == 0) {
+                    if (p.has_dot) p.dot_out[part_idx] = 0.0;
+                    if (p.has_dot2) p.dot_out2[part_idx] = 0.0;
+                }
+                continue;
+            }
+            const int b = i & 1;
+            const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&acc_full[b], (i >> 1) & 1, kWaitLimitNs,
+                                                                           p.err_flag, abort_flag)) &&
+                            !*abort_flag;
+            if (!ok) break;
             ptx::tc_fence_after();
+            // the mirror's share of a symmetric product's off-diagonal tile
+            const bool mirror = p.sym && m0 != n0;
+            double part = 0.0, part2 = 0.0;
             const int gm = m0 + r;
             float *crow = p.C + ((size_t)z * p.M + gm) * p.N + n0;
             const size_t xrow = (size_t)gm * p.N + n0;
             const void *xz = p.has_dot ? p.dot_x.p[z] : nullptr;
             const float *x2z = p.has_dot2 ? static_cast<const float *>(p.dot_x2.p[z]) : nullptr;
+            const uint32_t tbuf = tmem + (uint32_t)b * kTile + lane_off;
 #pragma unroll 1
             for (int c = 0; c < kTile / 32; ++c) {
                 uint32_t v[32];
-                ptx::tmem_ld32(tmem + lane_off + c * 32, v);
+                ptx::tmem_ld32(tbuf + c * 32, v);
                 ptx::tmem_wait_ld();
-                if (p.has_dot && gm < p.M) {
+                if (c == kTile / 32 - 1) {
+                    // the accumulator is in registers: hand it back to the MMA warp
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&acc_empty[b]);
+                }
+                if (p.has_dot) {
                     // products of two floats are exact in double; summed in a fixed order. The row's
                     // 32 values are read as 16-byte vectors (N is a multiple of 128).
                     float x[32];
@@ -225,7 +305,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
                         for (int q = 0; q < 32; ++q) part += (double)__uint_as_float(v[q]) * (double)x[q];
                     }
                 }
-                if (p.has_dot2 && gm < p.M) {
+                if (p.has_dot2) {
                     float x[32];
                     const float4 *src = reinterpret_cast<const float4 *>(x2z + xrow + c * 32);
 #pragma unroll
@@ -243,44 +323,67 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
                         for (int q = 0; q < 32; ++q) part2 += (double)__uint_as_float(v[q]) * (double)x[q];
                     }
                 }
-                if (p.write_c && gm < p.M) {
+                if (p.split_hi) {
+                    if (p.split_t) {
+                        // column n0 + c*32 + q of C is row n of the transposed split: the warp's
+                        // 32 rows write one 128-byte run per q
+                        const size_t base = ((size_t)z * p.N + n0 + c * 32) * p.M + gm;
 #pragma unroll
-                    for (int q = 0; q < 32; q += 4) {
-                        if (n0 + c * 32 + q + 3 < p.N) {
-                            *reinterpret_cast<float4 *>(crow + c * 32 + q) =
-                                make_float4(__uint_as_float(v[q]), __uint_as_float(v[q + 1]), __uint_as_float(v[q + 2]),
-                                            __uint_as_float(v[q + 3]));
-                        } else {
-                            for (int u = 0; u < 4; ++u)
-                                if (n0 + c * 32 + q + u < p.N) crow[c * 32 + q + u] = __uint_as_float(v[q + u]);
+                        for (int q = 0; q < 32; ++q) {
+                            const float x = __uint_as_float(v[q]), h = tf32_hi(x);
+                            p.split_hi[base + (size_t)q * p.M] = h;
+                            p.split_lo[base + (size_t)q * p.M] = x - h;
+                        }
+                    } else {
+                        float *hrow = p.split_hi + ((size_t)z * p.M + gm) * p.N + n0 + c * 32;
+                        float *lrow = p.split_lo + ((size_t)z * p.M + gm) * p.N + n0 + c * 32;
+#pragma unroll
+                        for (int q = 0; q < 32; q += 4) {
+                            float h[4], l[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const float x = __uint_as_float(v[q + u]);
+                                h[u] = tf32_hi(x);
+                                l[u] = x - h[u];
+                            }
+                            *reinterpret_cast<float4 *>(hrow + q) = make_float4(h[0], h[1], h[2], h[3]);
+                            *reinterpret_cast<float4 *>(lrow + q) = make_float4(l[0], l[1], l[2], l[3]);
                         }
                     }
                 }
+                if (p.write_c) {
+#pragma unroll
+                    for (int q = 0; q < 32; q += 4)
+                        *reinterpret_cast<float4 *>(crow + c * 32 + q) =
+                            make_float4(__uint_as_float(v[q]), __uint_as_float(v[q + 1]), __uint_as_float(v[q + 2]),
+                                        __uint_as_float(v[q + 3]));
+                }
             }
-        }
-        if (p.has_dot || p.has_dot2) {
-            // the tile's partials: warp sums, then warp 4 adds the four warps' sums in order
-            for (int o = 16; o > 0; o >>= 1) {
-                part += __shfl_down_sync(0xffffffffu, part, o);
-                part2 += __shfl_down_sync(0xffffffffu, part2, o);
+            if (has_parts) {
+                // the tile's partials: warp sums, then warp 4 adds the four warps' sums in order
+                for (int o = 16; o > 0; o >>= 1) {
+                    part += __shfl_down_sync(0xffffffffu, part, o);
+                    part2 += __shfl_down_sync(0xffffffffu, part2, o);
+                }
+                if (lane == 0) {
+                    red[wq] = part;
+                    red[4 + wq] = part2;
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (wq == 0 && lane == 0) {
+                    if (p.has_dot) p.dot_out[part_idx] = ((red[0] + red[1]) + red[2]) + red[3];
+                    if (p.has_dot2) p.dot_out2[part_idx] = ((red[4] + red[5]) + red[6]) + red[7];
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");
             }
-            double *red = reinterpret_cast<double *>(smem + kBarOff + 64);
-            if (lane == 0) {
-                red[wq] = part;
-                red[4 + wq] = part2;
-            }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (wq == 0 && lane == 0) {
-                if (p.has_dot) p.dot_out[part_idx] = ok ? ((red[0] + red[1]) + red[2]) + red[3] : 0.0;
-                if (p.has_dot2) p.dot_out2[part_idx] = ok ? ((red[4] + red[5]) + red[6]) + red[7] : 0.0;
-            }
+            ++i;
         }
     }
     ptx::tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem, 128);
+        ptx::tmem_dealloc(tmem, 256);
     }
 }
 
@@ -384,7 +487,9 @@ cudaError_t launch_split_tf32(const PtrBatch &src, ElemType t, float *hi, float 
 //          dot_out[z][t] = sum over output tile t (m-tile major) of C_ij * X_z[i][j] in double,
 //          with sym also C_ij * X_z[j][i] off the diagonal (so the partials add up to
 //          sum_ij (A A^T)_ij X_ij);
-//   write_c: C is written (always, when no dot is asked for).
+//   split_hi / split_lo: C's TF32 split for a later product, [batch][M][N] or with split_t
+//          transposed [batch][N][M];
+//   write_c: C is written (always, when neither a dot nor a split is asked for).
 cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh, const float *Bl, float *C, int M,
                                int N, int K, int batch, int *err_flag, cudaStream_t s, const Tf32Opts &o) {
     if (M % kTile || N % kTile || K % kKStep || batch <= 0) return cudaErrorInvalidValue;
@@ -406,11 +511,23 @@ cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh
     p.dot_x_bf16 = o.dot_x_bf16 ? 1 : 0;
     p.dot_out = o.dot_out;
     p.dot_out2 = o.dot_out2;
-    p.write_c = (o.write_c || !(p.has_dot || p.has_dot2)) ? 1 : 0;
+    p.split_hi = o.split_hi;
+    p.split_lo = o.split_hi ? o.split_lo : nullptr;
+    p.split_t = o.split_t ? 1 : 0;
+    if (p.split_hi && !p.split_lo) return cudaErrorInvalidValue;
+    p.write_c = (o.write_c || !(p.has_dot || p.has_dot2 || p.split_hi)) ? 1 : 0;
     p.err_flag = err_flag;
+    p.batch = batch;
     cudaError_t e = cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
-    gemm_tf32x3_kernel<<<dim3(N / kTile, M / kTile, batch), kThreads, kSmem, s>>>(ah, al, bh, bl, p);
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const long long tiles = (long long)(M / kTile) * (N / kTile) * batch;
+    const int grid = (int)(tiles < sms ? tiles : sms);
+    gemm_tf32x3_kernel<<<grid, kThreads, kSmem, s>>>(ah, al, bh, bl, p);
     note_launch();
     return cudaGetLastError();
 }

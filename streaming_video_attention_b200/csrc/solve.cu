@@ -1,14 +1,16 @@
 // Absorb solve and reconstruction error, float32, batched over layers
 // [ISPA §3.1 step 2, §3.2, §3.3, §4.1 "Eq. 5"].
 //
+//   with D a multiple of 128:
+//   M = G + lambda I = L L^T, X = L^-1        one launch, a thread-block cluster per layer
+//                                             (chol_inv_sm100.cu)
+//   dW = X^T X (C W)                          Z = X (C W), dW = X^T Z on the tensor cores
+//                                             (3xTF32, the zero triangle of X skipped)
+//   otherwise:
 //   M = G + lambda I                          fill_shifted
 //   M = L L^T (blocked, right-looking)        potrf_diag + trsm_panel + GEMM trailing update
-//   dW = L^-T L^-1 (C W)                      with D a multiple of 128: X = L^-1 by blocked
-//                                             forward substitution on the identity (the
-//                                             updates skip X's zero upper part), then
-//                                             Z = X (C W) and dW = X^T Z on the tensor
-//                                             cores (3xTF32); otherwise trsv_block + GEMM
-//                                             per block, both ways, on (C W) itself
+//   dW = L^-T L^-1 (C W)                      trsv_block + GEMM per block, both ways, on
+//                                             (C W) itself
 //   five traces -> E^2, T^2, eps              tensor cores: the Gram products W W^T and
 //                                             dW dW^T (lower tiles only) dotted with G and H,
 //                                             and tr(W^T C W), tr(dW^T C W), in the GEMM
@@ -180,17 +182,20 @@ __global__ void __launch_bounds__(256) dot_partials_kernel(PtrBatch X, PtrBatch 
     }
 }
 
-// terms[k][z][p] for k = 0..4: tr(dW^T G dW), tr(dW^T C W), tr(W^T H W), tr(W^T G W), tr(W^T C W)
-__global__ void finalize_eps_kernel(const double *terms, int nparts, int batch, const int *status, float *eps,
-                                    double *err_terms) {
-    const int z = blockIdx.x * blockDim.x + threadIdx.x;
-    if (z >= batch) return;
-    double t[5];
-    for (int k = 0; k < 5; ++k) {
-        double s = 0.0;
-        for (int p = 0; p < nparts; ++p) s += terms[((size_t)k * batch + z) * nparts + p];
-        t[k] = s;
-    }
+// terms[k][z][p] for k = 0..4: tr(dW^T G dW), tr(dW^T C W), tr(W^T H W), tr(W^T G W), tr(W^T C W).
+// One CTA of five warps per layer: warp k sums term k's partials (lane-strided, then a fixed
+// shuffle tree), so the order of every sum is fixed.
+__global__ void __launch_bounds__(160) finalize_eps_kernel(const double *terms, int nparts, int batch,
+                                                            const int *status, float *eps, double *err_terms) {
+    __shared__ double t[5];
+    const int z = blockIdx.x, k = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const double *src = terms + ((size_t)k * batch + z) * nparts;
+    double s = 0.0;
+    for (int p = lane; p < nparts; p += 32) s += src[p];
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_down_sync(0xffffffffu, s, o);
+    if (lane == 0) t[k] = s;
+    __syncthreads();
+    if (threadIdx.x != 0) return;
     const double E2 = t[0] - 2.0 * t[1] + t[2];
     const double T2 = t[3] + 2.0 * t[4] + t[2];
     float e = T2 == 0.0 ? 0.f : (float)(E2 / T2);
@@ -210,14 +215,6 @@ __global__ void add_delta_kernel(PtrBatch W, PtrBatch dW, PtrBatch out, size_t n
     TW *oz = static_cast<TW *>(out.p[z]);
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
         oz[i] = from_f32<TW>(to_f32(Wz[i]) + dz[i]);
-}
-
-__global__ void fill_identity_kernel(PtrBatch dst, int D) {
-    const int z = blockIdx.y;
-    float *d = static_cast<float *>(dst.p[z]);
-    const size_t n = (size_t)D * D;
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
-        d[i] = (i / D == i % D) ? 1.f : 0.f;
 }
 
 __global__ void copy_f32_kernel(PtrBatch src, PtrBatch dst, size_t n) {
@@ -254,11 +251,12 @@ static GemmBatch make_gemm_batch(const PtrBatch &A, size_t offA, const PtrBatch 
 // On the tensor cores (tc) the quadratic forms are taken as dots with Gram matrices,
 // tr(X^T S X) = sum_ij S_ij (X X^T)_ij: one symmetric product W W^T (its lower tiles only)
 // dotted with G and H in its epilogue gives t3 and t2, dW dW^T dotted with G gives t0; t4 was
-// taken when Y was formed and t1 too when t1_done (the solve's last product).
+// taken when Y was formed and t1 too when t1_done (the solve's last product), which also left
+// dW's split in (dw_hi, dw_lo) (else null: split here).
 cudaError_t error_terms(const PtrBatch &G, const PtrBatch &H, const PtrBatch &W, ElemType wt, const PtrBatch &dW,
                         const PtrBatch &Y, const PtrBatch &P, float *Pc, float *split, double *terms, int nparts,
                         const int *status, float *eps, double *err_terms, int D, int batch, int *err_flag, bool tc,
-                        bool t1_done, cudaStream_t s) {
+                        bool t1_done, const float *dw_hi, const float *dw_lo, cudaStream_t s) {
     const size_t n = (size_t)D * D;
     const size_t ew = wt == ElemType::BF16 ? 2 : 4;
     const size_t bn = (size_t)batch * n;
@@ -277,13 +275,17 @@ cudaError_t error_terms(const PtrBatch &G, const PtrBatch &H, const PtrBatch &W,
         ow.write_c = false;
         ISPA_TRY(launch_gemm_tf32x3(Ahi, wbf ? nullptr : Alo, Ahi, wbf ? nullptr : Alo, Pc, D, D, D, batch, err_flag,
                                     s, ow));
-        // dW dW^T dotted with G -> t0
-        ISPA_TRY(launch_split_tf32(dW, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
+        // dW dW^T dotted with G -> t0 (dW split here unless its split is given)
+        if (!dw_hi) {
+            ISPA_TRY(launch_split_tf32(dW, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
+            dw_hi = Ahi;
+            dw_lo = Alo;
+        }
         Tf32Opts od;
         od.sym = true;
         od.dot_x = &G; od.dot_out = t_dgd;
         od.write_c = false;
-        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Ahi, Alo, Pc, D, D, D, batch, err_flag, s, od));
+        ISPA_TRY(launch_gemm_tf32x3(dw_hi, dw_lo, dw_hi, dw_lo, Pc, D, D, D, batch, err_flag, s, od));
         if (!t1_done) { dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(dW, Y, n, t_dy); note_launch(); }
     } else {
         GemmDesc full{D, D, D, D, D, D, true, false, ElemType::F32, ElemType::F32, ElemType::F32, 1.f, 0.f, false, batch};
@@ -306,13 +308,14 @@ cudaError_t error_terms(const PtrBatch &G, const PtrBatch &H, const PtrBatch &W,
         else { dot_partials_kernel<float><<<rgrid, 256, 0, s>>>(W, Y, n, t_wy); note_launch(); }
     }
     ISPA_TRY(cudaGetLastError());
-    finalize_eps_kernel<<<(batch + 63) / 64, 64, 0, s>>>(terms, nparts, batch, status, eps, err_terms); note_launch();
+    finalize_eps_kernel<<<batch, 160, 0, s>>>(terms, nparts, batch, status, eps, err_terms); note_launch();
     ISPA_TRY(cudaGetLastError());
 
     return cudaSuccess;
 }
 
-// Y = C W for one batch of layers (W split into Whi/Wlo first when tc).
+// Y = C W for one batch of layers (W split into Whi/Wlo first when tc; then Y^T's split is left
+// in the B_hi/B_lo blocks).
 static cudaError_t c_times_w(const PtrBatch &C, const PtrBatch &W, ElemType wt, const PtrBatch &Y, float *Yc,
                              float *split, double *t_wy, int D, int batch, int *err_flag, bool tc, cudaStream_t s) {
     const size_t n = (size_t)D * D;
@@ -323,9 +326,11 @@ static cudaError_t c_times_w(const PtrBatch &C, const PtrBatch &W, ElemType wt, 
     if (tc) {
         ISPA_TRY(launch_split_tf32(W, wt, Whi, Wlo, D, D, true, batch, s));
         ISPA_TRY(launch_split_tf32(C, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
-        // Y = C W, with t4 = tr(W^T Y) from the epilogue
+        // Y = C W, with t4 = tr(W^T Y) and Y's transposed split (the B operand of the solve's
+        // first product) from the epilogue
         Tf32Opts o;
         o.dot_x = &W; o.dot_x_bf16 = wt == ElemType::BF16; o.dot_out = t_wy;
+        o.split_hi = split + 2 * bn; o.split_lo = split + 3 * bn; o.split_t = true;
         ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Whi, Wlo, Yc, D, D, D, batch, err_flag, s, o));
     } else {
         GemmDesc d{D, D, D, D, D, D, true, false, ElemType::F32, wt, ElemType::F32, 1.f, 0.f, false, batch};
@@ -343,7 +348,7 @@ cudaError_t error_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
     const bool tc = (D % 128 == 0) && split != nullptr;
     ISPA_TRY(c_times_w(C, W, wt, Y, Yc, split, terms + 4 * (size_t)batch * nparts, D, batch, err_flag, tc, s));
     return error_terms(G, H, W, wt, dW, Y, P, Pc, split, terms, nparts, nullptr, eps, err_terms, D, batch, err_flag,
-                       tc, false, s);
+                       tc, false, nullptr, nullptr, s);
 }
 
 // Solve for one batch of layers. All pointers are device pointers, one per layer.
@@ -362,65 +367,51 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
     // operands live in `split`: A_hi, A_lo, B_hi, B_lo, W_hi, W_lo, each [batch][D][D].
     const bool tc = (D % 128 == 0) && split != nullptr;
 
-    // M = G + lambda I
-    fill_shifted_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(G, M, D, lambda); note_launch();
-    ISPA_TRY(cudaGetLastError());
-
     // Y = C W
     ISPA_TRY(c_times_w(C, W, wt, Y, Yc, split, terms + 4 * (size_t)batch * nparts, D, batch, err_flag, tc, s));
 
-    // Cholesky factorisation, blocked
     const int nblk = D / NB;
-    for (int kb = 0; kb < nblk; ++kb) {
-        const int k0 = kb * NB;
-        potrf_diag_kernel<<<batch, NB, 0, s>>>(M, D, k0, status); note_launch();
-        ISPA_TRY(cudaGetLastError());
-        const int rest = D - k0 - NB;
-        if (rest <= 0) break;
-        trsm_panel_kernel<<<dim3((rest + NB - 1) / NB, batch), NB, 0, s>>>(M, D, k0); note_launch();
-        ISPA_TRY(cudaGetLastError());
-        GemmDesc d{rest, rest, NB, D, D, D, true, true, ElemType::F32, ElemType::F32, ElemType::F32, -1.f, 1.f,
-                   true, batch};
-        const size_t offA = (size_t)(k0 + NB) * D + k0;
-        const size_t offC = (size_t)(k0 + NB) * D + k0 + NB;
-        ISPA_TRY(launch_gemm_simt(d, make_gemm_batch(M, offA, M, offA, M, offC, batch, 4, 4), s));
-    }
-
     if (tc) {
-        // X = L^-1 in P: forward substitution L X = I. Block row k of X is nonzero only in its
-        // first k0 + NB columns, so the diagonal solve and the update below stop there.
-        fill_identity_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(P, D); note_launch();
-        ISPA_TRY(cudaGetLastError());
-        for (int kb = 0; kb < nblk; ++kb) {
-            const int k0 = kb * NB;
-            const int cols = k0 + NB;
-            trsv_block_kernel<false><<<dim3((cols + 127) / 128, batch), 128, 0, s>>>(M, P, D, k0); note_launch();
-            ISPA_TRY(cudaGetLastError());
-            const int rest = D - k0 - NB;
-            if (rest <= 0) break;
-            GemmDesc d{rest, cols, NB, D, D, D, true, false, ElemType::F32, ElemType::F32, ElemType::F32, -1.f, 1.f,
-                       false, batch};
-            ISPA_TRY(launch_gemm_simt(
-                d, make_gemm_batch(M, (size_t)(k0 + NB) * D + k0, P, (size_t)k0 * D, P, (size_t)(k0 + NB) * D, batch, 4, 4),
-                s));
-        }
-        // Z = X Y into dW, then dW = X^T Z (3xTF32; B operands are split transposed)
+        // M = G + lambda I = L L^T and X = L^-1 (in P) in one launch: a cluster of CTAs per layer
+        ISPA_TRY(launch_chol_inv(G, M, P, D, lambda, batch, status, s));
+        // Z = X Y, then dW = X^T Z (3xTF32; B operands are split transposed). Y^T's split is in the
+        // B blocks (from Y's epilogue); Z leaves only its transposed split (in the W blocks, free
+        // after Y), dW its own split (in the B blocks) for the error's dW dW^T.
         const size_t bn = (size_t)batch * n;
         float *Ahi = split, *Alo = split + bn, *Bhi = split + 2 * bn, *Blo = split + 3 * bn;
+        float *Zhi = split + 4 * bn, *Zlo = split + 5 * bn;
         float *dWc = static_cast<float *>(dW.p[0]);
         ISPA_TRY(launch_split_tf32(P, ElemType::F32, Ahi, Alo, D, D, false, batch, s));
-        ISPA_TRY(launch_split_tf32(Y, ElemType::F32, Bhi, Blo, D, D, true, batch, s));
         Tf32Opts oz;
         oz.a_tri = 1;   // X lower
+        oz.split_hi = Zhi; oz.split_lo = Zlo; oz.split_t = true;
+        oz.write_c = false;
         ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Bhi, Blo, dWc, D, D, D, batch, err_flag, s, oz));
         ISPA_TRY(launch_split_tf32(P, ElemType::F32, Ahi, Alo, D, D, true, batch, s));
-        ISPA_TRY(launch_split_tf32(dW, ElemType::F32, Bhi, Blo, D, D, true, batch, s));
         // X^T upper; t1 = tr(dW^T Y) from the epilogue
         Tf32Opts od;
         od.a_tri = 2;
         od.dot_x = &Y; od.dot_out = terms + (size_t)batch * nparts;
-        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Bhi, Blo, dWc, D, D, D, batch, err_flag, s, od));
+        od.split_hi = Bhi; od.split_lo = Blo;
+        ISPA_TRY(launch_gemm_tf32x3(Ahi, Alo, Zhi, Zlo, dWc, D, D, D, batch, err_flag, s, od));
     } else {
+        // M = G + lambda I, then the blocked Cholesky factorisation
+        fill_shifted_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(G, M, D, lambda); note_launch();
+        ISPA_TRY(cudaGetLastError());
+        for (int kb = 0; kb < nblk; ++kb) {
+            const int k0 = kb * NB;
+            potrf_diag_kernel<<<batch, NB, 0, s>>>(M, D, k0, status); note_launch();
+            ISPA_TRY(cudaGetLastError());
+            const int rest = D - k0 - NB;
+            if (rest <= 0) break;
+            trsm_panel_kernel<<<dim3((rest + NB - 1) / NB, batch), NB, 0, s>>>(M, D, k0); note_launch();
+            ISPA_TRY(cudaGetLastError());
+            GemmDesc d{rest, rest, NB, D, D, D, true, true, ElemType::F32, ElemType::F32, ElemType::F32, -1.f, 1.f,
+                       true, batch};
+            const size_t offA = (size_t)(k0 + NB) * D + k0;
+            const size_t offC = (size_t)(k0 + NB) * D + k0 + NB;
+            ISPA_TRY(launch_gemm_simt(d, make_gemm_batch(M, offA, M, offA, M, offC, batch, 4, 4), s));
+        }
         // dW <- Y, solved in place: forward substitution L Z = Y, then backward L^T X = Z
         copy_f32_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(Y, dW, n); note_launch();
         ISPA_TRY(cudaGetLastError());
@@ -450,8 +441,11 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
     }
 
     // Reconstruction error terms
-    ISPA_TRY(error_terms(G, H, W, wt, dW, Y, P, Pc, split, terms, nparts, status, eps, err_terms, D, batch, err_flag,
-                         tc, tc, s));
+    {
+        const size_t bn = (size_t)batch * n;
+        ISPA_TRY(error_terms(G, H, W, wt, dW, Y, P, Pc, split, terms, nparts, status, eps, err_terms, D, batch, err_flag,
+                             tc, tc, tc ? split + 2 * bn : nullptr, tc ? split + 3 * bn : nullptr, s));
+    }
 
     if (w_new) {
         if (wt == ElemType::BF16) { add_delta_kernel<bf16><<<dim3(fill_blocks, batch), 256, 0, s>>>(W, dW, *w_new, n); note_launch(); }
