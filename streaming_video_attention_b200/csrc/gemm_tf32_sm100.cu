@@ -67,18 +67,20 @@ struct Tf32Params {
 
 __device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u); }
 
-// Output tiles in the order the CTAs take them (t = blockIdx.x, + gridDim.x, ...): tile rows
-// outermost, the longest K ranges first when A is triangular, then batch entries, then columns.
+// Output tiles in the order the CTAs take them (t = blockIdx.x, + gridDim.x, ...): batch entries
+// outermost, so that the tiles in flight at once share one layer's operands in L2; within a
+// layer tile rows with the longest K range first when A is triangular, then columns.
 struct TileId {
     int z, m, n;
     bool skip;   // above the diagonal of a symmetric product
 };
-__device__ __forceinline__ TileId tile_of(int t, int gx, int gy, int batch, int a_tri, int sym) {
-    const int per_row = batch * gx;
-    const int mr = t / per_row, rem = t - mr * per_row;
+__device__ __forceinline__ TileId tile_of(int t, int gx, int gy, int a_tri, int sym) {
+    const int per_layer = gx * gy;
     TileId id;
-    id.z = rem / gx;
-    id.n = rem - id.z * gx;
+    id.z = t / per_layer;
+    const int rem = t - id.z * per_layer;
+    const int mr = rem / gx;
+    id.n = rem - mr * gx;
     id.m = a_tri == 1 ? gy - 1 - mr : mr;
     id.skip = sym && id.n > id.m;
     return id;
@@ -148,7 +150,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
         int it = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-            const TileId id = tile_of(t, gx, gy, p.batch, p.a_tri, p.sym);
+            const TileId id = tile_of(t, gx, gy, p.a_tri, p.sym);
             if (id.skip) continue;
             const int m0 = id.m * kTile, n0 = id.n * kTile;
             int kt0, n_k;
@@ -179,7 +181,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
         int it = 0, i = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-            const TileId id = tile_of(t, gx, gy, p.batch, p.a_tri, p.sym);
+            const TileId id = tile_of(t, gx, gy, p.a_tri, p.sym);
             if (id.skip) continue;
             int kt0, n_k;
             k_range(id.m * kTile, kt0, n_k);
@@ -233,7 +235,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
         const bool has_parts = p.has_dot || p.has_dot2;
         int i = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-            const TileId id = tile_of(t, gx, gy, p.batch, p.a_tri, p.sym);
+            const TileId id = tile_of(t, gx, gy, p.a_tri, p.sym);
             const int z = id.z, m0 = id.m * kTile, n0 = id.n * kTile;
             const size_t part_idx = ((size_t)z * gy + id.m) * gx + id.n;
             if (id.skip) {
