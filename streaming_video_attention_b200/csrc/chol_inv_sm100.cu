@@ -245,33 +245,39 @@ __device__ __noinline__ bool factor_invert_diag(const float *Mz, int D, int k, f
     return bad;
 }
 
+// FILL_M: M = G + lambda I first (the whole matrix, n = ld); otherwise M already holds the n x n
+// block to factor (row stride ld). P (the same block of the inverse) is set to I either way.
+template <bool FILL_M>
 __global__ void __cluster_dims__(kCL, 1, 1) __launch_bounds__(kThreads, 2)
-chol_inv_cluster_kernel(PtrBatch G, PtrBatch M, PtrBatch P, int D, float lambda, int *status) {
+chol_inv_cluster_kernel(PtrBatch G, PtrBatch M, PtrBatch P, int n, int ld, float lambda, int *status) {
     extern __shared__ __align__(16) float sm[];
     float *Ts = sm + kOffT, *Lf = sm + kOffLf, *buf0 = sm + kOffBuf, *inv = sm + kOffInv;
     float *col = inv + kNB;   // [2][64]
     const int rank = (int)blockIdx.x;   // cluster of kCL along x: blockIdx.x is the rank
     const int z = blockIdx.y;
-    const float *Gz = static_cast<const float *>(G.p[z]);
     float *Mz = static_cast<float *>(M.p[z]);
     float *Pz = static_cast<float *>(P.p[z]);
-    const int nb = D / kNB;
+    const int nb = n / kNB;
+    const int D = ld;   // row stride of M and P
     const int tid = threadIdx.x;
 
-    // M = G + lambda I, P = I: each CTA writes its share of rows
+    // (M = G + lambda I,) P = I: each CTA writes its share of rows
     {
-        const int r0 = (int)((long long)D * rank / kCL), r1 = (int)((long long)D * (rank + 1) / kCL);
-        const int q = D / 4;
+        const int r0 = (int)((long long)n * rank / kCL), r1 = (int)((long long)n * (rank + 1) / kCL);
+        const int q = n / 4;
         for (long long idx = tid; idx < (long long)(r1 - r0) * q; idx += kThreads) {
             const int r = r0 + (int)(idx / q), c4 = (int)(idx % q) * 4;
-            float4 g = *reinterpret_cast<const float4 *>(Gz + (size_t)r * D + c4);
             const int d = r - c4;
             const float4 e = make_float4(d == 0 ? 1.f : 0.f, d == 1 ? 1.f : 0.f, d == 2 ? 1.f : 0.f, d == 3 ? 1.f : 0.f);
-            g.x += d == 0 ? lambda : 0.f;
-            g.y += d == 1 ? lambda : 0.f;
-            g.z += d == 2 ? lambda : 0.f;
-            g.w += d == 3 ? lambda : 0.f;
-            __stcg(reinterpret_cast<float4 *>(Mz + (size_t)r * D + c4), g);
+            if (FILL_M) {
+                const float *Gz = static_cast<const float *>(G.p[z]);
+                float4 g = *reinterpret_cast<const float4 *>(Gz + (size_t)r * D + c4);
+                g.x += d == 0 ? lambda : 0.f;
+                g.y += d == 1 ? lambda : 0.f;
+                g.z += d == 2 ? lambda : 0.f;
+                g.w += d == 3 ? lambda : 0.f;
+                __stcg(reinterpret_cast<float4 *>(Mz + (size_t)r * D + c4), g);
+            }
             __stcg(reinterpret_cast<float4 *>(Pz + (size_t)r * D + c4), e);
         }
     }
@@ -310,9 +316,23 @@ chol_inv_cluster_kernel(PtrBatch G, PtrBatch M, PtrBatch P, int D, float lambda,
 cudaError_t launch_chol_inv(const PtrBatch &G, const PtrBatch &M, const PtrBatch &P, int D, float lambda, int batch,
                             int *status, cudaStream_t s) {
     if (D % kNB || batch <= 0 || batch > kMaxBatch) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(chol_inv_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e =
+        cudaFuncSetAttribute(chol_inv_cluster_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    chol_inv_cluster_kernel<<<dim3(kCL, batch), kThreads, kSmemBytes, s>>>(G, M, P, D, lambda, status);
+    chol_inv_cluster_kernel<true><<<dim3(kCL, batch), kThreads, kSmemBytes, s>>>(G, M, P, D, D, lambda, status);
+    note_launch();
+    return cudaGetLastError();
+}
+
+// The same for an n x n diagonal block already in M (pointers at the block, row stride ld):
+// its L^-1 into the matching block of P (M's block is overwritten as scratch).
+cudaError_t launch_chol_inv_block(const PtrBatch &M, const PtrBatch &P, int n, int ld, int batch, int *status,
+                                  cudaStream_t s) {
+    if (n % kNB || ld % 4 || n > ld || batch <= 0 || batch > kMaxBatch) return cudaErrorInvalidValue;
+    cudaError_t e =
+        cudaFuncSetAttribute(chol_inv_cluster_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    chol_inv_cluster_kernel<false><<<dim3(kCL, batch), kThreads, kSmemBytes, s>>>(M, M, P, n, ld, 0.f, status);
     note_launch();
     return cudaGetLastError();
 }

@@ -116,10 +116,15 @@ struct PtrBatch {
 // (chol_inv_sm100.cu); status[z] = ISPA_ERR_NOT_SPD on a non-positive pivot.
 cudaError_t launch_chol_inv(const PtrBatch &G, const PtrBatch &M, const PtrBatch &P, int D, float lambda, int batch,
                             int *status, cudaStream_t s);
+// The same for an n x n diagonal block already in M (pointers at the block, row stride ld): its
+// L^-1 into the matching block of P.
+cudaError_t launch_chol_inv_block(const PtrBatch &M, const PtrBatch &P, int n, int ld, int batch, int *status,
+                                  cudaStream_t s);
 
 // 3xTF32 tensor-core GEMM for D x D products (gemm_tf32_sm100.cu).
+// Source row stride ld (0: cols); destination entries dst_bstride elements apart (0: rows*cols).
 cudaError_t launch_split_tf32(const PtrBatch &src, ElemType t, float *hi, float *lo, int rows, int cols,
-                              bool transpose, int batch, cudaStream_t s);
+                              bool transpose, int batch, cudaStream_t s, size_t ld = 0, size_t dst_bstride = 0);
 struct Tf32Opts {
     int a_tri = 0;                      // 1: A lower triangular, 2: A upper triangular (M = K)
     bool sym = false;                   // B is A: only output tiles on and below the diagonal
@@ -131,6 +136,9 @@ struct Tf32Opts {
     float *split_hi = nullptr;          // C's TF32 split (hi, lo), [batch][M][N] or transposed
     float *split_lo = nullptr;
     bool split_t = false;
+    size_t split_bstride = 0;           // 0: M*N
+    size_t ldc = 0, c_bstride = 0;      // C's row and batch strides (0: N, M*N)
+    bool c_sub = false;                 // C = C - A B
     bool write_c = true;
 };
 cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh, const float *Bl, float *C, int M,

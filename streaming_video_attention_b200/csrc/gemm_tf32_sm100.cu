@@ -62,6 +62,10 @@ struct Tf32Params {
     // [batch][M][N] (split_t = 0) or transposed [batch][N][M] (split_t = 1)
     float *split_hi, *split_lo;
     int split_t;
+    size_t split_bstride;   // batch stride of the split (elements)
+    // C row z, i, column j at C[z * c_bstride + i * ldc + j]; c_sub: C = C - A B
+    size_t ldc, c_bstride;
+    int c_sub;
     int *err_flag;
 };
 
@@ -256,7 +260,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
             const bool mirror = p.sym && m0 != n0;
             double part = 0.0, part2 = 0.0;
             const int gm = m0 + r;
-            float *crow = p.C + ((size_t)z * p.M + gm) * p.N + n0;
+            float *crow = p.C + (size_t)z * p.c_bstride + (size_t)gm * p.ldc + n0;
             const size_t xrow = (size_t)gm * p.N + n0;
             const void *xz = p.has_dot ? p.dot_x.p[z] : nullptr;
             const float *x2z = p.has_dot2 ? static_cast<const float *>(p.dot_x2.p[z]) : nullptr;
@@ -329,7 +333,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
                     if (p.split_t) {
                         // column n0 + c*32 + q of C is row n of the transposed split: the warp's
                         // 32 rows write one 128-byte run per q
-                        const size_t base = ((size_t)z * p.N + n0 + c * 32) * p.M + gm;
+                        const size_t base = (size_t)z * p.split_bstride + (size_t)(n0 + c * 32) * p.M + gm;
 #pragma unroll
                         for (int q = 0; q < 32; ++q) {
                             const float x = __uint_as_float(v[q]), h = tf32_hi(x);
@@ -337,8 +341,8 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
                             p.split_lo[base + (size_t)q * p.M] = x - h;
                         }
                     } else {
-                        float *hrow = p.split_hi + ((size_t)z * p.M + gm) * p.N + n0 + c * 32;
-                        float *lrow = p.split_lo + ((size_t)z * p.M + gm) * p.N + n0 + c * 32;
+                        float *hrow = p.split_hi + (size_t)z * p.split_bstride + (size_t)gm * p.N + n0 + c * 32;
+                        float *lrow = p.split_lo + (size_t)z * p.split_bstride + (size_t)gm * p.N + n0 + c * 32;
 #pragma unroll
                         for (int q = 0; q < 32; q += 4) {
                             float h[4], l[4];
@@ -354,11 +358,23 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
                     }
                 }
                 if (p.write_c) {
+                    if (p.c_sub) {
+                        float4 old[8];
 #pragma unroll
-                    for (int q = 0; q < 32; q += 4)
-                        *reinterpret_cast<float4 *>(crow + c * 32 + q) =
-                            make_float4(__uint_as_float(v[q]), __uint_as_float(v[q + 1]), __uint_as_float(v[q + 2]),
-                                        __uint_as_float(v[q + 3]));
+                        for (int u = 0; u < 8; ++u) old[u] = *reinterpret_cast<const float4 *>(crow + c * 32 + 4 * u);
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            *reinterpret_cast<float4 *>(crow + c * 32 + 4 * u) =
+                                make_float4(old[u].x - __uint_as_float(v[4 * u]), old[u].y - __uint_as_float(v[4 * u + 1]),
+                                            old[u].z - __uint_as_float(v[4 * u + 2]),
+                                            old[u].w - __uint_as_float(v[4 * u + 3]));
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 32; q += 4)
+                            *reinterpret_cast<float4 *>(crow + c * 32 + q) =
+                                make_float4(__uint_as_float(v[q]), __uint_as_float(v[q + 1]), __uint_as_float(v[q + 2]),
+                                            __uint_as_float(v[q + 3]));
+                    }
                 }
             }
             if (has_parts) {
@@ -390,42 +406,48 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
 }
 
 // X_hi = X rounded to TF32 (round to nearest, ties away from zero on the 13 dropped bits),
-// X_lo = X - X_hi, for a batch of float32 or bf16 matrices of n elements, written to
-// contiguous [batch][n] arrays. bf16 inputs are exact in TF32: lo is not written.
+// X_lo = X - X_hi, for a batch of float32 or bf16 [rows][cols] matrices with row stride ld,
+// written to [rows][cols] arrays dst_bstride elements apart. bf16 inputs are exact in TF32: lo
+// is not written.
+__device__ __forceinline__ float tf32_round(float x) { return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u); }
+
 template <typename T>
-__global__ void split_tf32_kernel(PtrBatch src, float *hi, float *lo, size_t n) {
+__global__ void split_tf32_kernel(PtrBatch src, float *hi, float *lo, int rows, int cols, size_t ld,
+                                  size_t dst_bstride) {
     const int z = blockIdx.y;
     const T *s = static_cast<const T *>(src.p[z]);
-    float *h = hi + (size_t)z * n;
-    float *l = lo ? lo + (size_t)z * n : nullptr;
+    float *h = hi + (size_t)z * dst_bstride;
+    float *l = lo ? lo + (size_t)z * dst_bstride : nullptr;
+    const size_t n = (size_t)rows * cols;
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
-        const float x = to_f32(s[i]);
-        const float xh = __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
+        const size_t si = ld == (size_t)cols ? i : (i / cols) * ld + i % cols;
+        const float x = to_f32(s[si]);
+        const float xh = tf32_round(x);
         h[i] = xh;
         if (l) l[i] = x - xh;
     }
 }
 
-// The same split of a batch of row-major [rows][cols] matrices, written transposed
+// The same split of a batch of [rows][cols] matrices (row stride ld), written transposed
 // ([cols][rows]) through a 32 x 32 shared-memory tile so that reads and writes stay coalesced.
 template <typename T>
-__global__ void split_tf32_transposed_kernel(PtrBatch src, float *hi, float *lo, int rows, int cols) {
+__global__ void split_tf32_transposed_kernel(PtrBatch src, float *hi, float *lo, int rows, int cols, size_t ld,
+                                             size_t dst_bstride) {
     __shared__ float tile[32][33];
     const int z = blockIdx.z;
     const T *s = static_cast<const T *>(src.p[z]);
-    const size_t n = (size_t)rows * cols;
     const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
     for (int i = threadIdx.y; i < 32; i += blockDim.y) {
         const int r = r0 + i, c = c0 + threadIdx.x;
-        tile[i][threadIdx.x] = (r < rows && c < cols) ? to_f32(s[(size_t)r * cols + c]) : 0.f;
+        tile[i][threadIdx.x] = (r < rows && c < cols) ? to_f32(s[(size_t)r * ld + c]) : 0.f;
     }
     __syncthreads();
     for (int i = threadIdx.y; i < 32; i += blockDim.y) {
         const int c = c0 + i, r = r0 + threadIdx.x;
         if (r < rows && c < cols) {
             const float x = tile[threadIdx.x][i];
-            const float xh = __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
-            const size_t o = (size_t)z * n + (size_t)c * rows + r;
+            const float xh = tf32_round(x);
+            const size_t o = (size_t)z * dst_bstride + (size_t)c * rows + r;
             hi[o] = xh;
             if (lo) lo[o] = x - xh;
         }
@@ -464,16 +486,21 @@ bool make_map(CUtensorMap *m, const float *ptr, int batch, int rows, int cols, i
 }  // namespace
 
 cudaError_t launch_split_tf32(const PtrBatch &src, ElemType t, float *hi, float *lo, int rows, int cols,
-                              bool transpose, int batch, cudaStream_t s) {
+                              bool transpose, int batch, cudaStream_t s, size_t ld, size_t dst_bstride) {
+    if (rows <= 0 || cols <= 0 || batch <= 0) return cudaSuccess;
+    if (!ld) ld = cols;
+    if (!dst_bstride) dst_bstride = (size_t)rows * cols;
     if (transpose) {
         const dim3 grid((cols + 31) / 32, (rows + 31) / 32, batch), block(32, 8);
-        if (t == ElemType::BF16) split_tf32_transposed_kernel<bf16><<<grid, block, 0, s>>>(src, hi, nullptr, rows, cols);
-        else split_tf32_transposed_kernel<float><<<grid, block, 0, s>>>(src, hi, lo, rows, cols);
+        if (t == ElemType::BF16)
+            split_tf32_transposed_kernel<bf16><<<grid, block, 0, s>>>(src, hi, nullptr, rows, cols, ld, dst_bstride);
+        else split_tf32_transposed_kernel<float><<<grid, block, 0, s>>>(src, hi, lo, rows, cols, ld, dst_bstride);
     } else {
         const size_t n = (size_t)rows * cols;
         const int blocks = (int)std::min<size_t>((n + 255) / 256, 1024);
-        if (t == ElemType::BF16) split_tf32_kernel<bf16><<<dim3(blocks, batch), 256, 0, s>>>(src, hi, nullptr, n);
-        else split_tf32_kernel<float><<<dim3(blocks, batch), 256, 0, s>>>(src, hi, lo, n);
+        if (t == ElemType::BF16)
+            split_tf32_kernel<bf16><<<dim3(blocks, batch), 256, 0, s>>>(src, hi, nullptr, rows, cols, ld, dst_bstride);
+        else split_tf32_kernel<float><<<dim3(blocks, batch), 256, 0, s>>>(src, hi, lo, rows, cols, ld, dst_bstride);
     }
     note_launch();
     return cudaGetLastError();
@@ -490,7 +517,9 @@ cudaError_t launch_split_tf32(const PtrBatch &src, ElemType t, float *hi, float 
 //          with sym also C_ij * X_z[j][i] off the diagonal (so the partials add up to
 //          sum_ij (A A^T)_ij X_ij);
 //   split_hi / split_lo: C's TF32 split for a later product, [batch][M][N] or with split_t
-//          transposed [batch][N][M];
+//          transposed [batch][N][M], split_bstride elements per batch entry (0: M*N);
+//   ldc, c_bstride (0: N, M*N): C's row and batch strides (a block of a larger matrix);
+//   c_sub: C = C - A B (the old C read in the epilogue);
 //   write_c: C is written (always, when neither a dot nor a split is asked for).
 cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh, const float *Bl, float *C, int M,
                                int N, int K, int batch, int *err_flag, cudaStream_t s, const Tf32Opts &o) {
@@ -516,6 +545,11 @@ cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh
     p.split_hi = o.split_hi;
     p.split_lo = o.split_hi ? o.split_lo : nullptr;
     p.split_t = o.split_t ? 1 : 0;
+    p.split_bstride = o.split_bstride ? o.split_bstride : (size_t)M * N;
+    p.ldc = o.ldc ? o.ldc : (size_t)N;
+    p.c_bstride = o.c_bstride ? o.c_bstride : (size_t)M * N;
+    p.c_sub = o.c_sub ? 1 : 0;
+    if (p.ldc % 4 || p.c_bstride % 4) return cudaErrorInvalidValue;
     if (p.split_hi && !p.split_lo) return cudaErrorInvalidValue;
     p.write_c = (o.write_c || !(p.has_dot || p.has_dot2 || p.split_hi)) ? 1 : 0;
     p.err_flag = err_flag;

@@ -351,6 +351,80 @@ cudaError_t error_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
                        tc, false, nullptr, nullptr, s);
 }
 
+// M = G + lambda I = L L^T and X = L^-1 into P, blocked by nb2 columns (256, or 128 below
+// D = 1024): per block step k the cluster kernel factors and inverts the diagonal block (its
+// inverse T_k is X's diagonal block), and the tensor cores (3xTF32) take the rest --
+//   L_ik = A_ik T_k^T                    (the panel below, written to M with its split)
+//   A_ij -= L_ik L_jk^T                  (the trailing update, lower tiles)
+//   X_kc = T_k B_kc        (c < k)       (block row k of X from its accumulated right-hand side)
+//   B_ic -= L_ik X_kc      (i > k, c <= k)
+// with B = I at the start (P zeroed, the diagonal blocks set by the cluster kernel). Scratch: the
+// split blocks 0, 1 (panel splits) and 4, 5 (T_k, B_k^T, X_k^T splits); blocks 2, 3 hold Y^T's
+// split for the solve and are not touched. M and P hold `batch` contiguous D x D matrices.
+static cudaError_t chol_inv_blocked(const PtrBatch &G, const PtrBatch &M, const PtrBatch &P, float *split, int D,
+                                    float lambda, int batch, int *status, int *err_flag, int fill_blocks,
+                                    cudaStream_t s) {
+    const int nb2 = (D % 256 == 0 && D >= 1024) ? 256 : 128;
+    const int nblk = D / nb2;
+    if (nblk == 1) return launch_chol_inv(G, M, P, D, lambda, batch, status, s);
+    const size_t n = (size_t)D * D, bn = (size_t)batch * n;
+    float *Mc = static_cast<float *>(M.p[0]), *Pc = static_cast<float *>(P.p[0]);
+    // panel splits (block 0-1): A_ik then L_ik, each [batch][D - nb2][nb2]
+    const size_t pan = (size_t)(D - nb2) * nb2;
+    float *Ap_hi = split, *Ap_lo = Ap_hi + batch * pan, *Lp_hi = Ap_lo + batch * pan, *Lp_lo = Lp_hi + batch * pan;
+    // blocks 4-5: T_k [batch][nb2][nb2], B_k^T [batch][D - nb2][nb2], X_k^T [batch][D][nb2]
+    float *r45 = split + 4 * bn;
+    const size_t tsz = (size_t)nb2 * nb2, xsz = (size_t)D * nb2;
+    float *T_hi = r45, *T_lo = T_hi + batch * tsz, *Bt_hi = T_lo + batch * tsz, *Bt_lo = Bt_hi + batch * pan,
+          *Xt_hi = Bt_lo + batch * pan, *Xt_lo = Xt_hi + batch * xsz;
+
+    fill_shifted_kernel<<<dim3(fill_blocks, batch), 256, 0, s>>>(G, M, D, lambda); note_launch();
+    ISPA_TRY(cudaGetLastError());
+    ISPA_TRY(cudaMemsetAsync(Pc, 0, bn * sizeof(float), s));
+    auto at = [&](const PtrBatch &X, size_t off) {
+        PtrBatch o;
+        for (int z = 0; z < batch; ++z) o.p[z] = static_cast<float *>(X.p[z]) + off;
+        return o;
+    };
+    for (int k = 0; k < nblk; ++k) {
+        const int r0 = k * nb2, rest = D - r0 - nb2;
+        const size_t dk = (size_t)r0 * D + r0;
+        ISPA_TRY(launch_chol_inv_block(at(M, dk), at(P, dk), nb2, D, batch, status, s));
+        ISPA_TRY(launch_split_tf32(at(P, dk), ElemType::F32, T_hi, T_lo, nb2, nb2, false, batch, s, D));
+        if (rest > 0) {
+            const size_t below = (size_t)(r0 + nb2) * D + r0;
+            ISPA_TRY(launch_split_tf32(at(M, below), ElemType::F32, Ap_hi, Ap_lo, rest, nb2, false, batch, s, D));
+            Tf32Opts op;   // L_ik = A_ik T_k^T into M, and its split
+            op.ldc = D; op.c_bstride = n;
+            op.split_hi = Lp_hi; op.split_lo = Lp_lo;
+            ISPA_TRY(launch_gemm_tf32x3(Ap_hi, Ap_lo, T_hi, T_lo, Mc + below, rest, nb2, nb2, batch, err_flag, s, op));
+            Tf32Opts ou;   // A_ij -= L_ik L_jk^T, lower tiles
+            ou.sym = true; ou.c_sub = true; ou.ldc = D; ou.c_bstride = n;
+            ISPA_TRY(launch_gemm_tf32x3(Lp_hi, Lp_lo, Lp_hi, Lp_lo, Mc + below + nb2, rest, rest, nb2, batch, err_flag,
+                                        s, ou));
+        }
+        // X_k^T's split holds r0 + nb2 rows per layer: X_kc^T (c < k) from the product, then T_k^T
+        const size_t xt_bs = (size_t)(r0 + nb2) * nb2;
+        if (k > 0) {
+            ISPA_TRY(launch_split_tf32(at(P, (size_t)r0 * D), ElemType::F32, Bt_hi, Bt_lo, nb2, r0, true, batch, s, D));
+            Tf32Opts ox;   // X_kc = T_k B_kc, T_k lower
+            ox.a_tri = 1; ox.ldc = D; ox.c_bstride = n;
+            ox.split_hi = Xt_hi; ox.split_lo = Xt_lo; ox.split_t = true; ox.split_bstride = xt_bs;
+            ISPA_TRY(launch_gemm_tf32x3(T_hi, T_lo, Bt_hi, Bt_lo, Pc + (size_t)r0 * D, nb2, r0, nb2, batch, err_flag, s,
+                                        ox));
+        }
+        if (rest > 0) {
+            ISPA_TRY(launch_split_tf32(at(P, dk), ElemType::F32, Xt_hi + (size_t)r0 * nb2, Xt_lo + (size_t)r0 * nb2, nb2,
+                                       nb2, true, batch, s, D, xt_bs));
+            Tf32Opts ob;   // B_ic -= L_ik X_kc, c <= k
+            ob.c_sub = true; ob.ldc = D; ob.c_bstride = n;
+            ISPA_TRY(launch_gemm_tf32x3(Lp_hi, Lp_lo, Xt_hi, Xt_lo, Pc + (size_t)(r0 + nb2) * D, rest, r0 + nb2, nb2,
+                                        batch, err_flag, s, ob));
+        }
+    }
+    return cudaSuccess;
+}
+
 // Solve for one batch of layers. All pointers are device pointers, one per layer.
 //   G, C, H: statistics; W: weights of type wt; dW: output (the batch's matrices contiguous,
 //   dW.p[z] = dW.p[0] + z*D*D); M, Y: D*D float scratch each; P: D*D float scratch; Yc, Pc:
@@ -372,8 +446,8 @@ cudaError_t solve_batch(const PtrBatch &G, const PtrBatch &C, const PtrBatch &H,
 
     const int nblk = D / NB;
     if (tc) {
-        // M = G + lambda I = L L^T and X = L^-1 (in P) in one launch: a cluster of CTAs per layer
-        ISPA_TRY(launch_chol_inv(G, M, P, D, lambda, batch, status, s));
+        // M = G + lambda I = L L^T and X = L^-1 (in P)
+        ISPA_TRY(chol_inv_blocked(G, M, P, split, D, lambda, batch, status, err_flag, fill_blocks, s));
         // Z = X Y, then dW = X^T Z (3xTF32; B operands are split transposed). Y^T's split is in the
         // B blocks (from Y's epilogue); Z leaves only its transposed split (in the W blocks, free
         // after Y), dW its own split (in the B blocks) for the error's dW dW^T.
