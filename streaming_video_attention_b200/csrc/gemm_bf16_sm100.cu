@@ -3,10 +3,10 @@
 // §3.3].
 //
 // A [M][K] row-major (the attention output, K-major operand), W [K][N] row-major (the
-// projection stored [D_in, D_out], MN-major operand), y [M][N] row-major. One CTA per 128x128
-// output tile, K in steps of 64 through a 4-stage TMA ring (128-byte swizzle, no multicast);
-// warp 0 TMA, warp 1 lane 0 MMA, warps 4..7 epilogue. Rows of A beyond M are zero-filled by
-// TMA and their outputs are not stored.
+// projection stored [D_in, D_out], MN-major operand), y [M][N] row-major. Persistent CTAs (one
+// per SM) walk the 128x128 output tiles, K in steps of 64 through a 4-stage TMA ring (128-byte
+// swizzle, no multicast); warp 0 TMA, warp 1 MMA into two TMEM accumulators in turn, warps 4..7
+// epilogue. Rows of A beyond M are zero-filled by TMA and their outputs are not stored.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -32,6 +32,10 @@ struct ProjParams {
     int *err_flag;
 };
 
+// Persistent: one CTA per SM takes tiles t = blockIdx.x, + gridDim.x, ... (row tiles outermost).
+// Warp 0 streams the k-steps through the stage ring (running ahead into the next tile), warp 1
+// issues the MMAs into one of two TMEM accumulators, warps 4..7 drain the other, so a tile's
+// epilogue (conversion to bf16, stores) overlaps the next tile's MMAs.
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tB, const ProjParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -41,12 +45,15 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constant__
     }
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + kBarOff);
     uint64_t *empty = full + kStages;
-    uint64_t *acc_bar = empty + kStages;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_bar + 1);
+    uint64_t *acc_full = empty + kStages;
+    uint64_t *acc_empty = acc_full + 2;
+    uint64_t *done_bar = acc_empty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int n0 = blockIdx.x * kTile, m0 = blockIdx.y * kTile;
+    const int gx = p.N / kTile, gy = (p.M + kTile - 1) / kTile;
+    const int ntiles = gx * gy;
     const int n_k = (p.K + kKStep - 1) / kKStep;
 
     if (threadIdx.x == 0) {
@@ -54,12 +61,16 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constant__
             ptx::mbar_init(&full[s], 1);
             ptx::mbar_init(&empty[s], 1);
         }
-        ptx::mbar_init(acc_bar, 1);
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&acc_full[b], 1);
+            ptx::mbar_init(&acc_empty[b], 4);
+        }
+        ptx::mbar_init(done_bar, 1);
         *abort_flag = 0;
         ptx::fence_barrier_init();
     }
     if (warp == 1) {
-        ptx::tmem_alloc(tmem_slot, 128);
+        ptx::tmem_alloc(tmem_slot, 2 * kTile);
         ptx::tmem_relinquish();
     }
     ptx::tc_fence_before();
@@ -71,70 +82,100 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constant__
     if (warp == 0) {
         const uint64_t pol_a = ptx::policy_evict_normal();
         const uint64_t pol_b = ptx::policy_evict_last();
-        int issued = -1;
+        int it = 0;
         bool ok = true;
-        for (int kt = 0; kt < n_k; ++kt) {
-            const int s = kt % kStages;
-            ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&empty[s], ((kt / kStages) & 1) ^ 1, kWaitLimitNs,
-                                                                 p.err_flag, abort_flag));
-            if (!ok) break;
-            uint8_t *base = smem + s * kStageBytes;
-            ptx::mbar_arrive_expect_tx_warp(&full[s], kStageBytes);
-            const int k0 = kt * kKStep;
-            ptx::tma_load_2d_warp(base, &tA, &full[s], k0, m0, pol_a);
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const int m0 = (t / gx) * kTile, n0 = (t % gx) * kTile;
+            for (int kt = 0; kt < n_k; ++kt, ++it) {
+                const int s = it % kStages;
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&empty[s], ((it / kStages) & 1) ^ 1,
+                                                                     kWaitLimitNs, p.err_flag, abort_flag));
+                if (!ok) break;
+                uint8_t *base = smem + s * kStageBytes;
+                ptx::mbar_arrive_expect_tx_warp(&full[s], kStageBytes);
+                const int k0 = kt * kKStep;
+                ptx::tma_load_2d_warp(base, &tA, &full[s], k0, m0, pol_a);
 #pragma unroll
-            for (int b = 0; b < 2; ++b)
-                ptx::tma_load_2d_warp(base + kABytes + b * (kKStep * 128), &tB, &full[s], n0 + b * 64, k0, pol_b);
-            issued = kt;
+                for (int b = 0; b < 2; ++b)
+                    ptx::tma_load_2d_warp(base + kABytes + b * (kKStep * 128), &tB, &full[s], n0 + b * 64, k0, pol_b);
+            }
         }
-        if (!ok)
-            for (int kt = issued - kStages + 1 > 0 ? issued - kStages + 1 : 0; kt <= issued; ++kt)
-                ptx::mbar_wait_bounded(&full[kt % kStages], (kt / kStages) & 1, kWaitLimitNs, nullptr, nullptr);
+        if (!ok) {
+            // let copies in flight land before the CTA can exit (bounded)
+            const uint64_t t0 = ptx::globaltimer_ns();
+            while (ptx::globaltimer_ns() - t0 < 2000000ull) {
+            }
+        }
     } else if (warp == 1) {
         constexpr uint32_t idesc = ptx::make_idesc_bf16(kTile, kTile, false, true);
         const uint32_t sbase = ptx::smem_u32(smem);
+        int it = 0, i = 0;
         bool ok = true;
-        for (int kt = 0; kt < n_k && ok; ++kt) {
-            const int s = kt % kStages;
-            ok = __all_sync(0xffffffffu,
-                            ptx::mbar_wait_bounded(&full[s], (kt / kStages) & 1, kWaitLimitNs, p.err_flag, abort_flag));
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++i) {
+            const int b = i & 1;
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&acc_empty[b], ((i >> 1) & 1) ^ 1, kWaitLimitNs,
+                                                                 p.err_flag, abort_flag));
             if (!ok) break;
             ptx::tc_fence_after();
-            const uint32_t a = sbase + s * kStageBytes, b = a + kABytes;
+            const uint32_t d = tmem + (uint32_t)b * kTile;
+            for (int kt = 0; kt < n_k; ++kt, ++it) {
+                const int s = it % kStages;
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&full[s], (it / kStages) & 1, kWaitLimitNs,
+                                                                     p.err_flag, abort_flag));
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const uint32_t a = sbase + s * kStageBytes, bb = a + kABytes;
 #pragma unroll
-            for (int kk = 0; kk < kKStep / 16; ++kk) {
-                const uint64_t da = ptx::make_sdesc_sw128(a + kk * 32, 16, 1024);
-                const uint64_t db = ptx::make_sdesc_sw128(b + kk * 2048, kKStep * 128, 1024);
-                ptx::umma_f16_ss_warp(tmem, da, db, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < kKStep / 16; ++kk) {
+                    const uint64_t da = ptx::make_sdesc_sw128(a + kk * 32, 16, 1024);
+                    const uint64_t db = ptx::make_sdesc_sw128(bb + kk * 2048, kKStep * 128, 1024);
+                    ptx::umma_f16_ss_warp(d, da, db, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+                }
+                ptx::umma_commit_warp(&empty[s]);
             }
-            ptx::umma_commit_warp(&empty[s]);
+            if (!ok) break;
+            ptx::umma_commit_warp(&acc_full[b]);
         }
         if (!ok) {
             if (lane == 0) *abort_flag = 1;
             __threadfence_block();
         }
-        ptx::umma_commit_warp(acc_bar);
-        ptx::mbar_wait_bounded(acc_bar, 0, kWaitLimitNs, p.err_flag, nullptr);
+        // every MMA issued has completed before tensor memory is released
+        ptx::umma_commit_warp(done_bar);
+        ptx::mbar_wait_bounded(done_bar, 0, kWaitLimitNs, p.err_flag, nullptr);
     } else if (warp >= 4) {
         const int wq = warp - 4;
         const int r = wq * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-        const bool ok = ptx::mbar_wait_bounded(acc_bar, 0, kWaitLimitNs, p.err_flag, abort_flag) && !*abort_flag;
-        if (ok) {
+        int i = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
+            const int m0 = (t / gx) * kTile, n0 = (t % gx) * kTile;
+            const int b = i & 1;
+            const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&acc_full[b], (i >> 1) & 1, kWaitLimitNs,
+                                                                           p.err_flag, abort_flag)) &&
+                            !*abort_flag;
+            if (!ok) break;
             ptx::tc_fence_after();
             const int gm = m0 + r;
             bf16 *yrow = p.y + (size_t)gm * p.N + n0;
+            const uint32_t tbuf = tmem + (uint32_t)b * kTile + lane_off;
 #pragma unroll 1
             for (int c = 0; c < kTile / 32; ++c) {
                 uint32_t v[32];
-                ptx::tmem_ld32(tmem + lane_off + c * 32, v);
+                ptx::tmem_ld32(tbuf + c * 32, v);
                 ptx::tmem_wait_ld();
+                if (c == kTile / 32 - 1) {
+                    // the accumulator is in registers: hand it back to the MMA warp
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&acc_empty[b]);
+                }
                 if (gm < p.M) {
                     uint32_t pk[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-                        pk[i] = *reinterpret_cast<uint32_t *>(&h);
+                    for (int q = 0; q < 16; ++q) {
+                        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * q]), __uint_as_float(v[2 * q + 1]));
+                        pk[q] = *reinterpret_cast<uint32_t *>(&h);
                     }
                     uint4 *dst = reinterpret_cast<uint4 *>(yrow + c * 32);
 #pragma unroll
@@ -147,7 +188,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constant__
     __syncthreads();
     if (warp == 1) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem, 128);
+        ptx::tmem_dealloc(tmem, 2 * kTile);
     }
 }
 
@@ -195,7 +236,13 @@ cudaError_t launch_gemm_bf16(const void *A, const void *W, void *y, int M, int N
     p.err_flag = err_flag;
     cudaError_t e = cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
-    gemm_bf16_kernel<<<dim3(N / kTile, (M + kTile - 1) / kTile), kThreads, kSmem, s>>>(ta, tb, p);
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int tiles = (N / kTile) * ((M + kTile - 1) / kTile);
+    gemm_bf16_kernel<<<tiles < sms ? tiles : sms, kThreads, kSmem, s>>>(ta, tb, p);
     note_launch();
     return cudaGetLastError();
 }
