@@ -26,13 +26,9 @@ namespace {
 
 constexpr int kTile = 128;
 constexpr int kKStep = 32;                      // fp32 elements per stage = one 128-byte row
-constexpr int kStages = 3;
 constexpr int kThreads = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-constexpr int kOpBytes = kTile * kKStep * 4;    // 16 KB per operand part per stage
-constexpr int kStageBytes = 4 * kOpBytes;       // A_hi, A_lo, B_hi, B_lo
-constexpr int kBarOff = kStages * kStageBytes;
-constexpr int kSmem = kBarOff + 256;   // barriers, TMEM slot and abort flag, then 8 doubles at +128
+constexpr int kOpBytes = kTile * kKStep * 4;    // 16 KB: one A part (128 rows) per stage
 
 __host__ __device__ constexpr uint32_t make_idesc_tf32(int M, int N, bool b_mn) {
     return (1u << 4)                    // D: f32
@@ -71,13 +67,27 @@ struct Tf32Params {
 
 __device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u); }
 
+// Stage layout for an output tile of 128 rows and BN columns (128 or 256): per k-step of 32, A_hi
+// and A_lo (16 KB each), then B_hi and B_lo (BN x 128 bytes each). A 256-wide tile reads each A
+// slice once for twice the columns: per SM and MMA cycle 96 instead of 128 bytes of operand reads.
+template <int BN>
+struct Tf32Cfg {
+    static constexpr int kBBytes = BN * kKStep * 4;
+    static constexpr int kStageBytes = 2 * kOpBytes + 2 * kBBytes;
+    static constexpr int kStages = BN == 128 ? 3 : 2;
+    static constexpr int kBarOff = kStages * kStageBytes;
+    static constexpr int kSmem = kBarOff + 256;   // barriers, TMEM slot, abort flag; 16 doubles at +128
+};
+static_assert(Tf32Cfg<128>::kSmem <= 232448 && Tf32Cfg<256>::kSmem <= 232448, "shared memory budget");
+
 // Output tiles in the order the CTAs take them (t = blockIdx.x, + gridDim.x, ...): batch entries
 // outermost, so that the tiles in flight at once share one layer's operands in L2; within a
 // layer tile rows with the longest K range first when A is triangular, then columns.
 struct TileId {
     int z, m, n;
-    bool skip;   // above the diagonal of a symmetric product
+    bool skip;   // wholly above the diagonal of a symmetric product
 };
+template <int BN>
 __device__ __forceinline__ TileId tile_of(int t, int gx, int gy, int a_tri, int sym) {
     const int per_layer = gx * gy;
     TileId id;
@@ -86,40 +96,44 @@ __device__ __forceinline__ TileId tile_of(int t, int gx, int gy, int a_tri, int 
     const int mr = rem / gx;
     id.n = rem - mr * gx;
     id.m = a_tri == 1 ? gy - 1 - mr : mr;
-    id.skip = sym && id.n > id.m;
+    id.skip = sym && id.n * (BN / kTile) > id.m;
     return id;
 }
 
 // Persistent: one CTA per SM walks its share of the output tiles. Warp 0 streams the operand
 // k-steps through the stage ring (running ahead into the next tile), warp 1 issues the MMAs
 // into one of two TMEM accumulators, warps 4..7 drain the other: the epilogue of a tile (its
-// dots, splits and stores) overlaps the MMAs of the next.
+// dots, splits and stores) overlaps the MMAs of the next. Trace partials are kept per 128 x 128
+// sub-tile whatever BN is.
+template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constant__ CUtensorMap tAl,
                    const __grid_constant__ CUtensorMap tBh, const __grid_constant__ CUtensorMap tBl,
                    const Tf32Params p) {
+    using Cfg = Tf32Cfg<BN>;
+    constexpr int kSub = BN / kTile;   // 128-column sub-tiles per tile
     extern __shared__ __align__(1024) uint8_t smem[];
     if (ptx::smem_u32(smem) & 1023u) {
         if (threadIdx.x == 0) atomicCAS(p.err_flag, 0, ISPA_ERR_UNSUPPORTED);
         return;
     }
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kBarOff);
-    uint64_t *empty = full + kStages;
-    uint64_t *acc_full = empty + kStages;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOff);
+    uint64_t *empty = full + Cfg::kStages;
+    uint64_t *acc_full = empty + Cfg::kStages;
     uint64_t *acc_empty = acc_full + 2;
     uint64_t *done_bar = acc_empty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    double *red = reinterpret_cast<double *>(smem + kBarOff + 128);
+    double *red = reinterpret_cast<double *>(smem + Cfg::kBarOff + 128);   // [dot][sub][warp]
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int gx = p.N / kTile, gy = p.M / kTile;
+    const int gx = p.N / BN, gy = p.M / kTile, gx128 = p.N / kTile;
     const int ntiles = gx * gy * p.batch;
     const int n_kall = (p.K + kKStep - 1) / kKStep;
-    const uint32_t stage_tx = (2 + p.a_lo + p.b_lo) * kOpBytes;
+    const uint32_t stage_tx = (1 + p.a_lo) * kOpBytes + (1 + p.b_lo) * Cfg::kBBytes;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < Cfg::kStages; ++s) {
             ptx::mbar_init(&full[s], 1);
             ptx::mbar_init(&empty[s], 1);
         }
@@ -132,7 +146,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
         ptx::fence_barrier_init();
     }
     if (warp == 1) {
-        ptx::tmem_alloc(tmem_slot, 256);
+        ptx::tmem_alloc(tmem_slot, 2 * BN);
         ptx::tmem_relinquish();
     }
     ptx::tc_fence_before();
@@ -154,23 +168,23 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
         int it = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-            const TileId id = tile_of(t, gx, gy, p.a_tri, p.sym);
+            const TileId id = tile_of<BN>(t, gx, gy, p.a_tri, p.sym);
             if (id.skip) continue;
-            const int m0 = id.m * kTile, n0 = id.n * kTile;
+            const int m0 = id.m * kTile, n0 = id.n * BN;
             int kt0, n_k;
             k_range(m0, kt0, n_k);
             for (int kt = 0; kt < n_k; ++kt, ++it) {
-                const int s = it % kStages;
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&empty[s], ((it / kStages) & 1) ^ 1, kWaitLimitNs,
-                                                                     p.err_flag, abort_flag));
+                const int s = it % Cfg::kStages;
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&empty[s], ((it / Cfg::kStages) & 1) ^ 1,
+                                                                     kWaitLimitNs, p.err_flag, abort_flag));
                 if (!ok) break;
-                uint8_t *base = smem + s * kStageBytes;
+                uint8_t *base = smem + s * Cfg::kStageBytes;
                 ptx::mbar_arrive_expect_tx_warp(&full[s], stage_tx);
                 const int k0 = (kt0 + kt) * kKStep;
                 ptx::tma_load_3d_warp(base, &tAh, &full[s], k0, m0, id.z, pol);
                 if (p.a_lo) ptx::tma_load_3d_warp(base + kOpBytes, &tAl, &full[s], k0, m0, id.z, pol);
                 ptx::tma_load_3d_warp(base + 2 * kOpBytes, &tBh, &full[s], k0, n0, id.z, pol);
-                if (p.b_lo) ptx::tma_load_3d_warp(base + 3 * kOpBytes, &tBl, &full[s], k0, n0, id.z, pol);
+                if (p.b_lo) ptx::tma_load_3d_warp(base + 2 * kOpBytes + Cfg::kBBytes, &tBl, &full[s], k0, n0, id.z, pol);
             }
         }
         if (!ok) {
@@ -180,12 +194,12 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
             }
         }
     } else if (warp == 1) {
-        constexpr uint32_t idesc = make_idesc_tf32(kTile, kTile, false);
+        constexpr uint32_t idesc = make_idesc_tf32(kTile, BN, false);
         const uint32_t sbase = ptx::smem_u32(smem);
         int it = 0, i = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-            const TileId id = tile_of(t, gx, gy, p.a_tri, p.sym);
+            const TileId id = tile_of<BN>(t, gx, gy, p.a_tri, p.sym);
             if (id.skip) continue;
             int kt0, n_k;
             k_range(id.m * kTile, kt0, n_k);
@@ -194,14 +208,15 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
                                                                  p.err_flag, abort_flag));
             if (!ok) break;
             ptx::tc_fence_after();
-            const uint32_t d = tmem + (uint32_t)b * kTile;
+            const uint32_t d = tmem + (uint32_t)b * BN;
             for (int kt = 0; kt < n_k; ++kt, ++it) {
-                const int s = it % kStages;
-                ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&full[s], (it / kStages) & 1, kWaitLimitNs,
+                const int s = it % Cfg::kStages;
+                ok = __all_sync(0xffffffffu, ptx::mbar_wait_bounded(&full[s], (it / Cfg::kStages) & 1, kWaitLimitNs,
                                                                      p.err_flag, abort_flag));
                 if (!ok) break;
                 ptx::tc_fence_after();
-                const uint32_t ah = sbase + s * kStageBytes, al = ah + kOpBytes, bh = al + kOpBytes, bl = bh + kOpBytes;
+                const uint32_t ah = sbase + s * Cfg::kStageBytes, al = ah + kOpBytes, bh = al + kOpBytes,
+                               bl = bh + Cfg::kBBytes;
 #pragma unroll
                 for (int kk = 0; kk < kKStep / 8; ++kk) {
                     const uint64_t dah = ptx::make_sdesc_sw128(ah + kk * 32, 16, 1024);
@@ -239,15 +254,17 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
         const bool has_parts = p.has_dot || p.has_dot2;
         int i = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-            const TileId id = tile_of(t, gx, gy, p.a_tri, p.sym);
-            const int z = id.z, m0 = id.m * kTile, n0 = id.n * kTile;
-            const size_t part_idx = ((size_t)z * gy + id.m) * gx + id.n;
+            const TileId id = tile_of<BN>(t, gx, gy, p.a_tri, p.sym);
+            const int z = id.z, m0 = id.m * kTile, n0 = id.n * BN;
+            // partial of 128 x 128 sub-tile u of this tile
+            const size_t part0 = ((size_t)z * gy + id.m) * gx128 + (size_t)id.n * kSub;
             if (id.skip) {
-                // the mirror tile (n0, m0) accounts for this one
-                if (wq == 0 && lane == 0) {
-                    if (p.has_dot) p.dot_out[part_idx] = 0.0;
-                    if (p.has_dot2) p.dot_out2[part_idx] = 0.0;
-                }
+                // the mirror tiles account for these
+                if (wq == 0 && lane == 0)
+                    for (int u = 0; u < kSub; ++u) {
+                        if (p.has_dot) p.dot_out[part0 + u] = 0.0;
+                        if (p.has_dot2) p.dot_out2[part0 + u] = 0.0;
+                    }
                 continue;
             }
             const int b = i & 1;
@@ -256,26 +273,33 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
                             !*abort_flag;
             if (!ok) break;
             ptx::tc_fence_after();
-            // the mirror's share of a symmetric product's off-diagonal tile
-            const bool mirror = p.sym && m0 != n0;
-            double part = 0.0, part2 = 0.0;
+            double part[kSub], part2[kSub];
+#pragma unroll
+            for (int u = 0; u < kSub; ++u) part[u] = part2[u] = 0.0;
             const int gm = m0 + r;
             float *crow = p.C + (size_t)z * p.c_bstride + (size_t)gm * p.ldc + n0;
             const size_t xrow = (size_t)gm * p.N + n0;
             const void *xz = p.has_dot ? p.dot_x.p[z] : nullptr;
             const float *x2z = p.has_dot2 ? static_cast<const float *>(p.dot_x2.p[z]) : nullptr;
-            const uint32_t tbuf = tmem + (uint32_t)b * kTile + lane_off;
+            const uint32_t tbuf = tmem + (uint32_t)b * BN + lane_off;
 #pragma unroll 1
-            for (int c = 0; c < kTile / 32; ++c) {
+            for (int c = 0; c < BN / 32; ++c) {
                 uint32_t v[32];
                 ptx::tmem_ld32(tbuf + c * 32, v);
                 ptx::tmem_wait_ld();
-                if (c == kTile / 32 - 1) {
+                if (c == BN / 32 - 1) {
                     // the accumulator is in registers: hand it back to the MMA warp
                     ptx::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(&acc_empty[b]);
                 }
+                const int u = c / (kTile / 32);              // sub-tile of this chunk
+                const int nt = id.n * kSub + u;              // its 128-column tile index
+                // a symmetric product keeps only sub-tiles on or below the diagonal; an
+                // off-diagonal one also takes its mirror's share of the dots
+                if (p.sym && nt > id.m) continue;
+                const bool mirror = p.sym && nt != id.m;
+                double pa = 0.0, pb = 0.0;
                 if (p.has_dot) {
                     // products of two floats are exact in double; summed in a fixed order. The row's
                     // 32 values are read as 16-byte vectors (N is a multiple of 128).
@@ -283,52 +307,58 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
                     if (p.dot_x_bf16) {
                         const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const bf16 *>(xz) + xrow + c * 32);
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const uint4 w = src[u];
-                            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                        for (int w = 0; w < 4; ++w) {
+                            const uint4 q4 = src[w];
+                            const uint32_t ww[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
-                                x[8 * u + 2 * e] = __uint_as_float(ww[e] << 16);
-                                x[8 * u + 2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
+                                x[8 * w + 2 * e] = __uint_as_float(ww[e] << 16);
+                                x[8 * w + 2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
                             }
                         }
                     } else {
                         const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(xz) + xrow + c * 32);
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) {
-                            const float4 w = src[u];
-                            x[4 * u] = w.x; x[4 * u + 1] = w.y; x[4 * u + 2] = w.z; x[4 * u + 3] = w.w;
+                        for (int w = 0; w < 8; ++w) {
+                            const float4 q4 = src[w];
+                            x[4 * w] = q4.x; x[4 * w + 1] = q4.y; x[4 * w + 2] = q4.z; x[4 * w + 3] = q4.w;
                         }
                     }
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) part += (double)__uint_as_float(v[q]) * (double)x[q];
+                    for (int q = 0; q < 32; ++q) pa += (double)__uint_as_float(v[q]) * (double)x[q];
                     if (mirror) {
                         // X[n0 + c*32 + q][gm]: the warp's 32 rows read one 128-byte run per q
                         const float *xt = static_cast<const float *>(xz) + (size_t)(n0 + c * 32) * p.N + gm;
 #pragma unroll
                         for (int q = 0; q < 32; ++q) x[q] = xt[(size_t)q * p.N];
 #pragma unroll
-                        for (int q = 0; q < 32; ++q) part += (double)__uint_as_float(v[q]) * (double)x[q];
+                        for (int q = 0; q < 32; ++q) pa += (double)__uint_as_float(v[q]) * (double)x[q];
                     }
                 }
                 if (p.has_dot2) {
                     float x[32];
                     const float4 *src = reinterpret_cast<const float4 *>(x2z + xrow + c * 32);
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const float4 w = src[u];
-                        x[4 * u] = w.x; x[4 * u + 1] = w.y; x[4 * u + 2] = w.z; x[4 * u + 3] = w.w;
+                    for (int w = 0; w < 8; ++w) {
+                        const float4 q4 = src[w];
+                        x[4 * w] = q4.x; x[4 * w + 1] = q4.y; x[4 * w + 2] = q4.z; x[4 * w + 3] = q4.w;
                     }
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) part2 += (double)__uint_as_float(v[q]) * (double)x[q];
+                    for (int q = 0; q < 32; ++q) pb += (double)__uint_as_float(v[q]) * (double)x[q];
                     if (mirror) {
                         const float *xt = x2z + (size_t)(n0 + c * 32) * p.N + gm;
 #pragma unroll
                         for (int q = 0; q < 32; ++q) x[q] = xt[(size_t)q * p.N];
 #pragma unroll
-                        for (int q = 0; q < 32; ++q) part2 += (double)__uint_as_float(v[q]) * (double)x[q];
+                        for (int q = 0; q < 32; ++q) pb += (double)__uint_as_float(v[q]) * (double)x[q];
                     }
                 }
+#pragma unroll
+                for (int w = 0; w < kSub; ++w)
+                    if (w == u) {
+                        part[w] += pa;
+                        part2[w] += pb;
+                    }
                 if (p.split_hi) {
                     if (p.split_t) {
                         // column n0 + c*32 + q of C is row n of the transposed split: the warp's
@@ -347,10 +377,10 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
                         for (int q = 0; q < 32; q += 4) {
                             float h[4], l[4];
 #pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                const float x = __uint_as_float(v[q + u]);
-                                h[u] = tf32_hi(x);
-                                l[u] = x - h[u];
+                            for (int e = 0; e < 4; ++e) {
+                                const float x = __uint_as_float(v[q + e]);
+                                h[e] = tf32_hi(x);
+                                l[e] = x - h[e];
                             }
                             *reinterpret_cast<float4 *>(hrow + q) = make_float4(h[0], h[1], h[2], h[3]);
                             *reinterpret_cast<float4 *>(lrow + q) = make_float4(l[0], l[1], l[2], l[3]);
@@ -361,13 +391,13 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
                     if (p.c_sub) {
                         float4 old[8];
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) old[u] = *reinterpret_cast<const float4 *>(crow + c * 32 + 4 * u);
+                        for (int w = 0; w < 8; ++w) old[w] = *reinterpret_cast<const float4 *>(crow + c * 32 + 4 * w);
 #pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            *reinterpret_cast<float4 *>(crow + c * 32 + 4 * u) =
-                                make_float4(old[u].x - __uint_as_float(v[4 * u]), old[u].y - __uint_as_float(v[4 * u + 1]),
-                                            old[u].z - __uint_as_float(v[4 * u + 2]),
-                                            old[u].w - __uint_as_float(v[4 * u + 3]));
+                        for (int w = 0; w < 8; ++w)
+                            *reinterpret_cast<float4 *>(crow + c * 32 + 4 * w) =
+                                make_float4(old[w].x - __uint_as_float(v[4 * w]), old[w].y - __uint_as_float(v[4 * w + 1]),
+                                            old[w].z - __uint_as_float(v[4 * w + 2]),
+                                            old[w].w - __uint_as_float(v[4 * w + 3]));
                     } else {
 #pragma unroll
                         for (int q = 0; q < 32; q += 4)
@@ -378,20 +408,26 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
                 }
             }
             if (has_parts) {
-                // the tile's partials: warp sums, then warp 4 adds the four warps' sums in order
-                for (int o = 16; o > 0; o >>= 1) {
-                    part += __shfl_down_sync(0xffffffffu, part, o);
-                    part2 += __shfl_down_sync(0xffffffffu, part2, o);
-                }
-                if (lane == 0) {
-                    red[wq] = part;
-                    red[4 + wq] = part2;
+                // each sub-tile's partials: warp sums, then warp 4 adds the four warps' sums in order
+                // (a sub-tile above the diagonal of a symmetric product sums to 0)
+#pragma unroll
+                for (int u = 0; u < kSub; ++u) {
+                    for (int o = 16; o > 0; o >>= 1) {
+                        part[u] += __shfl_down_sync(0xffffffffu, part[u], o);
+                        part2[u] += __shfl_down_sync(0xffffffffu, part2[u], o);
+                    }
+                    if (lane == 0) {
+                        red[(0 * kSub + u) * 4 + wq] = part[u];
+                        red[(1 * kSub + u) * 4 + wq] = part2[u];
+                    }
                 }
                 asm volatile("bar.sync 1, 128;" ::: "memory");
-                if (wq == 0 && lane == 0) {
-                    if (p.has_dot) p.dot_out[part_idx] = ((red[0] + red[1]) + red[2]) + red[3];
-                    if (p.has_dot2) p.dot_out2[part_idx] = ((red[4] + red[5]) + red[6]) + red[7];
-                }
+                if (wq == 0 && lane == 0)
+                    for (int u = 0; u < kSub; ++u) {
+                        const double *r1 = red + (0 * kSub + u) * 4, *r2 = red + (1 * kSub + u) * 4;
+                        if (p.has_dot) p.dot_out[part0 + u] = ((r1[0] + r1[1]) + r1[2]) + r1[3];
+                        if (p.has_dot2) p.dot_out2[part0 + u] = ((r2[0] + r2[1]) + r2[2]) + r2[3];
+                    }
                 asm volatile("bar.sync 1, 128;" ::: "memory");
             }
             ++i;
@@ -401,7 +437,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tAh, const __grid_constan
     __syncthreads();
     if (warp == 1) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem, 256);
+        ptx::tmem_dealloc(tmem, 2 * BN);
     }
 }
 
@@ -525,9 +561,11 @@ cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh
                                int N, int K, int batch, int *err_flag, cudaStream_t s, const Tf32Opts &o) {
     if (M % kTile || N % kTile || K % kKStep || batch <= 0) return cudaErrorInvalidValue;
     if (o.sym && (M != N || o.dot_x_bf16 || o.a_tri)) return cudaErrorInvalidValue;
+    // 256-wide tiles where N allows (the A slices are read once for twice the columns)
+    const int bn = N % 256 == 0 ? 256 : 128;
     CUtensorMap ah, al, bh, bl;
     if (!make_map(&ah, Ah, batch, M, K, kTile) || !make_map(&al, Al ? Al : Ah, batch, M, K, kTile) ||
-        !make_map(&bh, Bh, batch, N, K, kTile) || !make_map(&bl, Bl ? Bl : Bh, batch, N, K, kTile))
+        !make_map(&bh, Bh, batch, N, K, bn) || !make_map(&bl, Bl ? Bl : Bh, batch, N, K, bn))
         return cudaErrorInvalidValue;
     Tf32Params p;
     p.C = C; p.M = M; p.N = N; p.K = K;
@@ -554,16 +592,24 @@ cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh
     p.write_c = (o.write_c || !(p.has_dot || p.has_dot2 || p.split_hi)) ? 1 : 0;
     p.err_flag = err_flag;
     p.batch = batch;
-    cudaError_t e = cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
-    e = cudaGetDevice(&dev);
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    const long long tiles = (long long)(M / kTile) * (N / kTile) * batch;
+    const long long tiles = (long long)(M / kTile) * (N / bn) * batch;
     const int grid = (int)(tiles < sms ? tiles : sms);
-    gemm_tf32x3_kernel<<<grid, kThreads, kSmem, s>>>(ah, al, bh, bl, p);
+    if (bn == 256) {
+        e = cudaFuncSetAttribute(gemm_tf32x3_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Tf32Cfg<256>::kSmem);
+        if (e != cudaSuccess) return e;
+        gemm_tf32x3_kernel<256><<<grid, kThreads, Tf32Cfg<256>::kSmem, s>>>(ah, al, bh, bl, p);
+    } else {
+        e = cudaFuncSetAttribute(gemm_tf32x3_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Tf32Cfg<128>::kSmem);
+        if (e != cudaSuccess) return e;
+        gemm_tf32x3_kernel<128><<<grid, kThreads, Tf32Cfg<128>::kSmem, s>>>(ah, al, bh, bl, p);
+    }
     note_launch();
     return cudaGetLastError();
 }
