@@ -561,8 +561,14 @@ cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh
                                int N, int K, int batch, int *err_flag, cudaStream_t s, const Tf32Opts &o) {
     if (M % kTile || N % kTile || K % kKStep || batch <= 0) return cudaErrorInvalidValue;
     if (o.sym && (M != N || o.dot_x_bf16 || o.a_tri)) return cudaErrorInvalidValue;
-    // 256-wide tiles where N allows (the A slices are read once for twice the columns)
-    const int bn = N % 256 == 0 ? 256 : 128;
+    // 256-wide tiles where N allows and they still give every SM two tiles or more (the A slices
+    // are read once for twice the columns; the small products keep 128 for parallelism)
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int bn = (N % 256 == 0 && (long long)(M / kTile) * (N / 256) * batch >= 2LL * sms) ? 256 : 128;
     CUtensorMap ah, al, bh, bl;
     if (!make_map(&ah, Ah, batch, M, K, kTile) || !make_map(&al, Al ? Al : Ah, batch, M, K, kTile) ||
         !make_map(&bh, Bh, batch, N, K, bn) || !make_map(&bl, Bl ? Bl : Bh, batch, N, K, bn))
@@ -592,11 +598,6 @@ cudaError_t launch_gemm_tf32x3(const float *Ah, const float *Al, const float *Bh
     p.write_c = (o.write_c || !(p.has_dot || p.has_dot2 || p.split_hi)) ? 1 : 0;
     p.err_flag = err_flag;
     p.batch = batch;
-    int dev = 0, sms = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
     const long long tiles = (long long)(M / kTile) * (N / bn) * batch;
     const int grid = (int)(tiles < sms ? tiles : sms);
     if (bn == 256) {
