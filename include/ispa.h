@@ -194,6 +194,10 @@ int ispa_stats_reset(const ispa_stats *stats, ispa_stream_t stream);
  *   layer_status: device [n_layers] int, ISPA_OK or ISPA_ERR_NOT_SPD per layer (dW and
  *     eps of such a layer are NaN).
  *   ws: ispa_workspace_bytes(NULL, n_layers, D) bytes.
+ * D must be a multiple of 64. With D a multiple of 128 every product runs on the tensor cores
+ * (float32-accurate, 3xTF32) and the factorisation is blocked (512, 256 or 128 columns), the
+ * diagonal blocks factored and inverted by thread-block clusters of 8 CTAs; otherwise the CUDA
+ * cores do it all.
  * The layers run as up to three concurrent sub-batches, each in its own part of ws: the call
  * forks from `stream` onto two streams the library creates on its first call on a device
  * (driver objects, no device memory; make that first call before any stream capture) and joins
