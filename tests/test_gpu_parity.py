@@ -202,6 +202,37 @@ def test_solve_absorb_matches_oracle(dtype, D, L):
     assert ispa.ispa_select_layers(eps_gpu, 1)[0] == oracle.select_layers(eps_ref, 1)[0]
 
 
+def test_solve_more_layers_than_one_batch():
+    """50 layers at D = 128: the call runs them as a batch of 48 and one of 2 (each as concurrent
+    sub-batches) reusing one workspace; every layer against the oracle on its own statistics."""
+    D, L, lam = 128, 50, 1e-2
+    stats_np = [_oracle_stats_for("bf16", 300 + l, 512, D, planted=(l % 3 == 0)) for l in range(L)]
+    W_np = [synth.normal_tensor(400 + l, (33,), (D, D), "bf16", std=1 / math.sqrt(D)) for l in range(L)]
+    stats = []
+    for st_np in stats_np:
+        st = ispa.Stats(D)
+        st.G.copy_(torch.from_numpy(st_np["G"].astype(np.float32)))
+        st.C.copy_(torch.from_numpy(st_np["C"].astype(np.float32)))
+        st.H.copy_(torch.from_numpy(st_np["H"].astype(np.float32)))
+        stats.append(st)
+    Ws = [to_device(w, "bf16") for w in W_np]
+    dW = torch.full((L, D, D), float("nan"), device="cuda")
+    eps = torch.full((L,), float("nan"), device="cuda")
+    status = torch.full((L,), 7, dtype=torch.int32, device="cuda")
+    ws = ispa.alloc_workspace(ispa.workspace_bytes(None, L, D))
+    ispa.ispa_solve_absorb(stats, Ws, ispa.ISPA_BF16, lam, dW, eps, None, None, status, ws)
+    torch.cuda.synchronize()
+    assert status.tolist() == [0] * L
+    for l in range(L):
+        G = stats_np[l]["G"].astype(np.float32).astype(np.float64)
+        C = stats_np[l]["C"].astype(np.float32).astype(np.float64)
+        H = stats_np[l]["H"].astype(np.float32).astype(np.float64)
+        dW_ref = oracle.absorb_solve(G, C, W_np[l], lam)
+        assert rel_fro(to_numpy(dW[l]), dW_ref) < 1e-3, l
+        e = oracle.reconstruction_error(G, C, H, W_np[l], dW_ref)
+        assert abs(float(eps[l]) - e["eps"]) <= 1e-3 * abs(e["eps"]) + 4e-6, (l, float(eps[l]), e["eps"])
+
+
 @pytest.mark.parametrize("dtype,D,L", [("fp32", 128, 2), ("bf16", 256, 3), ("bf16", 1536, 2), ("bf16", 192, 2)])
 def test_absorb_error_of_a_given_dW_matches_oracle(dtype, D, L):
     """ispa_absorb_error: eps of a given dW on given statistics (the live error of the
