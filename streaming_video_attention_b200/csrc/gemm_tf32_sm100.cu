@@ -1,6 +1,7 @@
-// Float32-accurate batched GEMM on the sm_100a tensor cores (3xTF32), for the absorb solve's
-// D x D products [ISPA §3.2, §3.3]: Y = C W, the two products with L^-1, and the Gram products
-// W W^T and dW dW^T whose dots with G and H give the error traces.
+// Float32-accurate batched GEMM on the sm_100a tensor cores (3xTF32), for every product of the
+// absorb solve [ISPA §3.2, §3.3]: Y = C W; the blocked factorisation's panels, trailing updates
+// and rows of L^-1; the two products with L^-1; the Gram products W W^T and dW dW^T whose dots
+// with G and H give the error traces.
 //
 // Each float32 operand X is split once into X_hi = X rounded to TF32 (11 significant bits)
 // and X_lo = X - X_hi (exact in float32; the tensor core keeps its leading 11 bits). The
@@ -11,10 +12,11 @@
 //
 // Layouts: both MMA operands are K-major (32-bit K-major tiles with the 128-byte swizzle):
 // A split as [batch][M][K], B split *and transposed* as [batch][N][K] (the split kernel for B
-// writes B^T), so C = A B = A (B^T)^T. C [batch][M][N] row-major float32, overwritten. The
-// split operands are contiguous batches in the workspace, so one 3-D tensor map covers all
-// layers. Persistent CTAs (one per SM) walk 128 x 128 output tiles; K in steps of 32 through
-// a 3-stage ring; warp 0 TMA, warp 1 MMA (kind::tf32, K = 8 per instruction) into two TMEM
+// writes B^T), so C = A B = A (B^T)^T. C float32 row-major with given row and batch strides,
+// overwritten or subtracted from. The split operands are contiguous batches in the workspace,
+// so one 3-D tensor map covers all layers. Persistent CTAs (one per SM) walk 128 x 256 output
+// tiles (128 x 128 where N or the tile count calls for it); K in steps of 32 through a 2- or
+// 3-stage ring; warp 0 TMA, warp 1 MMA (kind::tf32, K = 8 per instruction) into two TMEM
 // accumulators in turn, warps 4..7 epilogue.
 #include <cuda.h>
 

@@ -2,8 +2,12 @@
 // [ISPA §3.1 step 2, §3.2, §3.3, §4.1 "Eq. 5"].
 //
 //   with D a multiple of 128:
-//   M = G + lambda I = L L^T, X = L^-1        one launch, a thread-block cluster per layer
-//                                             (chol_inv_sm100.cu)
+//   Y = C W                                   3xTF32 product (gemm_tf32_sm100.cu)
+//   M = G + lambda I = L L^T, X = L^-1        blocked by 512 (256, 128) columns: each diagonal
+//                                             block factored and inverted by a thread-block
+//                                             cluster per layer (chol_inv_sm100.cu); the panel,
+//                                             the trailing update and the rows of X as 3xTF32
+//                                             products (chol_inv_blocked)
 //   dW = X^T X (C W)                          Z = X (C W), dW = X^T Z on the tensor cores
 //                                             (3xTF32, the zero triangle of X skipped)
 //   otherwise:
@@ -17,10 +21,11 @@
 //                                             epilogues; otherwise GEMMs G dW, H W, G W, then
 //                                             dot_partials
 //
-// Block size nb = 64 (D must be a multiple of 64). Each 64 x 64 diagonal block is factored
-// (potrf_diag) and each panel below it solved (trsm_panel) by CTAs whose threads hold one row
-// of the block in registers; everything of order D^3 runs in batched GEMMs. A non-positive
-// pivot marks the layer ISPA_ERR_NOT_SPD and turns its results to NaN; nothing traps.
+// On the CUDA-core path the block size is 64 (D must be a multiple of 64): each 64 x 64
+// diagonal block is factored (potrf_diag) and each panel below it solved (trsm_panel) by CTAs
+// whose threads hold one row of the block in registers, and everything of order D^3 runs in
+// batched GEMMs. A non-positive pivot marks the layer ISPA_ERR_NOT_SPD and turns its results to
+// NaN; nothing traps.
 #include "common.cuh"
 
 namespace ispa {
