@@ -1,5 +1,7 @@
-// Cholesky factor and explicit inverse of M = G + lambda I in one launch, one thread-block
-// cluster of kCL CTAs per layer [ISPA §3.2: the ridge system (G + lambda I) dW = C W].
+// Cholesky factor and explicit inverse of an n x n symmetric positive definite matrix in one
+// launch, one thread-block cluster of kCL CTAs per layer [ISPA §3.2: the ridge system
+// (G + lambda I) dW = C W]: either the whole M = G + lambda I (n = D), or one diagonal block of the
+// blocked factorisation in solve.cu, whose inverse is the matching diagonal block of L^-1.
 //
 // The cluster walks the 64-wide block columns k of M (right-looking); per step two phases, each
 // closed by a cluster barrier:
@@ -16,7 +18,7 @@
 // load that may see another CTA's write bypasses L1 (cp.async.cg, ld.global.cg) and the
 // barriers are release/acquire at cluster scope after a device-scope fence.
 //
-// The whole chain is 2 * D/64 cluster barriers and no kernel boundaries; the layers' clusters
+// The whole chain is 2 * n/64 cluster barriers and no kernel boundaries; the layers' clusters
 // are independent. A non-positive pivot marks the layer ISPA_ERR_NOT_SPD; the NaN it produces
 // runs through L and X (no trap, no early exit: every CTA takes every barrier).
 #include "common.cuh"
